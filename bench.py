@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the QuantWM 2-bit KV-cache hot path on B200.
+
+One step = one pass of the whole hot path for one new frame of the 480p
+93-frame layer (40 heads x 128, 1560 tokens per latent frame, cache of 24
+latent frames = 37 440 tokens, C = 256, G = 32, M = 4, r = 8):
+
+    qwm_update_query_stats(Q_f, refresh)   query second moment + basis refresh
+    qwm_append_kv(K_f, V_f)                QSAC + INT2 + PSAC keys, INT2 values
+    qwm_attention(Q_f)                     1560 queries over the full packed cache
+
+The cache is filled with the 24 frames before timing; each timed step
+re-appends the newest frame slot (the host length is rewound by one frame), so
+every step attends over the full 37 440-token cache.  Step inputs rotate over a
+pool of frames resident in HBM; together with the 161 MB packed cache every
+step touches more than the 126 MB L2.
+
+Prints one JSON line (rank 0).  `value` is query tokens per second for the
+whole job (all ranks); each rank runs its own replica (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import qwm_synth as syn  # noqa: E402
+
+METRIC = "quantized-KV attention query-tok/s & append GB/s; % of roofline"
+UNIT = "query-tok/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+def dev_bf16(a: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+class Workload:
+    def __init__(self, cfg: syn.LayerConfig, device, extra_versions: int, pool: int = 4):
+        import bit_kv_cache_23_b200 as q
+
+        self.cfg = cfg
+        self.device = device
+        c = cfg
+        self.cache = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand,
+                                    c.rank, c.total_tokens,
+                                    max_versions=c.frames // c.refresh_every + extra_versions + 4,
+                                    device=device)
+        src = syn.FrameSource(c)
+        self.src = src
+        self.pool = []
+        self.host_pool = []
+        for f in range(c.frames):
+            Q, K, V = src.frame(f)
+            Qd, Kd, Vd = dev_bf16(Q, device), dev_bf16(K, device), dev_bf16(V, device)
+            if f == 0:
+                self.cache.build_centroids(Kd, Vd, iters=c.kmeans_iters)
+            self.cache.update_query_stats(Qd, refresh_basis=(f % c.refresh_every) == 0)
+            self.cache.append_kv(Kd, Vd)
+            if f >= c.frames - pool:
+                self.pool.append((Qd, Kd, Vd))
+                self.host_pool.append(tuple(torch.from_numpy(a.view(np.int16)).pin_memory()
+                                            for a in (Q, K, V)))
+        torch.cuda.synchronize(device)
+        self.t_last = self.cache.len - c.tokens_per_frame
+        self.O = torch.empty_like(self.pool[0][0])
+        self.nstep = 0
+
+    def step(self, i: int, ev=None):
+        """One hot-path pass; `ev` = 4 events to record around the three calls."""
+        Qd, Kd, Vd = self.pool[i % len(self.pool)]
+        c = self.cache
+        c.c.len = self.t_last
+        if ev:
+            ev[0].record()
+        c.update_query_stats(Qd, refresh_basis=(self.nstep % self.cfg.refresh_every) == 0)
+        if ev:
+            ev[1].record()
+        c.append_kv(Kd, Vd)
+        if ev:
+            ev[2].record()
+        c.attention(Qd, self.O)
+        if ev:
+            ev[3].record()
+        self.nstep += 1
+
+    def step_host(self, i: int, bufs):
+        """The same pass through the public API from pinned host buffers."""
+        Qh, Kh, Vh = self.host_pool[i % len(self.host_pool)]
+        Qd, Kd, Vd, Oh = bufs
+        Qd.copy_(Qh, non_blocking=True)
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        c = self.cache
+        c.c.len = self.t_last
+        q16 = Qd.view(torch.bfloat16)
+        c.update_query_stats(q16, refresh_basis=(self.nstep % self.cfg.refresh_every) == 0)
+        c.append_kv(Kd.view(torch.bfloat16), Vd.view(torch.bfloat16))
+        c.attention(q16, self.O)
+        Oh.copy_(self.O.view(torch.int16), non_blocking=True)
+        self.nstep += 1
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_throughput(cfg: syn.LayerConfig, cache=None, budget_s: float = 12.0):
+    """The CPU oracle, as it stands, on a bounded sample of one step of the
+    workload; returns query-tokens/s extrapolated to the full step and a note."""
+    import oracle
+
+    c = cfg
+    src = syn.FrameSource(c)
+    f = c.frames - 1
+    Q, K, V = src.frame(f)
+    oc = oracle.OracleCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank,
+                            c.total_tokens)
+    if cache is not None:
+        torch.cuda.synchronize()
+        for name in ("k_codes", "k_params", "k_idx", "k_coef", "k_cscale", "v_codes",
+                     "v_params", "v_idx"):
+            v = cache.view(name)[:, : c.total_tokens].cpu().numpy()
+            dst = getattr(oc, name)
+            dst[:] = v.view(dst.dtype) if v.dtype.itemsize == dst.dtype.itemsize else v
+        oc.CK = cache.view("cent_k").cpu().numpy().view(np.uint16).copy()
+        oc.CV = cache.view("cent_v").cpu().numpy().view(np.uint16).copy()
+        oc.tok_ver[:] = cache.view("tokver")[: c.total_tokens].cpu().numpy().view(np.uint16)
+        nver = int(oc.tok_ver.max()) + 1
+        oc.U = list(cache.view("basis")[:nver].cpu().numpy())
+        oc.s = cache.view("sens").cpu().numpy().copy()
+        oc.w = cache.view("wgroup").cpu().numpy().copy()
+        oc.len = c.total_tokens
+    else:
+        oc.build_centroids(K[: max(c.n_centroids, 64)], V[: max(c.n_centroids, 64)], iters=1)
+        oc.len = c.total_tokens
+    # stats on a sample of query rows
+    nq_s = 16
+    t0 = time.perf_counter()
+    Msum = np.zeros((c.heads, c.head_dim, c.head_dim))
+    for h in range(c.heads):
+        oracle.stats_accumulate(Q[:nq_s, h, :], Msum[h])
+    t_stats = (time.perf_counter() - t0) * c.q_rows / nq_s
+    # append on a sample of tokens (at the last slot, like the GPU step)
+    n_s = 16
+    oc.len = c.total_tokens - c.tokens_per_frame
+    t0 = time.perf_counter()
+    oc.append_kv(K[:n_s], V[:n_s])
+    t_app = (time.perf_counter() - t0) * c.tokens_per_frame / n_s
+    oc.len = c.total_tokens
+    # attention on a sample of query rows, one head's cache reconstructed per head
+    rows = np.arange(2)
+    t0 = time.perf_counter()
+    oc.attention(Q, rows=rows)
+    t_att = (time.perf_counter() - t0) * c.q_rows / len(rows)
+    t_step = t_stats + t_app + t_att
+    note = (f"oracle (single-thread C via ctypes): stats on {nq_s} query rows, append of {n_s} "
+            f"tokens x {c.heads} heads, attention of {len(rows)} query rows x {c.heads} heads "
+            f"over the full {c.total_tokens}-token cache; each scaled to one {c.q_rows}-query step")
+    return c.q_rows / t_step, note, dict(stats_s=t_stats, append_s=t_app, attention_s=t_att)
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="480p", choices=sorted(syn.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-top1", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = syn.get_config(args.config)
+    workload_name = (f"{cfg.name} layer: {cfg.heads} heads x {cfg.head_dim}, cache "
+                     f"{cfg.frames} latent frames x {cfg.tokens_per_frame} tokens, "
+                     f"{cfg.q_rows}-query chunk, C={cfg.n_centroids}, G={cfg.group}, "
+                     f"M={cfg.n_cand}, r={cfg.rank}")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cores = 1
+        t0 = time.time()
+        vals = []
+        for _ in range(max(1, args.steps)):
+            v, note, parts = oracle_throughput(cfg, None)
+            vals.append(v)
+            if time.time() - t0 > 120:
+                break
+        v = statistics.median(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": len(vals), "warmup": 0, "ms_per_step": 1e3 * cfg.q_rows / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": workload_name},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": note, "value": v,
+                             "unit": UNIT},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    W, K = max(3, args.warmup), args.steps
+    wl = Workload(cfg, device, extra_versions=2 * (W + K) + 8)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(W):
+        wl.step(i)
+    torch.cuda.synchronize(device)
+    # ---- timed region (device time, CUDA events on the launching stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    start.record()
+    for i in range(K):
+        wl.step(i, evs[i])
+    end.record()
+    torch.cuda.synchronize(device)
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(start.elapsed_time(end))
+    seg = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                    for e in evs])
+    stats_ms, app_ms, att_ms = (float(x) for x in seg.mean(0))
+    ms_step = total_ms / K
+    value = world * cfg.q_rows / (ms_step * 1e-3)
+
+    # ---- end to end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        Qh, Kh, Vh = wl.host_pool[0]
+        bufs = (torch.empty_like(Qh, device=device), torch.empty_like(Kh, device=device),
+                torch.empty_like(Vh, device=device), torch.empty_like(Qh).pin_memory())
+        for i in range(W):
+            wl.step_host(i, bufs)
+        torch.cuda.synchronize(device)
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for i in range(K):
+            wl.step_host(i, bufs)
+        e2.record()
+        torch.cuda.synchronize(device)
+        barrier()
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2)) / K
+        e2e = {"value": world * cfg.q_rows / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),
+               "d2h_bytes_per_step": int(Qh.numel() * 2)}
+
+    # ---- derived figures
+    c = cfg
+    T = c.total_tokens
+    att_flop = 4.0 * c.q_rows * T * c.head_dim * c.heads
+    att_tflops = att_flop / (att_ms * 1e-3) / 1e12
+    per_tok = 2 * (c.head_dim // 4 + 4 * (c.head_dim // c.group) + (1 if c.n_centroids <= 256 else 2)) + c.rank + 2
+    app_bytes = c.tokens_per_frame * c.heads * (4 * c.head_dim + per_tok)
+    app_gbs = app_bytes / (app_ms * 1e-3) / 1e9
+    fixed = 2 * c.heads * c.n_centroids * c.head_dim * 2 + (c.frames // c.refresh_every) * c.heads * c.head_dim * c.rank * 4
+    compression = (4.0 * c.head_dim * T * c.heads) / (T * c.heads * per_tok + fixed)
+
+    top1 = None
+    if not args.no_top1 and rank == 0:
+        Kall = torch.cat([dev_bf16(wl.src.keys(f), device) for f in range(c.frames - 1)]
+                         + [wl.pool[(wl.nstep - 1) % len(wl.pool)][1]], 0)
+        ie, iq = wl.cache.top1_shift(wl.pool[(wl.nstep - 1) % len(wl.pool)][0], Kall)
+        top1 = float((ie != iq).float().mean().item())
+        del Kall
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_name,
+                   "l2": "inputs larger than L2: 161 MB packed cache read per step, step inputs rotate over 4 HBM-resident frames",
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": 6 * K,
+        "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16"],
+                     "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"], "traffic": None,
+                     "kernel": "qwm_attention", "peak_source": f"{peaks['source']} bf16 burst"},
+        "append": {"ms": app_ms, "tokens_per_s": c.tokens_per_frame / (app_ms * 1e-3),
+                   "GB_per_s": app_gbs, "frac_hbm": app_gbs / peaks["hbm"],
+                   "bytes_per_frame": app_bytes},
+        "attention": {"ms": att_ms, "TFLOP_per_s": att_tflops, "flop_per_call": att_flop,
+                      "frac_bf16": att_tflops / peaks["bf16"]},
+        "stats_refresh_ms": stats_ms,
+        "top1_shift": top1, "compression_ratio": compression,
+        "clocks": clk, "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, note, parts = oracle_throughput(cfg, wl.cache)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": note, "parts_s": parts}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

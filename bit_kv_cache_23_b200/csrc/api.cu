@@ -1,0 +1,217 @@
+// api.cu -- the extern "C" entry points of libqwm.so: argument validation,
+// buffer sizing, host-side cache bookkeeping and kernel dispatch.
+#include <string.h>
+
+#include "common.cuh"
+
+using namespace qwm;
+
+namespace {
+
+constexpr int32_t kMagic = 0x51574d31;  // "QWM1"
+
+bool config_ok(const qwm_config* c) {
+  if (!c) return false;
+  if (c->heads < 1 || c->heads > 4096) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->group != 16 && c->group != 32) return false;
+  if (c->head_dim % c->group) return false;
+  if (c->n_centroids < 1 || c->n_centroids > 512) return false;
+  if (c->n_cand < 1 || c->n_cand > 8 || c->n_cand > c->n_centroids) return false;
+  if (c->rank < 0 || c->rank > 16) return false;
+  if (c->max_versions < 1 || c->max_versions > 65535) return false;
+  if (c->reserved != 0) return false;
+  if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 40)) return false;
+  return true;
+}
+
+Dims dims_of(const qwm_config* c) {
+  Dims D;
+  D.H = c->heads;
+  D.d = c->head_dim;
+  D.C = c->n_centroids;
+  D.G = c->group;
+  D.M = c->n_cand;
+  D.r = c->rank;
+  D.ng = c->head_dim / c->group;
+  D.tcap = (c->max_tokens + 127) / 128 * 128;
+  D.idx_bytes = c->n_centroids <= 256 ? 1 : 2;
+  return D;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool cache_ok(const qwm_cache* c) { return c && c->magic == kMagic && config_ok(&c->cfg); }
+
+qwm_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QWM_OK;
+  return QWM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t qwm_abi_version(void) { return QWM_ABI_VERSION; }
+
+const char* qwm_status_string(qwm_status s) {
+  switch (s) {
+    case QWM_OK: return "ok";
+    case QWM_ERR_INVALID_ARG: return "invalid argument";
+    case QWM_ERR_ALIGNMENT: return "misaligned pointer";
+    case QWM_ERR_CAPACITY: return "capacity exceeded";
+    case QWM_ERR_STATE: return "invalid cache state for this call";
+    case QWM_ERR_CUDA: return "CUDA error";
+    case QWM_ERR_TIMEOUT: return "device wait timed out";
+    case QWM_ERR_UNSUPPORTED: return "unsupported device or configuration";
+  }
+  return "unknown status";
+}
+
+qwm_status qwm_cache_sizes(const qwm_config* cfg, qwm_sizes* out) {
+  if (!cfg || !out || !config_ok(cfg)) return QWM_ERR_INVALID_ARG;
+  Dims D = dims_of(cfg);
+  memset(out, 0, sizeof(*out));
+  const uint64_t HT = (uint64_t)D.H * D.tcap;
+  out->tcap = D.tcap;
+  out->bytes[QWM_BUF_K_CODES] = HT * (D.d / 4);
+  out->bytes[QWM_BUF_K_PARAMS] = HT * D.ng * 4;
+  out->bytes[QWM_BUF_K_IDX] = HT * D.idx_bytes;
+  out->bytes[QWM_BUF_K_COEF] = HT * D.r;
+  out->bytes[QWM_BUF_K_CSCALE] = HT * 2;
+  out->bytes[QWM_BUF_V_CODES] = HT * (D.d / 4);
+  out->bytes[QWM_BUF_V_PARAMS] = HT * D.ng * 4;
+  out->bytes[QWM_BUF_V_IDX] = HT * D.idx_bytes;
+  out->bytes[QWM_BUF_CENT_K] = (uint64_t)D.H * D.C * D.d * 2;
+  out->bytes[QWM_BUF_CENT_V] = (uint64_t)D.H * D.C * D.d * 2;
+  out->bytes[QWM_BUF_QSTATS] = (uint64_t)D.H * D.d * D.d * 8;
+  out->bytes[QWM_BUF_SENS] = (uint64_t)D.H * D.d * 4;
+  out->bytes[QWM_BUF_WGROUP] = (uint64_t)D.H * D.ng * 4;
+  out->bytes[QWM_BUF_BASIS] = (uint64_t)cfg->max_versions * D.H * D.d * (D.r > 0 ? D.r : 1) * 4;
+  out->bytes[QWM_BUF_TOKVER] = (uint64_t)D.tcap * 2;
+  out->bytes[QWM_BUF_EIGVEC] = (uint64_t)D.H * D.d * D.d * 8 + (uint64_t)D.H * 8;
+  out->bytes[QWM_BUF_WORKSPACE] = kmeans_workspace_bytes(D);
+  out->bytes_per_token_head = 2 * (D.d / 4 + 4 * D.ng + D.idx_bytes) + D.r + 2;
+  return QWM_OK;
+}
+
+qwm_status qwm_cache_init(qwm_cache* c, const qwm_config* cfg, const qwm_buffers* bufs,
+                          void* stream) {
+  if (!c || !cfg || !bufs || !config_ok(cfg)) return QWM_ERR_INVALID_ARG;
+  for (int i = 0; i < QWM_NBUF; ++i) {
+    if (i == QWM_BUF_K_COEF && cfg->rank == 0) continue;
+    if (!bufs->ptr[i]) return QWM_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < QWM_NBUF; ++i)
+    if (bufs->ptr[i] && !aligned(bufs->ptr[i], 256)) return QWM_ERR_ALIGNMENT;
+  Dims D = dims_of(cfg);
+  qwm_cache tmp;
+  memset(&tmp, 0, sizeof(tmp));
+  tmp.cfg = *cfg;
+  tmp.buf = *bufs;
+  tmp.tcap = D.tcap;
+  tmp.n_versions = 1;
+  tmp.cur_version = 0;
+  tmp.magic = kMagic;
+  CacheView v = view_of(&tmp);
+  cudaError_t e = launch_init_state(D, v, (cudaStream_t)stream);
+  if (e != cudaSuccess) return QWM_ERR_CUDA;
+  *c = tmp;
+  return QWM_OK;
+}
+
+qwm_status qwm_build_centroids(qwm_cache* c, const void* K, const void* V, int64_t n,
+                               int32_t iters, void* stream) {
+  if (!cache_ok(c) || !K || !V) return QWM_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16)) return QWM_ERR_ALIGNMENT;
+  Dims D = dims_of(&c->cfg);
+  if (n < D.C || n > D.tcap || iters < 1 || iters > 1000) return QWM_ERR_INVALID_ARG;
+  CacheView v = view_of(c);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_kmeans(D, (const uint16_t*)K, n, iters, v.cent_k, v.workspace, s);
+  if (e == cudaSuccess) e = launch_kmeans(D, (const uint16_t*)V, n, iters, v.cent_v, v.workspace, s);
+  if (e != cudaSuccess) return QWM_ERR_CUDA;
+  c->has_centroids = 1;
+  return QWM_OK;
+}
+
+qwm_status qwm_update_query_stats(qwm_cache* c, const void* Q, int64_t n_q, int32_t refresh_basis,
+                                  void* stream) {
+  if (!cache_ok(c) || n_q < 0 || (n_q > 0 && !Q)) return QWM_ERR_INVALID_ARG;
+  if (Q && !aligned(Q, 16)) return QWM_ERR_ALIGNMENT;
+  if (refresh_basis && c->n_versions >= c->cfg.max_versions) return QWM_ERR_CAPACITY;
+  Dims D = dims_of(&c->cfg);
+  CacheView v = view_of(c);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (n_q > 0) e = launch_stats_accumulate(D, (const uint16_t*)Q, n_q, v.qstats, s);
+  if (e != cudaSuccess) return QWM_ERR_CUDA;
+  c->n_queries += n_q;
+  if (refresh_basis) {
+    int ver = c->n_versions;
+    e = launch_refresh(D, v, c->n_queries, ver, c->has_eigvec, s);
+    if (e != cudaSuccess) return QWM_ERR_CUDA;
+    c->n_versions += 1;
+    c->cur_version = ver;
+    if (c->n_queries > 0) c->has_eigvec = 1;
+  }
+  return QWM_OK;
+}
+
+qwm_status qwm_append_kv(qwm_cache* c, const void* K, const void* V, int64_t n, void* stream) {
+  if (!cache_ok(c) || n < 0 || (n > 0 && (!K || !V))) return QWM_ERR_INVALID_ARG;
+  if ((K && !aligned(K, 16)) || (V && !aligned(V, 16))) return QWM_ERR_ALIGNMENT;
+  if (!c->has_centroids) return QWM_ERR_STATE;
+  if (c->len + n > c->tcap) return QWM_ERR_CAPACITY;
+  if (n == 0) return QWM_OK;
+  Dims D = dims_of(&c->cfg);
+  CacheView v = view_of(c);
+  cudaError_t e = launch_append(D, v, (const uint16_t*)K, (const uint16_t*)V, n, c->len,
+                                c->cur_version, (cudaStream_t)stream);
+  if (e != cudaSuccess) return QWM_ERR_CUDA;
+  c->len += n;
+  c->frames += 1;
+  return QWM_OK;
+}
+
+qwm_status qwm_attention(const qwm_cache* c, const void* Q, int64_t n_q, float scale, void* O,
+                         void* stream) {
+  if (!cache_ok(c) || n_q < 0 || (n_q > 0 && (!Q || !O))) return QWM_ERR_INVALID_ARG;
+  if ((Q && !aligned(Q, 16)) || (O && !aligned(O, 16))) return QWM_ERR_ALIGNMENT;
+  if (c->len <= 0 || !c->has_centroids) return QWM_ERR_STATE;
+  if (n_q == 0) return QWM_OK;
+  Dims D = dims_of(&c->cfg);
+  if (!(scale > 0.0f)) scale = 1.0f / sqrtf((float)D.d);
+  CacheView v = view_of(c);
+  return cuda_status(launch_attention(D, v, c->len, (const uint16_t*)Q, n_q, scale, (uint16_t*)O,
+                                      (cudaStream_t)stream));
+}
+
+qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, void* Kp, void* Vp,
+                           void* stream) {
+  if (!cache_ok(c) || t0 < 0 || n < 0 || t0 + n > c->len || (n > 0 && (!Kp || !Vp)))
+    return QWM_ERR_INVALID_ARG;
+  if ((Kp && !aligned(Kp, 16)) || (Vp && !aligned(Vp, 16))) return QWM_ERR_ALIGNMENT;
+  if (n == 0) return QWM_OK;
+  Dims D = dims_of(&c->cfg);
+  CacheView v = view_of(c);
+  return cuda_status(
+      launch_reconstruct(D, v, t0, n, (uint16_t*)Kp, (uint16_t*)Vp, (cudaStream_t)stream));
+}
+
+qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q, const void* K_exact,
+                          int32_t* idx_exact, int32_t* idx_quant, void* stream) {
+  if (!cache_ok(c) || n_q < 0 || (n_q > 0 && (!Q || !K_exact || !idx_exact || !idx_quant)))
+    return QWM_ERR_INVALID_ARG;
+  if ((Q && !aligned(Q, 16)) || (K_exact && !aligned(K_exact, 16)) ||
+      (idx_exact && !aligned(idx_exact, 4)) || (idx_quant && !aligned(idx_quant, 4)))
+    return QWM_ERR_ALIGNMENT;
+  if (c->len <= 0) return QWM_ERR_STATE;
+  if (n_q == 0) return QWM_OK;
+  Dims D = dims_of(&c->cfg);
+  CacheView v = view_of(c);
+  return cuda_status(launch_top1(D, v, c->len, (const uint16_t*)Q, n_q, (const uint16_t*)K_exact,
+                                 idx_exact, idx_quant, (cudaStream_t)stream));
+}
+
+}  // extern "C"

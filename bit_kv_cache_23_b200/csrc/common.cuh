@@ -1,0 +1,115 @@
+// common.cuh -- internal declarations shared by the CUDA translation units of
+// libqwm.so (device helpers, problem dimensions, kernel launchers).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qwm.h"
+
+namespace qwm {
+
+// Problem dimensions derived from a validated qwm_config.
+struct Dims {
+  int H, d, C, G, M, r, ng;
+  int64_t tcap;
+  int idx_bytes;  // 1 if C <= 256 else 2
+};
+
+// Views of the cache buffers (device pointers).
+struct CacheView {
+  uint8_t* k_codes;
+  uint16_t* k_params;
+  void* k_idx;
+  int8_t* k_coef;
+  uint16_t* k_cscale;
+  uint8_t* v_codes;
+  uint16_t* v_params;
+  void* v_idx;
+  uint16_t* cent_k;
+  uint16_t* cent_v;
+  double* qstats;
+  float* sens;
+  float* wgroup;
+  float* basis;
+  uint16_t* tokver;
+  double* eigvec;
+  void* workspace;
+};
+
+inline CacheView view_of(const qwm_cache* c) {
+  CacheView v;
+  v.k_codes = (uint8_t*)c->buf.ptr[QWM_BUF_K_CODES];
+  v.k_params = (uint16_t*)c->buf.ptr[QWM_BUF_K_PARAMS];
+  v.k_idx = c->buf.ptr[QWM_BUF_K_IDX];
+  v.k_coef = (int8_t*)c->buf.ptr[QWM_BUF_K_COEF];
+  v.k_cscale = (uint16_t*)c->buf.ptr[QWM_BUF_K_CSCALE];
+  v.v_codes = (uint8_t*)c->buf.ptr[QWM_BUF_V_CODES];
+  v.v_params = (uint16_t*)c->buf.ptr[QWM_BUF_V_PARAMS];
+  v.v_idx = c->buf.ptr[QWM_BUF_V_IDX];
+  v.cent_k = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_K];
+  v.cent_v = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_V];
+  v.qstats = (double*)c->buf.ptr[QWM_BUF_QSTATS];
+  v.sens = (float*)c->buf.ptr[QWM_BUF_SENS];
+  v.wgroup = (float*)c->buf.ptr[QWM_BUF_WGROUP];
+  v.basis = (float*)c->buf.ptr[QWM_BUF_BASIS];
+  v.tokver = (uint16_t*)c->buf.ptr[QWM_BUF_TOKVER];
+  v.eigvec = (double*)c->buf.ptr[QWM_BUF_EIGVEC];
+  v.workspace = c->buf.ptr[QWM_BUF_WORKSPACE];
+  return v;
+}
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f2bf(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ uint16_t f2h_rd(float x) { return __half_as_ushort(__float2half_rd(x)); }
+__device__ __forceinline__ uint16_t f2h_ru(float x) { return __half_as_ushort(__float2half_ru(x)); }
+
+// Canonical INT2 group parameters from the fp32 residual range [lo, hi]:
+// mn = fp16 round-down(lo), sc = fp16 round-up((hi - mn) / 3); zeros as +0.
+__device__ __forceinline__ void int2_params(float lo, float hi, uint16_t& mnh, uint16_t& sch,
+                                            float& mn, float& sc) {
+  if (lo == 0.0f) lo = 0.0f;
+  if (hi == 0.0f) hi = 0.0f;
+  mnh = f2h_rd(lo);
+  mn = h2f(mnh);
+  sch = f2h_ru(__fdiv_rn(__fsub_rn(hi, mn), 3.0f));
+  sc = h2f(sch);
+}
+
+// code = #{k in 0..2 : rho >= mn + (k + 0.5) sc}, 0 when sc == 0.
+__device__ __forceinline__ int int2_code(float rho, float mn, float sc) {
+  if (sc == 0.0f) return 0;
+  int c = 0;
+  c += rho >= __fadd_rn(mn, __fmul_rn(0.5f, sc));
+  c += rho >= __fadd_rn(mn, __fmul_rn(1.5f, sc));
+  c += rho >= __fadd_rn(mn, __fmul_rn(2.5f, sc));
+  return c;
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_init_state(const Dims& D, const CacheView& v, cudaStream_t s);
+cudaError_t launch_kmeans(const Dims& D, const uint16_t* X, int64_t n, int iters, uint16_t* cent_out,
+                          void* workspace, cudaStream_t s);
+cudaError_t launch_stats_accumulate(const Dims& D, const uint16_t* Q, int64_t n, double* qstats,
+                                    cudaStream_t s);
+cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, int version,
+                           int warm, cudaStream_t s);
+cudaError_t launch_append(const Dims& D, const CacheView& v, const uint16_t* K, const uint16_t* V,
+                          int64_t n, int64_t t0, int version, cudaStream_t s);
+cudaError_t launch_attention(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
+                             int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+cudaError_t launch_reconstruct(const Dims& D, const CacheView& v, int64_t t0, int64_t n,
+                               uint16_t* Kp, uint16_t* Vp, cudaStream_t s);
+cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
+                        int64_t nq, const uint16_t* Kexact, int32_t* idx_exact,
+                        int32_t* idx_quant, cudaStream_t s);
+
+size_t kmeans_workspace_bytes(const Dims& D);
+
+}  // namespace qwm

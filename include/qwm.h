@@ -1,0 +1,197 @@
+/*
+ * qwm.h -- C ABI of the B200 QuantWM 2-bit KV-cache library (libqwm.so).
+ *
+ * What the library computes (QuantWM: Temporally Consistent 2-Bit KV Cache
+ * Quantization for Video World Models):
+ *   - Keys are stored as a centroid (bf16) plus an INT2 residual; the centroid
+ *     is chosen by QSAC (quantization-sensitivity-aware clustering): shortlist
+ *     by Query-sensitivity-weighted distance, then the expected squared
+ *     logit-perturbation of the INT2 residual decides.
+ *     ["Flickering after quantization?" (SynthePulse en-US), QSAC paragraph;
+ *      evolve.pub review, Summary and Strengths, Eq. 7]
+ *   - PSAC (principal-subspace attention compensation) stores the remaining Key
+ *     error projected on the top-r principal Query directions as INT8, added
+ *     back when the cache is reconstructed.
+ *     [same SynthePulse page, PSAC paragraph; review Summary, Fig. 4, Table 9]
+ *   - Values: nearest centroid plus INT2 residual (the centroid-residual scheme
+ *     QuantWM builds on; review Summary).
+ *   - Attention of new queries over the packed cache with the reconstruction
+ *     K' = C[a] + deq(R) + U deq8(c), V' = C_V[b] + deq(R_V) fused in.
+ *
+ * Conventions
+ *   - Every device buffer is allocated and owned by the caller, at the sizes
+ *     qwm_cache_sizes() reports, 256-byte aligned.  The library never allocates
+ *     device memory.  qwm_cache is a small host struct the caller owns.
+ *   - `stream` is a cudaStream_t passed as void*.  Calls enqueue kernels on it
+ *     and return without synchronizing.  Calls on one cache must be ordered on
+ *     one stream.  The host fields of qwm_cache change at enqueue time.
+ *   - Tensors Q, K, V, O are token-major [n][heads][head_dim] bf16 (uint16 bit
+ *     patterns), contiguous, device pointers, 16-byte aligned.
+ *   - Errors: every argument is validated before anything is enqueued; on error
+ *     nothing is enqueued and the cache is unchanged.  QWM_ERR_CUDA reports a
+ *     launch failure (cudaGetLastError).  Nothing aborts or throws across the ABI.
+ *   - Inputs must be finite.  Residuals beyond the fp16 range (|k - c| > 65504)
+ *     are outside the supported domain.
+ */
+#ifndef QWM_H
+#define QWM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QWM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define QWM_API __attribute__((visibility("default")))
+#else
+#define QWM_API
+#endif
+
+typedef enum qwm_status {
+  QWM_OK = 0,
+  QWM_ERR_INVALID_ARG = 1, /* null pointer, bad size, unsupported combination */
+  QWM_ERR_ALIGNMENT = 2,   /* pointer not aligned as documented             */
+  QWM_ERR_CAPACITY = 3,    /* tokens or basis versions beyond the capacity  */
+  QWM_ERR_STATE = 4,       /* e.g. append before centroids were built       */
+  QWM_ERR_CUDA = 5,        /* a CUDA launch or runtime call failed          */
+  QWM_ERR_TIMEOUT = 6,     /* a bounded device wait gave up                  */
+  QWM_ERR_UNSUPPORTED = 7  /* no kernel for this device / configuration     */
+} qwm_status;
+
+/* Quantizer and capacity.  Supported: head_dim 64 or 128; group 16 or 32 and
+ * dividing head_dim; 1 <= n_centroids <= 512; 1 <= n_cand <= min(8, C);
+ * 0 <= rank <= 16; 1 <= max_versions <= 65535; max_tokens >= 1. */
+typedef struct qwm_config {
+  int32_t heads;        /* H                                             */
+  int32_t head_dim;     /* d                                             */
+  int32_t n_centroids;  /* C (per head, same count for K and V)          */
+  int32_t group;        /* G: channels per INT2 group                    */
+  int32_t n_cand;       /* M: QSAC shortlist size                        */
+  int32_t rank;         /* r: PSAC rank                                  */
+  int32_t max_versions; /* slots for successive bases U (one per refresh) */
+  int32_t reserved;     /* must be 0                                     */
+  int64_t max_tokens;   /* cache capacity per head                       */
+} qwm_config;
+
+/* Device buffers, indexed by qwm_buffer_id.  Layout (Tcap = max_tokens rounded
+ * up to a multiple of 128, ng = d / G, idx = uint8 if C <= 256 else uint16):
+ *   K_CODES   [H][Tcap][d/4]   uint8   4 INT2 codes per byte, channel j in bits 2(j%4)
+ *   K_PARAMS  [H][Tcap][ng][2] fp16    per group {mn, sc}: deq = mn + code * sc
+ *   K_IDX     [H][Tcap]        idx     centroid of each key
+ *   K_COEF    [H][Tcap][r]     int8    PSAC coefficients
+ *   K_CSCALE  [H][Tcap]        fp16    PSAC per-token scale
+ *   V_CODES, V_PARAMS, V_IDX   as for K
+ *   CENT_K, CENT_V [H][C][d]   bf16    centroid tables
+ *   QSTATS    [H][d][d]        fp64    running sum of q q^T
+ *   SENS      [H][d]           fp32    s_j = E[q_j^2] in force
+ *   WGROUP    [H][ng]          fp32    w_g = sum of s_j over group g
+ *   BASIS     [max_versions][H][d][r] fp32  PSAC bases, slot = version
+ *   TOKVER    [Tcap]           uint16  basis version of each cached token
+ *   EIGVEC    [H][d][d] + [H]  fp64    eigenvectors of the last refresh, then one
+ *                                      warm-start flag per head
+ *   WORKSPACE                  bytes   scratch for centroid building and basis refresh */
+typedef enum qwm_buffer_id {
+  QWM_BUF_K_CODES = 0, QWM_BUF_K_PARAMS, QWM_BUF_K_IDX, QWM_BUF_K_COEF, QWM_BUF_K_CSCALE,
+  QWM_BUF_V_CODES, QWM_BUF_V_PARAMS, QWM_BUF_V_IDX, QWM_BUF_CENT_K, QWM_BUF_CENT_V,
+  QWM_BUF_QSTATS, QWM_BUF_SENS, QWM_BUF_WGROUP, QWM_BUF_BASIS, QWM_BUF_TOKVER,
+  QWM_BUF_EIGVEC, QWM_BUF_WORKSPACE, QWM_NBUF
+} qwm_buffer_id;
+
+typedef struct qwm_sizes {
+  uint64_t bytes[QWM_NBUF]; /* size of each buffer                       */
+  int64_t tcap;             /* token capacity per head after rounding    */
+  int64_t bytes_per_token_head; /* packed bytes per cached token and head */
+} qwm_sizes;
+
+typedef struct qwm_buffers {
+  void* ptr[QWM_NBUF];
+} qwm_buffers;
+
+/* Host-side cache state; owned by the caller, filled by qwm_cache_init. */
+typedef struct qwm_cache {
+  qwm_config cfg;
+  qwm_buffers buf;
+  int64_t tcap;
+  int64_t len;          /* tokens cached (per head)                 */
+  int64_t n_queries;    /* query rows accumulated into QSTATS       */
+  int32_t frames;       /* qwm_append_kv calls so far               */
+  int32_t n_versions;   /* basis versions written (>= 1 after init) */
+  int32_t cur_version;  /* version used by the next append          */
+  int32_t has_centroids;
+  int32_t has_eigvec;   /* EIGVEC holds a previous decomposition    */
+  int32_t magic;
+} qwm_cache;
+
+QWM_API int32_t qwm_abi_version(void);
+QWM_API const char* qwm_status_string(qwm_status s);
+
+/* Buffer sizes for `cfg` (host only, no device work).
+ * Errors: QWM_ERR_INVALID_ARG for a null pointer or an unsupported config. */
+QWM_API qwm_status qwm_cache_sizes(const qwm_config* cfg, qwm_sizes* out);
+
+/* Fill `c` and enqueue the initial device state: QSTATS = 0, SENS = 1,
+ * WGROUP = G, BASIS version 0 = 0 (no history: PSAC adds nothing).
+ * Every pointer in `bufs` must be non-null (K_COEF may be null when rank is 0)
+ * and 256-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+QWM_API qwm_status qwm_cache_init(qwm_cache* c, const qwm_config* cfg, const qwm_buffers* bufs,
+                          void* stream);
+
+/* Centroid tables from the first cached frame (k-means, per head, separately
+ * for K and V).  The pages say only that each Key is assigned to a cluster
+ * centre kept at higher precision (SynthePulse, QSAC paragraph).  Here:
+ * centroid i starts at token floor(i n / C); `iters` Lloyd rounds with fp32
+ * squared distances (ties to the lower index) and fp64 means taken in token
+ * order; an empty cluster keeps its centroid; the result is rounded to bf16.
+ * K, V: [n][H][d] bf16 device.  Requires n >= C, n <= tcap and
+ * 1 <= iters <= 1000.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+QWM_API qwm_status qwm_build_centroids(qwm_cache* c, const void* K, const void* V, int64_t n,
+                               int32_t iters, void* stream);
+
+/* Historical Query statistics [review, Summary: "historical Query
+ * second-moment statistics"; Eq. 7 M = E[q q^T]]: QSTATS[h] += sum_t q_t q_t^T,
+ * n_queries += n_q.  With refresh_basis != 0 it then refreshes what QSAC and
+ * PSAC read: s_j = M_jj / n, w_g = sum_{j in g} s_j, U = top-r eigenvectors of
+ * M / n (Jacobi, warm-started from the last refresh), stored as a new basis
+ * version used by later appends.  Q: [n_q][H][d] bf16 device, n_q >= 0.
+ * Errors: INVALID_ARG, ALIGNMENT, CAPACITY (no free basis slot), CUDA. */
+QWM_API qwm_status qwm_update_query_stats(qwm_cache* c, const void* Q, int64_t n_q,
+                                  int32_t refresh_basis, void* stream);
+
+/* Quantize and append n tokens at position len (QSAC + INT2 + PSAC for Keys,
+ * nearest centroid + INT2 for Values) with the statistics and basis in force.
+ * Codes, indices and INT8 coefficients are bit-identical to the canonical
+ * fp32 definition the CPU oracle implements.  K, V: [n][H][d] bf16 device.
+ * Errors: INVALID_ARG, ALIGNMENT, CAPACITY (len + n > tcap), STATE (no
+ * centroids), CUDA. */
+QWM_API qwm_status qwm_append_kv(qwm_cache* c, const void* K, const void* V, int64_t n, void* stream);
+
+/* O = softmax(scale Q K'^T) V' over all `len` cached tokens, with K', V'
+ * reconstructed on the fly from the packed cache (each key with the basis
+ * version in force when it was appended).  No mask.  Q, O: [n_q][H][d] bf16
+ * device (O written, fp32 accumulation).  scale <= 0 selects 1/sqrt(d).
+ * Errors: INVALID_ARG, ALIGNMENT, STATE (empty cache), CUDA. */
+QWM_API qwm_status qwm_attention(const qwm_cache* c, const void* Q, int64_t n_q, float scale, void* O,
+                         void* stream);
+
+/* Reconstructed cache, for inspection: K', V' of tokens [t0, t0+n) as
+ * [H][n][d] bf16 device arrays.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+QWM_API qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, void* Kp, void* Vp,
+                           void* stream);
+
+/* Top-1 key selection of each query row (argmax_t q . k_t, fp32 dot, ties to
+ * the lower t) over the exact keys `K_exact` ([len][H][d] bf16, the keys as
+ * they were appended) and over the reconstructed cache; the fraction that
+ * differ is the selection shift the pages report ("Flickering after
+ * quantization?", attention-analysis paragraph).  idx_exact, idx_quant:
+ * [n_q][H] int32 device.  Errors: INVALID_ARG, ALIGNMENT, STATE, CUDA. */
+QWM_API qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q, const void* K_exact,
+                          int32_t* idx_exact, int32_t* idx_quant, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QWM_H */

@@ -348,7 +348,8 @@ QO_API void qo_int2_encode(const float* rho, int d, int G, uint8_t* codes, uint1
       lo = fminf(lo, rho[j]);
       hi = fmaxf(hi, rho[j]);
     }
-    if (lo == 0.0f) lo = 0.0f; /* a zero minimum is +0 (never -0) */
+    if (lo == 0.0f) lo = 0.0f; /* zeros enter as +0 (never -0), so the fp16 */
+    if (hi == 0.0f) hi = 0.0f; /* parameters of an all-zero group are +0    */
     uint16_t mnh = qo_f32_to_f16(lo, QO_RD);
     float mn = qo_f16_to_f32(mnh);
     uint16_t sch = qo_f32_to_f16((hi - mn) / 3.0f, QO_RU);

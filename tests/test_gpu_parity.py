@@ -1,0 +1,108 @@
+"""GPU path (C ABI through the binding) against the CPU oracle.
+
+Bit-exact: centroid tables, centroid indices, INT2 codes, fp16 group
+parameters, INT8 coefficients and scales.  Tolerance: attention output within
+max-abs 2e-2 and mean-abs 2e-3 of the oracle's fp64 attention over the same
+reconstructed cache; statistics and basis against the oracle's fp64 versions.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qwm_synth as syn
+from parity_util import ATOL_MAX, ATOL_MEAN, run_layer, to_dev, u16
+
+pytestmark = pytest.mark.gpu
+
+
+def _assert_common(out, proj_tol=1e-4):
+    assert out["cent_k_equal"] and out["cent_v_equal"], "k-means centroids differ"
+    assert out["packed_mismatch"] == {}, out["packed_mismatch"]
+    assert out["stats_rel"] < 1e-5, out["stats_rel"]
+    assert out["orth_err"] < 1e-5, out["orth_err"]
+    assert out["proj_err"] < proj_tol, out["proj_err"]
+    for f, mx, mean in out["attn"]:
+        assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (f, mx, mean)
+
+
+def test_tiny_full():
+    out = run_layer("tiny")
+    _assert_common(out)
+    # reconstruction: GPU fp32 sum vs oracle fp64 sum, both rounded to bf16
+    g, oc = out["gpu"], out["oracle"]
+    Kp, Vp = g.reconstruct()
+    Ko, Vo = oc.reconstruct(0)
+    kg = syn.bf16_bits_to_f32(u16(Kp[0]))
+    ko = syn.bf16_bits_to_f32(Ko)
+    assert np.all(np.abs(kg - ko) <= np.spacing(np.abs(ko)) * 1.01 + 1e-30)
+    assert np.array_equal(u16(Vp[0]), Vo)
+
+
+def test_small_full():
+    out = run_layer("small", attn_rows=24, attn_frames={0, 4, 8})
+    _assert_common(out)
+
+
+def test_top1_shift_tiny():
+    out = run_layer("tiny")
+    g, oc, src, c = out["gpu"], out["oracle"], out["src"], out["cfg"]
+    Kall = np.concatenate([src.keys(f) for f in range(c.frames)], axis=0)
+    Q = src.queries(c.frames - 1)
+    ie, iq = g.top1_shift(to_dev(Q), to_dev(Kall))
+    ie, iq = ie.cpu().numpy(), iq.cpu().numpy()
+    Ko, _ = oc.reconstruct(0)
+    ref_e = oracle.top1(Q[:, 0, :], Kall[:, 0, :])
+    ref_q = oracle.top1(Q[:, 0, :], Ko)
+    qf = syn.bf16_bits_to_f32(Q[:, 0, :]).astype(np.float64)
+    for ref, got, K in ((ref_e, ie[:, 0], Kall[:, 0, :]), (ref_q, iq[:, 0], Ko)):
+        sc = qf @ syn.bf16_bits_to_f32(K).astype(np.float64).T
+        best = sc[np.arange(len(ref)), ref]
+        mine = sc[np.arange(len(ref)), got]
+        assert np.all(best - mine <= 1e-4 * np.abs(best) + 1e-4)
+
+
+def test_degenerate_inputs():
+    """Constant keys (zero residual groups), repeated tokens, one-token appends,
+    a ragged tail and zero-variance channels."""
+    c = syn.get_config("tiny")
+    H, d, C = 1, 64, 16
+    g = pytest.importorskip("bit_kv_cache_23_b200").QuantKVCache(H, d, C, 16, 4, 4, 300,
+                                                                 max_versions=8)
+    oc = oracle.OracleCache(H, d, C, 16, 4, 4, 300)
+    rng = np.random.default_rng(77)
+    base = rng.standard_normal((40, H, d)).astype(np.float32)
+    base[:, :, :16] = 0.25       # a constant group
+    base[5:15] = base[5]         # repeated tokens
+    K = syn.f32_to_bf16_bits(base)
+    V = syn.f32_to_bf16_bits(rng.standard_normal((40, H, d)).astype(np.float32))
+    g.build_centroids(to_dev(K), to_dev(V), iters=3)
+    torch.cuda.synchronize()
+    CK = g.view("cent_k").cpu().numpy().view(np.uint16).copy()
+    CV = g.view("cent_v").cpu().numpy().view(np.uint16).copy()
+    ck, _ = oracle.kmeans(K[:, 0, :], C, 3)
+    assert np.array_equal(ck, CK[0])
+    oc.set_state(CK=CK, CV=CV)
+    # appends before any query statistics: s = 1, U = 0
+    for n in (1, 7, 32):
+        t0 = g.len
+        g.append_kv(to_dev(K[:n]), to_dev(V[:n]))
+        oc.append_kv(K[:n], V[:n])
+        from parity_util import compare_packed
+        assert compare_packed(g, oc, t0, g.len) == {}
+    Q = syn.f32_to_bf16_bits(rng.standard_normal((3, H, d)).astype(np.float32))
+    g.update_query_stats(to_dev(Q), refresh_basis=True)   # fewer queries than rank
+    s, w, U = (g.view("sens").cpu().numpy(), g.view("wgroup").cpu().numpy(),
+               g.view("basis")[g.version].cpu().numpy())
+    assert np.all(np.isfinite(U))
+    oc.set_state(s=s, w=w, U=U)
+    t0 = g.len
+    g.append_kv(to_dev(K), to_dev(V))
+    oc.append_kv(K, V)
+    from parity_util import compare_packed
+    assert compare_packed(g, oc, t0, g.len) == {}
+    O = g.attention(to_dev(Q))
+    torch.cuda.synchronize()
+    Oref = oc.attention(Q)
+    err = np.abs(syn.bf16_bits_to_f32(u16(O)) - Oref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3
