@@ -21,7 +21,7 @@ __all__ = [
     "QwmError", "qwm_config", "qwm_sizes", "qwm_buffers", "qwm_cache", "BUFFER_NAMES",
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
     "qwm_build_centroids", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
-    "qwm_reconstruct", "qwm_top1_shift", "QuantKVCache",
+    "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +92,7 @@ def lib():
             "qwm_attention": (I32, [pc, _P, I64, F32, _P, _P]),
             "qwm_reconstruct": (I32, [pc, I64, I64, _P, _P, _P]),
             "qwm_top1_shift": (I32, [pc, _P, I64, _P, _P, _P, _P]),
+            "qwm_device_status": (I32, [ctypes.POINTER(ctypes.c_int32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -194,6 +195,16 @@ def qwm_top1_shift(cache: qwm_cache, Q: torch.Tensor, K_exact: torch.Tensor, str
         _dev_ptr(K_exact, "K_exact", torch.bfloat16), _dev_ptr(ie, "idx_exact"),
         _dev_ptr(iq, "idx_quant"), _stream(stream, Q.device)))
     return ie, iq
+
+
+def qwm_device_status() -> int:
+    """Synchronize and return 1 if a bounded device wait timed out since the
+    last call (the flag is cleared), else 0."""
+    f = ctypes.c_int32(0)
+    st = lib().qwm_device_status(ctypes.byref(f))
+    if st not in (0, 6):
+        raise QwmError("qwm_device_status", st)
+    return int(f.value)
 
 
 # ----------------------------------------------------------------- convenience owner

@@ -214,4 +214,13 @@ qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q, const 
                                  idx_exact, idx_quant, (cudaStream_t)stream));
 }
 
+qwm_status qwm_device_status(int32_t* flags) {
+  if (!flags) return QWM_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QWM_ERR_CUDA;
+  int v = read_and_clear_tc_timeout();
+  if (v < 0) return QWM_ERR_CUDA;
+  *flags = v;
+  return v ? QWM_ERR_TIMEOUT : QWM_OK;
+}
+
 }  // extern "C"

@@ -228,9 +228,10 @@ cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint
   return cudaGetLastError();
 }
 
-// Until the tensor-core kernel lands every attention call takes this path.
+// head_dim 128 runs on the tensor cores; other shapes use the CUDA-core kernel.
 cudaError_t launch_attention(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
                              int64_t nq, float scale, uint16_t* O, cudaStream_t s) {
+  if (attention_tc_supported(D)) return launch_attention_tc(D, v, T, Q, nq, scale, O, s);
   return launch_attention_simt(D, v, T, Q, nq, scale, O, s);
 }
 

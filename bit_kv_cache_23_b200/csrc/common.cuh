@@ -111,5 +111,11 @@ cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint
                         int32_t* idx_quant, cudaStream_t s);
 
 size_t kmeans_workspace_bytes(const Dims& D);
+bool attention_tc_supported(const Dims& D);
+cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
+                                int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+cudaError_t launch_attention_simt(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
+                                  int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+int read_and_clear_tc_timeout();
 
 }  // namespace qwm

@@ -191,6 +191,13 @@ QWM_API qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, vo
 QWM_API qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q, const void* K_exact,
                           int32_t* idx_exact, int32_t* idx_quant, void* stream);
 
+/* Device-side health check: synchronizes the current device, then reads and
+ * clears the flag that the tensor-core kernels set when one of their bounded
+ * waits gave up (about one second per wait) instead of hanging.  *flags = 1 and
+ * QWM_ERR_TIMEOUT if any wait timed out since the last call, else 0 and QWM_OK.
+ * Errors: INVALID_ARG (null), CUDA. */
+QWM_API qwm_status qwm_device_status(int32_t* flags);
+
 #ifdef __cplusplus
 }
 #endif

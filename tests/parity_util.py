@@ -134,6 +134,7 @@ def run_layer(name: str, frames=None, attn_rows=None, attn_frames=None, check_ev
         if attn_frames is None or f in attn_frames:
             Od = g.attention(Qd)
             torch.cuda.synchronize()
+            assert q.qwm_device_status() == 0, "a bounded device wait timed out"
             Og = syn.bf16_bits_to_f32(u16(Od))
             rows = (np.arange(Q.shape[0]) if attn_rows is None
                     else np.sort(rng.choice(Q.shape[0], size=min(attn_rows, Q.shape[0]),
