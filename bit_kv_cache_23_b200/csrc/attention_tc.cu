@@ -7,21 +7,29 @@
 // when the cache is reconstructed; U_v is the basis in force when the key was
 // appended).
 //
+// The compensation term runs on the tensor cores instead of per element:
+//   q . (U_v c_t) = (U_v^T q) . c_t,
+// so each QK^T gains one extra K16 step (two for r > 8) whose A operand holds
+// [Q U_va | Q U_vb] for the (at most two) basis versions va, vb of the tile and
+// whose B operand holds each key's c8 cs in the slot of its version.  A key whose
+// version is neither (a tile spanning more than two versions) is compensated
+// element-wise by the dequant thread instead.
+//
 // One CTA per (head, 128 query rows); 288 threads in three roles:
 //   warps 0-3  softmax: warp w owns TMEM lanes 32w..32w+31 = query rows; loads
 //              S from TMEM, online softmax in the log2 domain, writes P (bf16)
-//              to shared memory; rescales O in TMEM when a row max moves.
+//              to shared memory; rescales O in TMEM when a row max moves; builds
+//              the [Q U_va | Q U_vb] slab two tiles ahead.
 //   warps 4-7  dequant: thread i reconstructs key row i of each 128-key tile
-//              (K' and V', bf16) straight into the 128B-swizzled shared-memory
-//              layout the UMMA descriptors read.
-//   warp 8     MMA: one thread issues S = Q K'^T (8 x K16 steps, M=128, N=128)
-//              and O += P V' (V' read MN-major), commits to mbarriers.
-// Buffers: K'/V' tiles, S and P are double-buffered, so the QK^T of tile j+1
-// runs while the softmax works on tile j.  O accumulates in TMEM across all
-// tiles.  TMEM: S[2] at columns 0/128, O at 256 (512 columns allocated; one
-// CTA per SM by shared memory).
-// Every mbarrier wait is bounded (about 1 s); a timeout sets a device flag
-// that qwm_device_status() reports, and every role then leaves its loop.
+//              (K-hat and V', bf16) straight into the 128B-swizzled layout the
+//              UMMA descriptors read, plus the key's compensation slab row.
+//   warp 8     MMA: one thread issues S = Q K'^T and O += P V' (V' read
+//              MN-major) and commits to mbarriers.
+// K-hat/V' tiles, the slabs and S are double-buffered, so the QK^T of tile j+1
+// runs while the softmax works on tile j.  TMEM: S[2] at columns 0/128, O at
+// 256 (512 columns; one CTA per SM by shared memory).  Every mbarrier wait is
+// bounded (about 1 s); a timeout sets a device flag that qwm_device_status()
+// reports, and every role then leaves its loop.
 #include <math.h>
 
 #include "dequant.cuh"
@@ -38,25 +46,29 @@ constexpr int BQ = 128;        // query rows per CTA
 constexpr int KT = 128;        // keys per tile
 constexpr int DH = 128;        // head_dim handled here
 constexpr int NTHREADS = 288;
-constexpr uint32_t TILE = 128 * 128 * 2;  // one bf16 128x128 tile
+constexpr uint32_t TILE = 128 * 128 * 2;   // one bf16 128x128 tile
+constexpr uint32_t XSLAB = 128 * 32 * 2;   // [128][<=32] bf16 compensation slab
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + TILE;          // 2 slots
-constexpr uint32_t OFF_V = OFF_K + 2 * TILE;      // 2 slots
-constexpr uint32_t OFF_P = OFF_V + 2 * TILE;      // 2 buffers
-constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
+constexpr uint32_t OFF_K = OFF_Q + TILE;         // 2 slots
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE;     // 2 slots
+constexpr uint32_t OFF_P = OFF_V + 2 * TILE;     // 1 buffer
+constexpr uint32_t OFF_AX = OFF_P + TILE;        // 2 buffers (by tile parity)
+constexpr uint32_t OFF_BX = OFF_AX + 2 * XSLAB;  // 2 slots (with K-hat/V')
+constexpr uint32_t OFF_BAR = OFF_BX + 2 * XSLAB;
 constexpr int NBAR = 16;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 
 enum {
-  B_KV_FULL = 0,  // [2] dequant -> MMA (128 arrivals)
+  B_KV_FULL = 0,  // [2] dequant (128) -> MMA
   B_KV_EMPTY = 2, // [2] MMA commit -> dequant
   B_S_FULL = 4,   // [2] MMA commit -> softmax
   B_S_FREE = 6,   // [2] softmax (128) -> MMA
-  B_P_FULL = 8,   // [2] softmax (128) -> MMA
-  B_O_FULL = 10,  // MMA commit after each P V' -> softmax (rescale, epilogue)
-  B_Q_READY = 11, // softmax (128) -> MMA
-  B_DONE = 12,    // MMA commit -> MMA (drain before exit)
-  B_O_LAST = 13   // MMA commit after the last P V' -> softmax epilogue
+  B_AX_FULL = 8,  // [2] softmax (128) -> MMA: slab for the tile of that parity
+  B_P_FULL = 10,  // softmax (128) -> MMA
+  B_O_FULL = 11,  // MMA commit after each P V'
+  B_Q_READY = 12, // softmax (128) -> MMA
+  B_DONE = 13,    // MMA commit -> MMA (drain before exit)
+  B_O_LAST = 14   // MMA commit after the last P V'
 };
 
 struct TcArgs {
@@ -67,6 +79,7 @@ struct TcArgs {
   int64_t nq;
   float scale_log2;
   uint16_t* O;
+  int kx;  // extra K width for the compensation (0, 16 or 32)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -82,7 +95,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 __device__ __forceinline__ void timeout_flag() { atomicExch(&g_tc_timeout, 1); }
 
-// ------------------------------------------------------------------ softmax role
+// byte offset of 16-byte chunk c (8 bf16) of row r in a no-swizzle K-major slab
+// with kx columns: core matrices of 8 rows x 16 B, K-adjacent cores 128 B apart,
+// 8-row groups kx*16 B apart.
+__device__ __forceinline__ uint32_t xslab_off(int r, int c, int kx) {
+  return (uint32_t)((r >> 3) * (kx * 16) + c * 128 + (r & 7) * 16);
+}
+
+// versions in force for the first and the last key of tile j
+__device__ __forceinline__ void tile_versions(const uint16_t* tokver, int64_t T, int j, int& va,
+                                              int& vb) {
+  const int64_t t0 = (int64_t)j * KT;
+  const int64_t t1 = ((t0 + KT) < T ? (t0 + KT) : T) - 1;
+  va = tokver[t0];
+  vb = tokver[t1];
+}
+
 // 32 lanes x 32 fp32 columns to TMEM (the store wait is part of the statement).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -98,10 +126,52 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+// ------------------------------------------------------------------ softmax role
 // The exponent reference m_used of a row moves only when the row maximum has
 // grown by more than TAU (log2 units); P then stays below 2^TAU and O, which
 // accumulates in TMEM across tiles, is rescaled in place only on such moves.
 constexpr float TAU = 8.0f;
+
+// Slot `sl` (columns [sl*sw, sl*sw + sw), sw = kx/2) of row `row` of the slab
+// [Q U_va | Q U_vb] for one tile: (U_v^T q) for version v, zeros when v < 0 or
+// past r.
+__device__ __forceinline__ void build_ax(const TcArgs& A, uint8_t* slab, int row, int64_t q,
+                                         int v, int sl) {
+  const Dims& Dm = A.Dm;
+  const int r = Dm.r, kx = A.kx, sw = kx / 2, h = blockIdx.y;
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
+  if (q < A.nq && v >= 0) {
+    const uint4* qrow = reinterpret_cast<const uint4*>(A.Q + ((size_t)q * Dm.H + h) * DH);
+    const float* Uv = basis_of(A.v, Dm, v, h);
+    for (int c = 0; c < 16; ++c) {
+      const uint4 w = __ldg(qrow + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float qv = __uint_as_float(e & 1 ? (ww[e / 2] & 0xffff0000u) : (ww[e / 2] << 16));
+        const float* Uj = Uv + (c * 8 + e) * r;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (k < r) acc[k] = fmaf(qv, __ldg(Uj + k), acc[k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (c < sw / 8)
+      *reinterpret_cast<uint4*>(slab + xslab_off(row, sl * (sw / 8) + c, kx)) = make_uint4(
+          pack_bf16(acc[8 * c], acc[8 * c + 1]), pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
+          pack_bf16(acc[8 * c + 4], acc[8 * c + 5]), pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
+  }
+}
+
+__device__ __forceinline__ void build_ax_pair(const TcArgs& A, uint8_t* slab, int row, int64_t q,
+                                              int va, int vb) {
+  build_ax(A, slab, row, q, va, 0);
+  build_ax(A, slab, row, q, vb != va ? vb : -1, 1);
+}
 
 __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              uint32_t tmem, int ntile) {
@@ -119,8 +189,23 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
       *reinterpret_cast<uint4*>(smem + OFF_Q + sw128_off(row, c, BQ)) = val;
     }
   }
+  // (va, vb) pair held by slab buffer 0 and 1, packed as va | vb << 16
+  uint32_t ax_pair0 = 0xffffffffu, ax_pair1 = 0xffffffffu;
+  if (A.kx) {
+    for (int j = 0; j < 2 && j < ntile; ++j) {
+      int va, vb;
+      tile_versions(A.v.tokver, A.T, j, va, vb);
+      build_ax_pair(A, smem + OFF_AX + j * XSLAB, row, q, va, vb);
+      if (j == 0) ax_pair0 = (uint32_t)va | ((uint32_t)vb << 16);
+      else ax_pair1 = (uint32_t)va | ((uint32_t)vb << 16);
+    }
+  }
   fence_proxy_async_smem();
   mbar_arrive(&bars[B_Q_READY]);
+  if (A.kx) {
+    mbar_arrive(&bars[B_AX_FULL + 0]);
+    if (ntile > 1) mbar_arrive(&bars[B_AX_FULL + 1]);
+  }
 
   float m_used = -INFINITY, l = 0.0f;
   const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
@@ -147,15 +232,15 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     if (j == 0) {
       m_used = m_row;
     } else {
+      // P V' of tile j-1 must be done before P is overwritten and before O is
+      // touched.  S_FULL(j) implies P V' of tile j-2 is done (commits track all
+      // earlier MMAs) and P V' of tile j cannot start before P_FULL(j), so
+      // O_FULL sits in phase j-1 or j and the parity test is exact.
+      bool w2 = mbar_wait(&bars[B_O_FULL], (j - 1) & 1);
+      if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+      tc_fence_after();
       const bool need = m_row > m_used + TAU;
       if (__any_sync(0xffffffffu, need)) {
-        // O holds P V' of tiles < j: wait for the last of them, then rescale.
-        // S_FULL(j) already implies P V' of tile j-2 is done (commits track all
-        // earlier MMAs) and P V' of tile j cannot start before P_FULL(j), so
-        // the barrier sits in phase j-1 or j and the parity test is exact.
-        bool w2 = mbar_wait(&bars[B_O_FULL], (j - 1) & 1);
-        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-        tc_fence_after();
         const float f = need ? ex2(m_used - m_row) : 1.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -170,7 +255,7 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
       }
     }
     float lsum = 0.0f;
-    uint8_t* pb = smem + OFF_P + b * TILE;
+    uint8_t* pb = smem + OFF_P;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float s[32];
@@ -178,8 +263,8 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        float p0 = (c * 32 + e < nvalid) ? ex2(fmaf(s[e], sl2, -m_used)) : 0.0f;
-        float p1 = (c * 32 + e + 1 < nvalid) ? ex2(fmaf(s[e + 1], sl2, -m_used)) : 0.0f;
+        const float p0 = (c * 32 + e < nvalid) ? ex2(fmaf(s[e], sl2, -m_used)) : 0.0f;
+        const float p1 = (c * 32 + e + 1 < nvalid) ? ex2(fmaf(s[e + 1], sl2, -m_used)) : 0.0f;
         lsum += p0 + p1;
         pk[e / 2] = pack_bf16(p0, p1);
       }
@@ -192,7 +277,20 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     tc_fence_before();
     mbar_arrive(&bars[B_S_FREE + b]);
     fence_proxy_async_smem();
-    mbar_arrive(&bars[B_P_FULL + b]);
+    mbar_arrive(&bars[B_P_FULL]);
+    // slab for tile j+2 into buffer b (QK^T of tile j, its last reader, is done)
+    if (A.kx && j + 2 < ntile) {
+      int va, vb;
+      tile_versions(A.v.tokver, A.T, j + 2, va, vb);
+      const uint32_t pair = (uint32_t)va | ((uint32_t)vb << 16);
+      if (pair != (b ? ax_pair1 : ax_pair0)) {
+        build_ax_pair(A, smem + OFF_AX + b * XSLAB, row, q, va, vb);
+        if (b) ax_pair1 = pair;
+        else ax_pair0 = pair;
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&bars[B_AX_FULL + b]);
+    }
   }
   if (ok) {
     bool w = mbar_wait(&bars[B_O_LAST], 0);
@@ -221,41 +319,71 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
 }
 
 // ------------------------------------------------------------------ dequant role
-__device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars, int ntile) {
+// exact float of a 2-bit code: (2^23 + code) - 2^23
+__device__ __forceinline__ float code_f(uint32_t bits, int e) {
+  return __uint_as_float(0x4B000000u | ((bits >> (2 * e)) & 3u)) - 8388608.0f;
+}
+
+__device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
+                                             int ntile) {
   const int dt = threadIdx.x - 128;  // key row in the tile
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead p = packed_head(A.v, Dm, h);
-  const int G = Dm.G, ng = Dm.ng, r = Dm.r;
+  const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
   for (int j = 0; j < ntile; ++j) {
     const int slot = j & 1;
-    if (j >= 2) {
-      if (!mbar_wait(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1)) {
-        timeout_flag();
-        return;
-      }
+    if (j >= 2 && !mbar_wait_sleep(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1)) {
+      timeout_flag();
+      return;
     }
     uint8_t* kb = smem + OFF_K + slot * TILE;
     uint8_t* vb = smem + OFF_V + slot * TILE;
+    uint8_t* xb = smem + OFF_BX + slot * XSLAB;
     const int64_t t = (int64_t)j * KT + dt;
     if (t < A.T) {
       const int a = load_idx(p.k_idx, t, Dm.idx_bytes);
       const int bi = load_idx(p.v_idx, t, Dm.idx_bytes);
-      const float* U = basis_of(A.v, Dm, A.v.tokver[t], h);
+      const int ver = A.v.tokver[t];
+      bool fallback = false;
       float chat[16];
-      const float cs = h2f(p.k_cscale[t]);
 #pragma unroll
-      for (int qq = 0; qq < 16; ++qq) chat[qq] = (qq < r) ? (float)p.k_coef[t * r + qq] * cs : 0.0f;
-      const uint4* kc4 = reinterpret_cast<const uint4*>(p.k_codes + t * (DH / 4));
-      const uint4* vc4 = reinterpret_cast<const uint4*>(p.v_codes + t * (DH / 4));
-      uint32_t kcode[8], vcode[8];
-      {
-        uint4 x0 = __ldg(kc4), x1 = __ldg(kc4 + 1), y0 = __ldg(vc4), y1 = __ldg(vc4 + 1);
-        kcode[0] = x0.x; kcode[1] = x0.y; kcode[2] = x0.z; kcode[3] = x0.w;
-        kcode[4] = x1.x; kcode[5] = x1.y; kcode[6] = x1.z; kcode[7] = x1.w;
-        vcode[0] = y0.x; vcode[1] = y0.y; vcode[2] = y0.z; vcode[3] = y0.w;
-        vcode[4] = y1.x; vcode[5] = y1.y; vcode[6] = y1.z; vcode[7] = y1.w;
+      for (int k = 0; k < 16; ++k) chat[k] = 0.0f;
+      if (r > 0) {
+        int va, vbv;
+        tile_versions(A.v.tokver, A.T, j, va, vbv);
+        const float cs = h2f(p.k_cscale[t]);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (k < r) chat[k] = (float)p.k_coef[t * r + k] * cs;
+        fallback = (ver != va) && (ver != vbv);
+        // compensation slab row: c8 cs in the slot of the key's version
+        const int sw = kx / 2;
+        const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < kx / 8) {
+            const int cs0 = c - (sl >= 0 ? sl * (sw / 8) : 0);
+            const bool mine = sl >= 0 && cs0 >= 0 && cs0 < sw / 8;
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float v = 0.0f;
+#pragma unroll
+              for (int m = 0; m < 16; ++m)
+                if (mine && m == cs0 * 8 + e) v = chat[m];
+              x[e] = v;
+            }
+            *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) =
+                make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                           pack_bf16(x[6], x[7]));
+          }
+        }
       }
+      const float* U = basis_of(A.v, Dm, ver, h);
+      const uint32_t* kc32 = reinterpret_cast<const uint32_t*>(p.k_codes + t * (DH / 4));
+      const uint32_t* vc32 = reinterpret_cast<const uint32_t*>(p.v_codes + t * (DH / 4));
+      uint32_t kword = 0, vword = 0;
       const uint32_t* kpar = reinterpret_cast<const uint32_t*>(p.k_params) + t * ng;
       const uint32_t* vpar = reinterpret_cast<const uint32_t*>(p.v_params) + t * ng;
       const uint4* ck = reinterpret_cast<const uint4*>(p.cent_k + (size_t)a * DH);
@@ -267,49 +395,38 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
         const uint32_t kp = __ldg(kpar + g), vp = __ldg(vpar + g);
         const float kmn = h2f((uint16_t)(kp & 0xffff)), ksc = h2f((uint16_t)(kp >> 16));
         const float vmn = h2f((uint16_t)(vp & 0xffff)), vsc = h2f((uint16_t)(vp >> 16));
-        const uint32_t kbits = (kcode[c / 2] >> (16 * (c & 1))) & 0xffff;
-        const uint32_t vbits = (vcode[c / 2] >> (16 * (c & 1))) & 0xffff;
+        if ((c & 1) == 0) {
+          kword = __ldg(kc32 + c / 2);
+          vword = __ldg(vc32 + c / 2);
+        }
+        const uint32_t kbits = (kword >> (16 * (c & 1))) & 0xffff;
+        const uint32_t vbits = (vword >> (16 * (c & 1))) & 0xffff;
         const uint4 kcv = __ldg(ck + c), vcv = __ldg(cv + c);
         const uint32_t kw[4] = {kcv.x, kcv.y, kcv.z, kcv.w};
         const uint32_t vw[4] = {vcv.x, vcv.y, vcv.z, vcv.w};
-        float kx[8], vx[8];
+        float kxv[8], vxv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float kc = __uint_as_float(e & 1 ? (kw[e / 2] & 0xffff0000u) : (kw[e / 2] << 16));
           const float vc = __uint_as_float(e & 1 ? (vw[e / 2] & 0xffff0000u) : (vw[e / 2] << 16));
-          kx[e] = kc + fmaf((float)((kbits >> (2 * e)) & 3), ksc, kmn);
-          vx[e] = vc + fmaf((float)((vbits >> (2 * e)) & 3), vsc, vmn);
+          kxv[e] = kc + fmaf(code_f(kbits, e), ksc, kmn);
+          vxv[e] = vc + fmaf(code_f(vbits, e), vsc, vmn);
         }
-        if (r > 0) {
-#pragma unroll
+        if (fallback) {  // a third basis version in this tile: compensate here
           for (int e = 0; e < 8; ++e) {
-            const float* Uj = U + (size_t)(j0 + e) * r;
             float corr = 0.0f;
-            if (r == 8) {
-              const float4 u0 = __ldg(reinterpret_cast<const float4*>(Uj));
-              const float4 u1 = __ldg(reinterpret_cast<const float4*>(Uj) + 1);
-              corr = fmaf(u0.x, chat[0], corr);
-              corr = fmaf(u0.y, chat[1], corr);
-              corr = fmaf(u0.z, chat[2], corr);
-              corr = fmaf(u0.w, chat[3], corr);
-              corr = fmaf(u1.x, chat[4], corr);
-              corr = fmaf(u1.y, chat[5], corr);
-              corr = fmaf(u1.z, chat[6], corr);
-              corr = fmaf(u1.w, chat[7], corr);
-            } else {
 #pragma unroll
-              for (int qq = 0; qq < 16; ++qq)
-                if (qq < r) corr = fmaf(__ldg(Uj + qq), chat[qq], corr);
-            }
-            kx[e] += corr;
+            for (int k = 0; k < 16; ++k)
+              if (k < r) corr = fmaf(__ldg(U + (size_t)(j0 + e) * r + k), chat[k], corr);
+            kxv[e] += corr;
           }
         }
         *reinterpret_cast<uint4*>(kb + sw128_off(dt, c, KT)) =
-            make_uint4(pack_bf16(kx[0], kx[1]), pack_bf16(kx[2], kx[3]),
-                       pack_bf16(kx[4], kx[5]), pack_bf16(kx[6], kx[7]));
+            make_uint4(pack_bf16(kxv[0], kxv[1]), pack_bf16(kxv[2], kxv[3]),
+                       pack_bf16(kxv[4], kxv[5]), pack_bf16(kxv[6], kxv[7]));
         *reinterpret_cast<uint4*>(vb + sw128_off(dt, c, KT)) =
-            make_uint4(pack_bf16(vx[0], vx[1]), pack_bf16(vx[2], vx[3]),
-                       pack_bf16(vx[4], vx[5]), pack_bf16(vx[6], vx[7]));
+            make_uint4(pack_bf16(vxv[0], vxv[1]), pack_bf16(vxv[2], vxv[3]),
+                       pack_bf16(vxv[4], vxv[5]), pack_bf16(vxv[6], vxv[7]));
       }
     } else {
 #pragma unroll
@@ -317,48 +434,57 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
         *reinterpret_cast<uint4*>(kb + sw128_off(dt, c, KT)) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(vb + sw128_off(dt, c, KT)) = make_uint4(0, 0, 0, 0);
       }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < kx / 8)
+          *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     mbar_arrive(&bars[B_KV_FULL + slot]);
   }
 }
 
-// S[j&1] = Q K'_j^T: 8 K-steps of 16 over head_dim (two 64-wide swizzled blocks).
-__device__ __forceinline__ bool issue_qk(uint64_t* bars, uint32_t sq, uint32_t sk, uint32_t tmem,
-                                         int j) {
+// ------------------------------------------------------------------ MMA role
+// S[j&1] = Q K-hat_j^T (8 K16 steps over head_dim, two 64-wide swizzled blocks)
+// + the compensation steps [Q U_va | Q U_vb] [c slots]^T.
+__device__ __forceinline__ bool issue_qk(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
+                                         int kx) {
   constexpr uint32_t IDQ = idesc_bf16(128, 128, false, false);
   const int slot = j & 1;
   if (!mbar_wait(&bars[B_KV_FULL + slot], (j >> 1) & 1)) return false;
+  if (kx && !mbar_wait(&bars[B_AX_FULL + slot], (j >> 1) & 1)) return false;
   if (j >= 2 && !mbar_wait(&bars[B_S_FREE + slot], ((j - 2) >> 1) & 1)) return false;
   tc_fence_after();
+  const uint32_t sq = sbase + OFF_Q, sk = sbase + OFF_K + slot * TILE;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint32_t koff = (k >> 2) * (128 * 128) + (k & 3) * 32;
-    const uint64_t da = desc_sw128(sq + koff, 16, 1024);
-    const uint64_t db = desc_sw128(sk + slot * TILE + koff, 16, 1024);
-    mma_bf16_ss(tmem + slot * 128, da, db, IDQ, k > 0);
+    mma_bf16_ss(tmem + slot * 128, desc_sw128(sq + koff, 16, 1024),
+                desc_sw128(sk + koff, 16, 1024), IDQ, k > 0);
   }
+  const uint32_t sa = sbase + OFF_AX + slot * XSLAB, sb = sbase + OFF_BX + slot * XSLAB;
+  for (int k = 0; k < kx / 16; ++k)
+    mma_bf16_ss(tmem + slot * 128, desc_noswz(sa + k * 256, 128, kx * 16),
+                desc_noswz(sb + k * 256, 128, kx * 16), IDQ, 1u);
   mma_commit(&bars[B_S_FULL + slot]);
   return true;
 }
 
-// ------------------------------------------------------------------ MMA role
-__device__ __forceinline__ void mma_role(uint8_t* smem, uint64_t* bars, uint32_t tmem, int ntile) {
+__device__ __forceinline__ void mma_role(uint8_t* smem, uint64_t* bars, uint32_t tmem, int ntile,
+                                         int kx) {
   constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);
-  const uint32_t sq = smem_u32(smem + OFF_Q);
-  const uint32_t sk = smem_u32(smem + OFF_K);
-  const uint32_t sv = smem_u32(smem + OFF_V);
-  const uint32_t sp = smem_u32(smem + OFF_P);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sv = sbase + OFF_V, sp = sbase + OFF_P;
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
-  if (ok) ok = issue_qk(bars, sq, sk, tmem, 0);
+  if (ok) ok = issue_qk(bars, sbase, tmem, 0, kx);
   for (int j = 0; ok && j < ntile; ++j) {
-    if (j + 1 < ntile && !(ok = issue_qk(bars, sq, sk, tmem, j + 1))) break;
+    if (j + 1 < ntile && !(ok = issue_qk(bars, sbase, tmem, j + 1, kx))) break;
     const int b = j & 1;
-    if (!mbar_wait(&bars[B_P_FULL + b], (j >> 1) & 1)) { ok = false; break; }
+    if (!mbar_wait(&bars[B_P_FULL], j & 1)) { ok = false; break; }
     tc_fence_after();
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint64_t da = desc_sw128(sp + b * TILE + (k >> 2) * (BQ * 128) + (k & 3) * 32, 16, 1024);
+      const uint64_t da = desc_sw128(sp + (k >> 2) * (BQ * 128) + (k & 3) * 32, 16, 1024);
       const uint64_t db = desc_sw128(sv + b * TILE + k * 2048, KT * 128, 1024);
       mma_bf16_ss(tmem + 256, da, db, IDP, (j > 0 || k > 0) ? 1u : 0u);
     }
@@ -385,8 +511,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
       mbar_init(&bars[B_KV_EMPTY + i], 1);
       mbar_init(&bars[B_S_FULL + i], 1);
       mbar_init(&bars[B_S_FREE + i], 128);
-      mbar_init(&bars[B_P_FULL + i], 128);
+      mbar_init(&bars[B_AX_FULL + i], 128);
     }
+    mbar_init(&bars[B_P_FULL], 128);
     mbar_init(&bars[B_O_FULL], 1);
     mbar_init(&bars[B_Q_READY], 128);
     mbar_init(&bars[B_DONE], 1);
@@ -406,7 +533,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   } else if (warp < 8) {
     dequant_role(A, smem, bars, ntile);
   } else if ((threadIdx.x & 31) == 0) {
-    mma_role(smem, bars, tmem, ntile);
+    mma_role(smem, bars, tmem, ntile, A.kx);
   }
   tc_fence_before();
   __syncthreads();
@@ -431,6 +558,7 @@ cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, co
   a.nq = nq;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
+  a.kx = (D.r == 0) ? 0 : (D.r <= 8 ? 16 : 32);  // two slots of 8 or 16 columns
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;

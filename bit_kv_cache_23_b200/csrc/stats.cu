@@ -12,15 +12,10 @@
 // added to the fp64 running sum, so the result does not depend on scheduling.
 //
 // refresh: s_j = M_jj / n, w_g = sum_{j in g} s_j (fp32 fold over the group),
-// U = top-r eigenvectors of A = M / n.  The eigenvectors come from one-sided
-// (Hestenes) Jacobi in fp64 on X = A V0, where V0 is the previous refresh's
-// eigenvector matrix (warm start: the statistics move little between frames,
-// so one or two sweeps usually suffice) or the identity.  Rotations are
-// applied to disjoint column pairs in round-robin order; at convergence the
-// columns of X are A v_k = lambda_k v_k (A is positive semi-definite), so
-// lambda_k = |x_k| and v_k = x_k / lambda_k.  Columns are ordered by
-// descending lambda (ties: lower column) and each U column is signed so that
-// its largest-magnitude entry (lowest index on ties) is positive.
+// U = top-r eigenvectors of A = M / n by block subspace iteration (see
+// refresh_kernel), warm-started from the previous refresh since the statistics
+// move little between frames.  Each U column is signed so that its
+// largest-magnitude entry (lowest index on ties) is positive.
 #include "common.cuh"
 
 namespace qwm {
@@ -69,47 +64,178 @@ __global__ void __launch_bounds__(256) stats_acc(const uint16_t* __restrict__ Q,
     }
 }
 
-// X0 (column-major [k][i]) = (M / n) V0 with V0 column-major (warm), or M / n
-// (cold; M is symmetric so its rows are its columns).
-__global__ void refresh_prep(const double* __restrict__ M, int64_t n, int d,
-                             const double* __restrict__ eigvec, const double* __restrict__ flags,
-                             double* __restrict__ X0) {
-  const int h = blockIdx.y;
-  const double* A = M + (size_t)h * d * d;
-  const double* V = eigvec + (size_t)h * d * d;
-  double* X = X0 + (size_t)h * d * d;
-  const bool warm = flags[h] != 0.0;
-  const double inv = 1.0 / (double)n;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < d * d; e += gridDim.x * blockDim.x) {
-    int k = e / d, i = e % d;
-    double v;
-    if (warm) {
+// Block subspace ("orthogonal") iteration for the top eigenvectors of the
+// symmetric positive semi-definite A = M / n, fp64, one CTA per head.  The
+// block X (d x p, p = 16 for r <= 8, else 32) starts from the previous
+// refresh's Ritz vectors (warm) or from the columns of A with the largest
+// diagonal (cold).  Each step orthonormalizes X by Cholesky-QR (twice) and
+// multiplies by A; it stops when the trace of Q^T A Q changes by less than
+// 1e-14 relative (or after a cap).  A final Rayleigh-Ritz step diagonalizes
+// H = Q^T A Q (p x p) by one-sided Jacobi; the Ritz vectors Q W, sorted by
+// descending Ritz value, give U (first r columns) and the next warm start.
+struct RefreshSmem {
+  double* A;   // [d][d+1] row-major, padded
+  double* X;   // [p][d+1] column-major (column k at X + k*(d+1))
+  double* Y;   // [p][d+1]
+  double* G;   // [p][p]  Gram / projected matrix (column-major for Jacobi)
+  double* L;   // [p][p]  Cholesky factor
+  double* th;  // [p]     Ritz values
+  int* ord;    // [p]
+  double* red; // [32]    block reduction scratch
+};
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int w = 0; w < (int)(blockDim.x / 32); ++w) t += red[w];
+  return t;
+}
+
+// Y = A X  (each warp takes columns, lanes take rows)
+__device__ void gemm_AX(const RefreshSmem& S, const double* X, double* Y, int d, int p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+  for (int k = warp; k < p; k += nw) {
+    const double* xk = X + k * (d + 1);
+    for (int i = lane; i < d; i += 32) {
+      const double* ai = S.A + i * (d + 1);
       double acc = 0.0;
-      for (int j = 0; j < d; ++j) acc += A[(size_t)i * d + j] * V[(size_t)k * d + j];
-      v = acc * inv;
-    } else {
-      v = A[(size_t)k * d + i] * inv;
+      for (int j = 0; j < d; ++j) acc = fma(ai[j], xk[j], acc);
+      Y[k * (d + 1) + i] = acc;
     }
-    X[e] = v;
+  }
+  __syncthreads();
+}
+
+// G = X^T Y (p x p); one warp per entry, lanes split the rows.
+__device__ void gram(const double* X, const double* Y, double* G, int d, int p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+  for (int e = warp; e < p * p; e += nw) {
+    const int a = e / p, b = e % p;
+    const double* xa = X + a * (d + 1);
+    const double* yb = Y + b * (d + 1);
+    double acc = 0.0;
+    for (int i = lane; i < d; i += 32) acc = fma(xa[i], yb[i], acc);
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) G[b * p + a] = acc;  // column-major
+  }
+  __syncthreads();
+}
+
+// One Cholesky-QR pass: X <- X R^-1 with R^T R = X^T X.  Columns whose pivot
+// vanishes (dependent columns) become zero.
+__device__ void cholqr(const RefreshSmem& S, double* X, int d, int p) {
+  gram(X, X, S.G, d, p);
+  if (threadIdx.x < 32) {
+    const int i = threadIdx.x;  // row of L owned by this lane
+    double tr = 0.0;
+    for (int k = 0; k < p; ++k) tr += S.G[k * p + k];
+    for (int k = 0; k < p; ++k) {
+      const double piv = S.G[k * p + k];
+      const bool ok = piv > 1e-26 * tr && piv > 0.0;
+      const double dkk = ok ? sqrt(piv) : 0.0;
+      if (i >= k && i < p) S.L[k * p + i] = ok ? S.G[k * p + i] / (i == k ? piv / dkk : dkk) : 0.0;
+      __syncwarp();
+      if (i > k && i < p) {
+        const double lik = S.L[k * p + i];
+        for (int j = k + 1; j <= i; ++j) S.G[j * p + i] -= lik * S.L[k * p + j];
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // rows of X: solve y R = x with R = L^T (forward substitution over columns)
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    double y[32];
+    for (int k = 0; k < p; ++k) {
+      double v = X[k * (d + 1) + i];
+      for (int m = 0; m < k; ++m) v -= y[m] * S.L[m * p + k];
+      const double lkk = S.L[k * p + k];
+      y[k] = (lkk != 0.0) ? v / lkk : 0.0;
+    }
+    for (int k = 0; k < p; ++k) X[k * (d + 1) + i] = y[k];
+  }
+  __syncthreads();
+}
+
+// One-sided Jacobi on the p x p column-major matrix G (positive semi-definite):
+// rotate column pairs until orthogonal; 8 threads per pair.  Also applies the
+// rotations to W (p x p, column-major, starts as the identity).
+__device__ void small_jacobi(double* G, double* W, int p, double* red) {
+  const int tid = threadIdx.x;
+  const int grp = tid / 8, sub = tid % 8;
+  const int npairs = p / 2;
+  for (int e = tid; e < p * p; e += blockDim.x) W[e] = ((e / p) == (e % p)) ? 1.0 : 0.0;
+  __syncthreads();
+  for (int sweep = 0; sweep < 30; ++sweep) {
+    float worst = 0.0f;
+    for (int rnd = 0; rnd < p - 1; ++rnd) {
+      if (grp < npairs) {
+        const int a = (grp == 0) ? 0 : 1 + (grp - 1 + rnd) % (p - 1);
+        const int bb = 1 + (p - 1 - grp - 1 + rnd) % (p - 1);
+        const int pp = min(a, bb), qq = max(a, bb);
+        double* gp = G + pp * p;
+        double* gq = G + qq * p;
+        double al = 0.0, be = 0.0, ga = 0.0;
+        for (int i = sub; i < p; i += 8) {
+          al += gp[i] * gp[i];
+          be += gq[i] * gq[i];
+          ga += gp[i] * gq[i];
+        }
+        for (int o = 4; o >= 1; o >>= 1) {
+          al += __shfl_xor_sync(0xffffffffu, al, o);
+          be += __shfl_xor_sync(0xffffffffu, be, o);
+          ga += __shfl_xor_sync(0xffffffffu, ga, o);
+        }
+        const double nrm = sqrt(al * be);
+        if (ga != 0.0 && fabs(ga) > 1e-15 * nrm) {
+          worst = fmaxf(worst, (float)(fabs(ga) / nrm));
+          const double zeta = (be - al) / (2.0 * ga);
+          const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
+          const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
+          double* wp = W + pp * p;
+          double* wq = W + qq * p;
+          for (int i = sub; i < p; i += 8) {
+            const double u = gp[i], v = gq[i];
+            gp[i] = c * u - s * v;
+            gq[i] = s * u + c * v;
+            const double wu = wp[i], wv = wq[i];
+            wp[i] = c * wu - s * wv;
+            wq[i] = s * wu + c * wv;
+          }
+        }
+      }
+      __syncthreads();
+    }
+    const double wmax = -block_sum(-0.0, red);  // keeps every thread in step
+    (void)wmax;
+    for (int o = 16; o >= 1; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+    __syncthreads();
+    if ((tid & 31) == 0) red[tid / 32] = worst;
+    __syncthreads();
+    float m = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) m = fmaxf(m, (float)red[w]);
+    __syncthreads();
+    if (m <= 1e-13f) break;
   }
 }
 
-// One CTA per head, 4*d threads (8 per column pair).
-__global__ void refresh_jacobi(const double* __restrict__ M, int64_t n, int d, int G, int r,
-                               const double* __restrict__ X0, float* __restrict__ sens,
-                               float* __restrict__ wgroup, float* __restrict__ basis_slot,
-                               double* __restrict__ eigvec, double* __restrict__ flags, int H) {
-  extern __shared__ double X[];  // [d][d] column-major
-  __shared__ double lam[128];
-  __shared__ int order[128];
-  __shared__ float sred[32];
-  __shared__ int sweeps_done;
+// One CTA per head, 512 threads.
+__global__ void __launch_bounds__(512) refresh_kernel(const double* __restrict__ Mall, int64_t n,
+                                                      int d, int G, int r, int p,
+                                                      float* __restrict__ sens,
+                                                      float* __restrict__ wgroup,
+                                                      float* __restrict__ basis_slot,
+                                                      double* __restrict__ eigvec,
+                                                      double* __restrict__ flags) {
+  extern __shared__ double sm[];
   const int h = blockIdx.x;
   const int tid = threadIdx.x, nt = blockDim.x;
   float* s_out = sens + (size_t)h * d;
   float* w_out = wgroup + (size_t)h * (d / G);
   float* U = basis_slot + (size_t)h * d * (r > 0 ? r : 1);
-
   if (n <= 0) {
     for (int j = tid; j < d; j += nt) s_out[j] = 1.0f;
     for (int e = tid; e < d * r; e += nt) U[e] = 0.0f;
@@ -121,126 +247,126 @@ __global__ void refresh_jacobi(const double* __restrict__ M, int64_t n, int d, i
     }
     return;
   }
-  const double* A = M + (size_t)h * d * d;
-  for (int j = tid; j < d; j += nt) s_out[j] = __double2float_rn(A[(size_t)j * d + j] / (double)n);
-  for (int e = tid; e < d * d; e += nt) X[e] = X0[(size_t)h * d * d + e];
+  RefreshSmem S;
+  S.A = sm;
+  S.X = S.A + d * (d + 1);
+  S.Y = S.X + p * (d + 1);
+  S.G = S.Y + p * (d + 1);
+  S.L = S.G + p * p;
+  S.th = S.L + p * p;
+  S.red = S.th + p;
+  S.ord = reinterpret_cast<int*>(S.red + 32);
+  const double* M = Mall + (size_t)h * d * d;
+  const double inv = 1.0 / (double)n;
+  for (int e = tid; e < d * d; e += nt) S.A[(e / d) * (d + 1) + (e % d)] = M[e] * inv;
+  for (int j = tid; j < d; j += nt) s_out[j] = __double2float_rn(M[(size_t)j * d + j] / (double)n);
   __syncthreads();
   if (tid < d / G) {
     float acc = 0.0f;
     for (int j = tid * G; j < (tid + 1) * G; ++j) acc = __fadd_rn(acc, s_out[j]);
     w_out[tid] = acc;
   }
-
-  const int grp = tid / 8, sub = tid % 8;  // pair slot, lane within the pair group
-  const int npairs = d / 2;
-  const double tol = 1e-13;
-  for (int sweep = 0; sweep < 40; ++sweep) {
-    float worst = 0.0f;
-    for (int rnd = 0; rnd < d - 1; ++rnd) {
-      if (grp < npairs) {
-        // circle method: position 0 fixed, the others rotate by `rnd`
-        int a = (grp == 0) ? 0 : 1 + (grp - 1 + rnd) % (d - 1);
-        int bpos = d - 1 - grp;
-        int b = 1 + (bpos - 1 + rnd) % (d - 1);
-        int p = min(a, b), q = max(a, b);
-        double* xp = X + (size_t)p * d;
-        double* xq = X + (size_t)q * d;
-        double al = 0.0, be = 0.0, ga = 0.0;
-        for (int i = sub; i < d; i += 8) {
-          double u = xp[i], v = xq[i];
-          al += u * u;
-          be += v * v;
-          ga += u * v;
-        }
-        for (int o = 4; o >= 1; o >>= 1) {
-          al += __shfl_xor_sync(0xffffffffu, al, o);
-          be += __shfl_xor_sync(0xffffffffu, be, o);
-          ga += __shfl_xor_sync(0xffffffffu, ga, o);
-        }
-        double nrm = sqrt(al * be);
-        if (ga != 0.0 && fabs(ga) > tol * nrm) {
-          worst = fmaxf(worst, (float)(fabs(ga) / nrm));
-          double zeta = (be - al) / (2.0 * ga);
-          double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-          double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
-          for (int i = sub; i < d; i += 8) {
-            double u = xp[i], v = xq[i];
-            xp[i] = c * u - s * v;
-            xq[i] = s * u + c * v;
-          }
-        }
+  // ---- starting block
+  const double* Vprev = eigvec + (size_t)h * d * d;
+  const bool warm = flags[h] != 0.0;
+  if (warm) {
+    for (int e = tid; e < p * d; e += nt) S.X[(e / d) * (d + 1) + (e % d)] = Vprev[e];
+  } else {
+    // columns of A with the p largest diagonal entries (ties: lower index)
+    if (tid < d) {
+      const double v = S.A[tid * (d + 1) + tid];
+      int rank = 0;
+      for (int j = 0; j < d; ++j) {
+        const double u = S.A[j * (d + 1) + j];
+        rank += (u > v) || (u == v && j < tid);
       }
-      __syncthreads();
-    }
-    // block max of the largest relative off-diagonal seen in this sweep
-    for (int o = 16; o >= 1; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
-    if (tid % 32 == 0) sred[tid / 32] = worst;
-    __syncthreads();
-    if (tid == 0) {
-      float m = 0.0f;
-      for (int w = 0; w < nt / 32; ++w) m = fmaxf(m, sred[w]);
-      sweeps_done = (m <= 1e-12f) ? 1 : 0;
+      if (rank < p) S.ord[rank] = tid;
     }
     __syncthreads();
-    if (sweeps_done) break;
-    __syncthreads();
+    for (int e = tid; e < p * d; e += nt) {
+      const int k = e / d, i = e % d;
+      S.X[k * (d + 1) + i] = S.A[i * (d + 1) + S.ord[k]];
+    }
   }
-  // eigenvalues as column norms (each 8-lane group handles d/(nt/8) = 2 columns)
-  for (int k = grp; k < d; k += nt / 8) {
+  __syncthreads();
+  // ---- orthogonal iteration
+  double prev = -1.0;
+  const int maxit = warm ? 24 : 200;
+  for (int it = 0; it < maxit; ++it) {
+    cholqr(S, S.X, d, p);
+    cholqr(S, S.X, d, p);
+    gemm_AX(S, S.X, S.Y, d, p);
+    double part = 0.0;
+    for (int e = tid; e < p * d; e += nt) {
+      const int k = e / d, i = e % d;
+      part += S.X[k * (d + 1) + i] * S.Y[k * (d + 1) + i];
+    }
+    const double tr = block_sum(part, S.red);
+    const bool done = (prev >= 0.0) && fabs(tr - prev) <= 1e-14 * fabs(tr);
+    prev = tr;
+    // X <- A X for the next step
+    for (int e = tid; e < p * d; e += nt) {
+      const int k = e / d, i = e % d;
+      S.X[k * (d + 1) + i] = S.Y[k * (d + 1) + i];
+    }
+    __syncthreads();
+    if (done) break;
+  }
+  // ---- Rayleigh-Ritz on the final block
+  cholqr(S, S.X, d, p);
+  cholqr(S, S.X, d, p);
+  gemm_AX(S, S.X, S.Y, d, p);
+  gram(S.X, S.Y, S.G, d, p);              // H = Q^T A Q (column-major, symmetric)
+  double* W = S.Y;                         // Y is free again: W [p][p] in its space
+  double* Hc = S.Y + p * p;                // copy of H to rotate
+  for (int e = tid; e < p * p; e += nt) Hc[e] = S.G[e];
+  __syncthreads();
+  small_jacobi(Hc, W, p, S.red);
+  __syncthreads();
+  if (tid < p) {
     double acc = 0.0;
-    for (int i = sub; i < d; i += 8) acc += X[(size_t)k * d + i] * X[(size_t)k * d + i];
-    for (int o = 4; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (sub == 0) lam[k] = sqrt(acc);
+    for (int i = 0; i < p; ++i) acc += Hc[tid * p + i] * Hc[tid * p + i];
+    S.th[tid] = sqrt(acc);
   }
   __syncthreads();
-  double lmax = 0.0;
-  for (int k = 0; k < d; ++k) lmax = fmax(lmax, lam[k]);
-  if (tid < d) {
-    double lk = lam[tid];
+  if (tid < p) {
+    const double v = S.th[tid];
     int rank = 0;
-    for (int j = 0; j < d; ++j) {
-      double lj = lam[j];
-      rank += (lj > lk) || (lj == lk && j < tid);
-    }
-    order[rank] = tid;
+    for (int j = 0; j < p; ++j) rank += (S.th[j] > v) || (S.th[j] == v && j < tid);
+    S.ord[rank] = tid;
   }
   __syncthreads();
-  const double floor_l = lmax * 1e-12;
-  // normalized eigenvectors -> eigvec (column-major, same column order as X)
-  for (int e = tid; e < d * d; e += nt) {
-    int k = e / d;
-    double lk = lam[k];
-    eigvec[(size_t)h * d * d + e] = (lk > floor_l) ? X[e] / lk : 0.0;
+  // Ritz vectors V = Q W (sorted), written to eigvec (column-major) for the
+  // next warm start; the first r columns, sign-normalized, are U.
+  double* Vout = eigvec + (size_t)h * d * d;
+  for (int e = tid; e < p * d; e += nt) {
+    const int c = e / d, i = e % d;
+    const int k = S.ord[c];
+    double acc = 0.0;
+    for (int m = 0; m < p; ++m) acc = fma(S.X[m * (d + 1) + i], W[k * p + m], acc);
+    Vout[(size_t)c * d + i] = acc;
   }
-  // U columns, sign-normalized; every 8-lane group runs the shuffles (r <= nt/8)
-  {
-    const int c = grp;
-    const bool act = c < r;
-    const int k = order[act ? c : 0];
-    const double lk = lam[k];
-    const double* x = X + (size_t)k * d;
+  __syncthreads();
+  const int lane = tid & 31, warp = tid / 32;
+  for (int c = warp; c < r; c += nt / 32) {
+    const double* v = Vout + (size_t)c * d;
     double big = -1.0;
     int arg = 0;
-    for (int i = sub; i < d; i += 8) {
-      double m = fabs(x[i]);
+    for (int i = lane; i < d; i += 32) {
+      const double m = fabs(v[i]);
       if (m > big) { big = m; arg = i; }
     }
-    for (int o = 4; o >= 1; o >>= 1) {
-      double ob = __shfl_xor_sync(0xffffffffu, big, o);
-      int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+    for (int o = 16; o >= 1; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, big, o);
+      const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
       if (ob > big || (ob == big && oa < arg)) { big = ob; arg = oa; }
     }
-    const double sg = (x[arg] < 0.0) ? -1.0 : 1.0;
-    if (act)
-      for (int i = sub; i < d; i += 8) {
-        double v = (lk > floor_l) ? sg * x[i] / lk : 0.0;
-        U[(size_t)i * r + c] = __double2float_rn(v);
-      }
+    const double sg = (v[arg] < 0.0) ? -1.0 : 1.0;
+    for (int i = lane; i < d; i += 32) U[(size_t)i * r + c] = __double2float_rn(sg * v[i]);
   }
   if (tid == 0) {
-    bool ok = lmax > 0.0;
-    for (int k = 0; k < d; ++k) ok = ok && (lam[k] > lmax * 1e-8);
-    flags[h] = ok ? 1.0 : 0.0;
+    const double t0 = S.th[S.ord[0]], tl = S.th[S.ord[p - 1]];
+    flags[h] = (t0 > 0.0 && tl > 1e-10 * t0) ? 1.0 : 0.0;
   }
 }
 
@@ -274,20 +400,20 @@ cudaError_t launch_stats_accumulate(const Dims& D, const uint16_t* Q, int64_t n,
   return cudaGetLastError();
 }
 
+int refresh_block(int d, int r) { return (r <= 8 ? 16 : 32) < d ? (r <= 8 ? 16 : 32) : d; }
+
 cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, int version,
                            int /*warm_hint*/, cudaStream_t s) {
   double* flags = v.eigvec + (size_t)D.H * D.d * D.d;
-  double* X0 = (double*)v.workspace;
   float* slot = v.basis + (size_t)version * D.H * D.d * (D.r > 0 ? D.r : 1);
-  if (n_total > 0) {
-    refresh_prep<<<dim3(16, D.H), 256, 0, s>>>(v.qstats, n_total, D.d, v.eigvec, flags, X0);
-  }
-  size_t smem = (size_t)D.d * D.d * sizeof(double);
+  const int p = refresh_block(D.d, D.r);
+  size_t smem = ((size_t)D.d * (D.d + 1) + 2 * (size_t)p * (D.d + 1) + 2 * p * p + p + 32) * 8 +
+                (size_t)p * 4 + 64;
   cudaError_t e =
-      cudaFuncSetAttribute(refresh_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(refresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  refresh_jacobi<<<D.H, 4 * D.d, smem, s>>>(v.qstats, n_total, D.d, D.G, D.r, X0, v.sens,
-                                            v.wgroup, slot, v.eigvec, flags, D.H);
+  refresh_kernel<<<D.H, 512, smem, s>>>(v.qstats, n_total, D.d, D.G, D.r, p, v.sens, v.wgroup,
+                                        slot, v.eigvec, flags);
   return cudaGetLastError();
 }
 

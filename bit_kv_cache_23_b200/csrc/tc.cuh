@@ -103,6 +103,32 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle (K-major core matrices of
+// 8 rows x 16 bytes; lbo = byte distance between the two K-adjacent core
+// matrices, sbo = byte distance between 8-row groups).
+__device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Bounded wait that backs off with nanosleep between polls; for waits that are
+// usually long (producers waiting for a free slot), so that spinning threads
+// leave issue slots to the working warps.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try(addr, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if (mbar_try(addr, parity)) return true;
+    if (clock64() - t0 > (1ll << 31)) return false;
+  }
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
                                                   bool b_mn_major) {
