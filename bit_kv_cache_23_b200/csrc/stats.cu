@@ -209,8 +209,6 @@ __device__ void small_jacobi(double* G, double* W, int p, double* red) {
       }
       __syncthreads();
     }
-    const double wmax = -block_sum(-0.0, red);  // keeps every thread in step
-    (void)wmax;
     for (int o = 16; o >= 1; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
     __syncthreads();
     if ((tid & 31) == 0) red[tid / 32] = worst;
