@@ -15,15 +15,16 @@
 // version is neither (a tile spanning more than two versions) is compensated
 // element-wise by the dequant thread instead.
 //
-// One CTA per (head, 128 query rows); 288 threads in three roles:
+// One CTA per (head, 128 query rows); 416 threads in three roles:
 //   warps 0-3  softmax: warp w owns TMEM lanes 32w..32w+31 = query rows; loads
 //              S from TMEM, online softmax in the log2 domain, writes P (bf16)
 //              to shared memory; rescales O in TMEM when a row max moves; builds
 //              the [Q U_va | Q U_vb] slab two tiles ahead.
-//   warps 4-7  dequant: thread i reconstructs key row i of each 128-key tile
-//              (K-hat and V', bf16) straight into the 128B-swizzled layout the
-//              UMMA descriptors read, plus the key's compensation slab row.
-//   warp 8     MMA: one thread issues S = Q K'^T and O += P V' (V' read
+//   warps 4-11 dequant: two threads per key row of each 128-key tile (64
+//              channels each) issue all their loads first, then write K-hat and
+//              V' (bf16) straight into the 128B-swizzled layout the UMMA
+//              descriptors read, plus the key's compensation slab row.
+//   warp 12    MMA: one thread issues S = Q K'^T and O += P V' (V' read
 //              MN-major) and commits to mbarriers.
 // K-hat/V' tiles, the slabs and S are double-buffered, so the QK^T of tile j+1
 // runs while the softmax works on tile j.  TMEM: S[2] at columns 0/128, O at
@@ -45,7 +46,8 @@ using namespace tc;
 constexpr int BQ = 128;        // query rows per CTA
 constexpr int KT = 128;        // keys per tile
 constexpr int DH = 128;        // head_dim handled here
-constexpr int NTHREADS = 288;
+constexpr int NTHREADS = 416;  // 4 softmax + 8 dequant + 1 MMA warps
+constexpr int NDQ = 256;       // dequant threads: two per key row
 constexpr uint32_t TILE = 128 * 128 * 2;   // one bf16 128x128 tile
 constexpr uint32_t XSLAB = 128 * 32 * 2;   // [128][<=32] bf16 compensation slab
 constexpr uint32_t OFF_Q = 0;
@@ -59,7 +61,7 @@ constexpr int NBAR = 16;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 
 enum {
-  B_KV_FULL = 0,  // [2] dequant (128) -> MMA
+  B_KV_FULL = 0,  // [2] dequant (256) -> MMA
   B_KV_EMPTY = 2, // [2] MMA commit -> dequant
   B_S_FULL = 4,   // [2] MMA commit -> softmax
   B_S_FREE = 6,   // [2] softmax (128) -> MMA
@@ -221,12 +223,12 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     const int nvalid = (int)((A.T - kb) < KT ? (A.T - kb) : KT);
     float mx = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tmem_ld32(trow + b * 128 + c * 32, s);
+    for (int c = 0; c < 2; ++c) {
+      float s[64];
+      tmem_ld64(trow + b * 128 + c * 64, s);
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (c * 32 + e < nvalid) mx = fmaxf(mx, s[e]);
+      for (int e = 0; e < 64; ++e)
+        if (c * 64 + e < nvalid) mx = fmaxf(mx, s[e]);
     }
     const float m_row = mx * sl2;
     if (j == 0) {
@@ -257,21 +259,23 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     float lsum = 0.0f;
     uint8_t* pb = smem + OFF_P;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tmem_ld32(trow + b * 128 + c * 32, s);
-      uint32_t pk[16];
+    for (int c = 0; c < 2; ++c) {
+      float s[64];
+      tmem_ld64(trow + b * 128 + c * 64, s);
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const float p0 = (c * 32 + e < nvalid) ? ex2(fmaf(s[e], sl2, -m_used)) : 0.0f;
-        const float p1 = (c * 32 + e + 1 < nvalid) ? ex2(fmaf(s[e + 1], sl2, -m_used)) : 0.0f;
-        lsum += p0 + p1;
-        pk[e / 2] = pack_bf16(p0, p1);
+      for (int k = 0; k < 8; ++k) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const int col = c * 64 + k * 8 + e;
+          const float p0 = (col < nvalid) ? ex2(fmaf(s[k * 8 + e], sl2, -m_used)) : 0.0f;
+          const float p1 = (col + 1 < nvalid) ? ex2(fmaf(s[k * 8 + e + 1], sl2, -m_used)) : 0.0f;
+          lsum += p0 + p1;
+          pk[e / 2] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(pb + sw128_off(row, c * 8 + k, BQ)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<uint4*>(pb + sw128_off(row, c * 4 + k, BQ)) =
-            make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
     }
     l += lsum;
     tc_fence_before();
@@ -326,7 +330,9 @@ __device__ __forceinline__ float code_f(uint32_t bits, int e) {
 
 __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              int ntile) {
-  const int dt = threadIdx.x - 128;  // key row in the tile
+  const int dq = threadIdx.x - 128;  // 0..255
+  const int dt = dq >> 1;            // key row in the tile
+  const int hf = dq & 1;             // channel half [64 hf, 64 hf + 64)
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead p = packed_head(A.v, Dm, h);
@@ -342,8 +348,21 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
     uint8_t* xb = smem + OFF_BX + slot * XSLAB;
     const int64_t t = (int64_t)j * KT + dt;
     if (t < A.T) {
+      // ---- all loads of this half-row first (memory-level parallelism)
       const int a = load_idx(p.k_idx, t, Dm.idx_bytes);
       const int bi = load_idx(p.v_idx, t, Dm.idx_bytes);
+      const uint4* ck = reinterpret_cast<const uint4*>(p.cent_k + (size_t)a * DH) + hf * 8;
+      const uint4* cv = reinterpret_cast<const uint4*>(p.cent_v + (size_t)bi * DH) + hf * 8;
+      uint4 kc[8], vc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        kc[c] = __ldg(ck + c);
+        vc[c] = __ldg(cv + c);
+      }
+      const uint4 kw4 = __ldg(reinterpret_cast<const uint4*>(p.k_codes + t * (DH / 4)) + hf);
+      const uint4 vw4 = __ldg(reinterpret_cast<const uint4*>(p.v_codes + t * (DH / 4)) + hf);
+      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(p.k_params) + t * ng;
+      const uint32_t* vpar = reinterpret_cast<const uint32_t*>(p.v_params) + t * ng;
       const int ver = A.v.tokver[t];
       bool fallback = false;
       float chat[16];
@@ -352,65 +371,60 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
       if (r > 0) {
         int va, vbv;
         tile_versions(A.v.tokver, A.T, j, va, vbv);
-        const float cs = h2f(p.k_cscale[t]);
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (k < r) chat[k] = (float)p.k_coef[t * r + k] * cs;
         fallback = (ver != va) && (ver != vbv);
-        // compensation slab row: c8 cs in the slot of the key's version
-        const int sw = kx / 2;
-        const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
+        if (hf == 0 || fallback) {
+          const float cs = h2f(p.k_cscale[t]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < kx / 8) {
-            const int cs0 = c - (sl >= 0 ? sl * (sw / 8) : 0);
-            const bool mine = sl >= 0 && cs0 >= 0 && cs0 < sw / 8;
-            float x[8];
+          for (int k = 0; k < 16; ++k)
+            if (k < r) chat[k] = (float)p.k_coef[t * r + k] * cs;
+        }
+        if (hf == 0) {
+          // compensation slab row: c8 cs in the slot of the key's version
+          const int sw = kx / 2;
+          const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float v = 0.0f;
+          for (int c = 0; c < 4; ++c) {
+            if (c < kx / 8) {
+              const int cs0 = c - (sl >= 0 ? sl * (sw / 8) : 0);
+              const bool mine = sl >= 0 && cs0 >= 0 && cs0 < sw / 8;
+              float x[8];
 #pragma unroll
-              for (int m = 0; m < 16; ++m)
-                if (mine && m == cs0 * 8 + e) v = chat[m];
-              x[e] = v;
+              for (int e = 0; e < 8; ++e) {
+                float v = 0.0f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                  if (mine && m == cs0 * 8 + e) v = chat[m];
+                x[e] = v;
+              }
+              *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) =
+                  make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                             pack_bf16(x[6], x[7]));
             }
-            *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) =
-                make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                           pack_bf16(x[6], x[7]));
           }
         }
       }
       const float* U = basis_of(A.v, Dm, ver, h);
-      const uint32_t* kc32 = reinterpret_cast<const uint32_t*>(p.k_codes + t * (DH / 4));
-      const uint32_t* vc32 = reinterpret_cast<const uint32_t*>(p.v_codes + t * (DH / 4));
-      uint32_t kword = 0, vword = 0;
-      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(p.k_params) + t * ng;
-      const uint32_t* vpar = reinterpret_cast<const uint32_t*>(p.v_params) + t * ng;
-      const uint4* ck = reinterpret_cast<const uint4*>(p.cent_k + (size_t)a * DH);
-      const uint4* cv = reinterpret_cast<const uint4*>(p.cent_v + (size_t)bi * DH);
+      const uint32_t kwv[4] = {kw4.x, kw4.y, kw4.z, kw4.w};
+      const uint32_t vwv[4] = {vw4.x, vw4.y, vw4.z, vw4.w};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int cc = 0; cc < 8; ++cc) {
+        const int c = hf * 8 + cc;  // chunk of 8 channels within the row
         const int j0 = c * 8;
         const int g = j0 / G;
         const uint32_t kp = __ldg(kpar + g), vp = __ldg(vpar + g);
         const float kmn = h2f((uint16_t)(kp & 0xffff)), ksc = h2f((uint16_t)(kp >> 16));
         const float vmn = h2f((uint16_t)(vp & 0xffff)), vsc = h2f((uint16_t)(vp >> 16));
-        if ((c & 1) == 0) {
-          kword = __ldg(kc32 + c / 2);
-          vword = __ldg(vc32 + c / 2);
-        }
-        const uint32_t kbits = (kword >> (16 * (c & 1))) & 0xffff;
-        const uint32_t vbits = (vword >> (16 * (c & 1))) & 0xffff;
-        const uint4 kcv = __ldg(ck + c), vcv = __ldg(cv + c);
-        const uint32_t kw[4] = {kcv.x, kcv.y, kcv.z, kcv.w};
-        const uint32_t vw[4] = {vcv.x, vcv.y, vcv.z, vcv.w};
+        const uint32_t kbits = (kwv[cc / 2] >> (16 * (cc & 1))) & 0xffff;
+        const uint32_t vbits = (vwv[cc / 2] >> (16 * (cc & 1))) & 0xffff;
+        const uint32_t kw[4] = {kc[cc].x, kc[cc].y, kc[cc].z, kc[cc].w};
+        const uint32_t vw[4] = {vc[cc].x, vc[cc].y, vc[cc].z, vc[cc].w};
         float kxv[8], vxv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float kc = __uint_as_float(e & 1 ? (kw[e / 2] & 0xffff0000u) : (kw[e / 2] << 16));
-          const float vc = __uint_as_float(e & 1 ? (vw[e / 2] & 0xffff0000u) : (vw[e / 2] << 16));
-          kxv[e] = kc + fmaf(code_f(kbits, e), ksc, kmn);
-          vxv[e] = vc + fmaf(code_f(vbits, e), vsc, vmn);
+          const float kcf = __uint_as_float(e & 1 ? (kw[e / 2] & 0xffff0000u) : (kw[e / 2] << 16));
+          const float vcf = __uint_as_float(e & 1 ? (vw[e / 2] & 0xffff0000u) : (vw[e / 2] << 16));
+          kxv[e] = kcf + fmaf(code_f(kbits, e), ksc, kmn);
+          vxv[e] = vcf + fmaf(code_f(vbits, e), vsc, vmn);
         }
         if (fallback) {  // a third basis version in this tile: compensate here
           for (int e = 0; e < 8; ++e) {
@@ -430,14 +444,16 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        *reinterpret_cast<uint4*>(kb + sw128_off(dt, c, KT)) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(vb + sw128_off(dt, c, KT)) = make_uint4(0, 0, 0, 0);
+      for (int cc = 0; cc < 8; ++cc) {
+        *reinterpret_cast<uint4*>(kb + sw128_off(dt, hf * 8 + cc, KT)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(vb + sw128_off(dt, hf * 8 + cc, KT)) = make_uint4(0, 0, 0, 0);
       }
+      if (hf == 0) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < kx / 8)
-          *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 4; ++c)
+          if (c < kx / 8)
+            *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) = make_uint4(0, 0, 0, 0);
+      }
     }
     fence_proxy_async_smem();
     mbar_arrive(&bars[B_KV_FULL + slot]);
@@ -507,7 +523,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   const int ntile = (int)((A.T + KT - 1) / KT);
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[B_KV_FULL + i], 128);
+      mbar_init(&bars[B_KV_FULL + i], NDQ);
       mbar_init(&bars[B_KV_EMPTY + i], 1);
       mbar_init(&bars[B_S_FULL + i], 1);
       mbar_init(&bars[B_S_FREE + i], 128);
@@ -520,7 +536,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
     mbar_init(&bars[B_O_LAST], 1);
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -530,14 +546,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   const uint32_t tmem = *tmem_holder;
   if (warp < 4) {
     softmax_role(A, smem, bars, tmem, ntile);
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     dequant_role(A, smem, bars, ntile);
   } else if ((threadIdx.x & 31) == 0) {
     mma_role(smem, bars, tmem, ntile, A.kx);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -84,16 +84,6 @@ struct RefreshSmem {
   double* red; // [32]    block reduction scratch
 };
 
-__device__ __forceinline__ double block_sum(double v, double* red) {
-  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = v;
-  __syncthreads();
-  double t = 0.0;
-  for (int w = 0; w < (int)(blockDim.x / 32); ++w) t += red[w];
-  return t;
-}
-
 // Y = A X  (each warp takes columns, lanes take rows)
 __device__ void gemm_AX(const RefreshSmem& S, const double* X, double* Y, int d, int p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x / 32, nw = blockDim.x / 32;
@@ -124,19 +114,21 @@ __device__ void gram(const double* X, const double* Y, double* G, int d, int p) 
   __syncthreads();
 }
 
-// One Cholesky-QR pass: X <- X R^-1 with R^T R = X^T X.  Columns whose pivot
-// vanishes (dependent columns) become zero.
+// One Cholesky-QR pass: X <- X R^-1 with R^T R = X^T X (R = L^T).  One warp
+// factors the p x p Gram matrix and inverts L; then every thread applies
+// L^-1 to rows of X.  Columns whose pivot vanishes (dependent columns) become
+// zero.
 __device__ void cholqr(const RefreshSmem& S, double* X, int d, int p) {
   gram(X, X, S.G, d, p);
   if (threadIdx.x < 32) {
-    const int i = threadIdx.x;  // row of L owned by this lane
+    const int i = threadIdx.x;  // row owned by this lane
     double tr = 0.0;
     for (int k = 0; k < p; ++k) tr += S.G[k * p + k];
     for (int k = 0; k < p; ++k) {
       const double piv = S.G[k * p + k];
       const bool ok = piv > 1e-26 * tr && piv > 0.0;
       const double dkk = ok ? sqrt(piv) : 0.0;
-      if (i >= k && i < p) S.L[k * p + i] = ok ? S.G[k * p + i] / (i == k ? piv / dkk : dkk) : 0.0;
+      if (i >= k && i < p) S.L[k * p + i] = ok ? (i == k ? dkk : S.G[k * p + i] / dkk) : 0.0;
       __syncwarp();
       if (i > k && i < p) {
         const double lik = S.L[k * p + i];
@@ -144,18 +136,33 @@ __device__ void cholqr(const RefreshSmem& S, double* X, int d, int p) {
       }
       __syncwarp();
     }
+    // Linv (lower triangular) into G: lane c computes column c by forward
+    // substitution down the column, using only L and its own earlier entries
+    __syncwarp();
+    if (i < p) {
+      const int c = i;
+      for (int r2 = 0; r2 < c; ++r2) S.G[c * p + r2] = 0.0;
+      for (int r2 = c; r2 < p; ++r2) {
+        double v = (r2 == c) ? 1.0 : 0.0;
+        for (int m = c; m < r2; ++m) v -= S.L[m * p + r2] * S.G[c * p + m];
+        const double l = S.L[r2 * p + r2];
+        S.G[c * p + r2] = (l != 0.0) ? v / l : 0.0;
+      }
+    }
   }
   __syncthreads();
-  // rows of X: solve y R = x with R = L^T (forward substitution over columns)
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double y[32];
-    for (int k = 0; k < p; ++k) {
-      double v = X[k * (d + 1) + i];
-      for (int m = 0; m < k; ++m) v -= y[m] * S.L[m * p + k];
-      const double lkk = S.L[k * p + k];
-      y[k] = (lkk != 0.0) ? v / lkk : 0.0;
-    }
-    for (int k = 0; k < p; ++k) X[k * (d + 1) + i] = y[k];
+  // Q = X R^-1 = X Linv^T: Q[:, k] = sum_{m <= k} X[:, m] Linv[k][m]
+  double* Y = S.Y;
+  for (int e = threadIdx.x; e < p * d; e += blockDim.x) {
+    const int k = e / d, i = e % d;
+    double acc = 0.0;
+    for (int m = 0; m <= k; ++m) acc = fma(X[m * (d + 1) + i], S.G[m * p + k], acc);
+    Y[k * (d + 1) + i] = acc;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p * d; e += blockDim.x) {
+    const int k = e / d, i = e % d;
+    X[k * (d + 1) + i] = Y[k * (d + 1) + i];
   }
   __syncthreads();
 }
@@ -287,28 +294,19 @@ __global__ void __launch_bounds__(512) refresh_kernel(const double* __restrict__
     }
   }
   __syncthreads();
-  // ---- orthogonal iteration
-  double prev = -1.0;
-  const int maxit = warm ? 24 : 200;
-  for (int it = 0; it < maxit; ++it) {
-    cholqr(S, S.X, d, p);
+  // ---- orthogonal iteration: a fixed number of steps (the top-r subspace
+  // converges at rate lambda_{p+1}/lambda_r per step; the trailing part of the
+  // block may be nearly degenerate, so the block as a whole is not a stopping
+  // test).  Warm starts track a basis that moves little between refreshes.
+  const int iters = warm ? 3 : 30;
+  for (int it = 0; it < iters; ++it) {
     cholqr(S, S.X, d, p);
     gemm_AX(S, S.X, S.Y, d, p);
-    double part = 0.0;
-    for (int e = tid; e < p * d; e += nt) {
-      const int k = e / d, i = e % d;
-      part += S.X[k * (d + 1) + i] * S.Y[k * (d + 1) + i];
-    }
-    const double tr = block_sum(part, S.red);
-    const bool done = (prev >= 0.0) && fabs(tr - prev) <= 1e-14 * fabs(tr);
-    prev = tr;
-    // X <- A X for the next step
     for (int e = tid; e < p * d; e += nt) {
       const int k = e / d, i = e % d;
       S.X[k * (d + 1) + i] = S.Y[k * (d + 1) + i];
     }
     __syncthreads();
-    if (done) break;
   }
   // ---- Rayleigh-Ritz on the final block
   cholqr(S, S.X, d, p);
