@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "QwmError", "qwm_config", "qwm_sizes", "qwm_buffers", "qwm_cache", "BUFFER_NAMES",
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
-    "qwm_build_centroids", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
+    "qwm_build_centroids", "qwm_build_centroids_noalloc", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
     "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
 ]
 
@@ -93,6 +93,7 @@ def lib():
             "qwm_reconstruct": (I32, [pc, I64, I64, _P, _P, _P]),
             "qwm_top1_shift": (I32, [pc, _P, I64, _P, _P, _P, _P]),
             "qwm_device_status": (I32, [ctypes.POINTER(ctypes.c_int32)]),
+            "qwm_build_centroids_noalloc": (I32, [pc, _P, _P, I64, I32, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -149,6 +150,15 @@ def qwm_cache_init(cache: qwm_cache, cfg: qwm_config, bufs: qwm_buffers, stream=
 def qwm_build_centroids(cache: qwm_cache, K: torch.Tensor, V: torch.Tensor, iters: int = 10,
                         stream=None) -> None:
     _check("qwm_build_centroids", lib().qwm_build_centroids(
+        ctypes.byref(cache), _dev_ptr(K, "K", torch.bfloat16), _dev_ptr(V, "V", torch.bfloat16),
+        K.shape[0], iters, _stream(stream, K.device)))
+
+
+def qwm_build_centroids_noalloc(cache: qwm_cache, K: torch.Tensor, V: torch.Tensor,
+                                iters: int = 10, stream=None) -> None:
+    """Same result as qwm_build_centroids, with the scratch taken from a fixed
+    device array inside the library (for callers that cannot allocate)."""
+    _check("qwm_build_centroids_noalloc", lib().qwm_build_centroids_noalloc(
         ctypes.byref(cache), _dev_ptr(K, "K", torch.bfloat16), _dev_ptr(V, "V", torch.bfloat16),
         K.shape[0], iters, _stream(stream, K.device)))
 

@@ -191,6 +191,31 @@ QWM_API qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, vo
 QWM_API qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q, const void* K_exact,
                           int32_t* idx_exact, int32_t* idx_quant, void* stream);
 
+/* Size of the fixed device scratch array used by
+ * qwm_build_centroids_noalloc (16 MiB per GPU that loads the library). */
+#define QWM_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* qwm_build_centroids for callers that cannot allocate device memory -- no
+ * counterpart in the paper.  Hosts such as inference servers or engine plugin
+ * frameworks own the GPU memory budget and hand out fixed buffers; code running
+ * inside them may not call cudaMalloc/cudaFree (these synchronize the device
+ * and fragment the host's pool).  This variant writes the same centroid tables
+ * as qwm_build_centroids but takes its scratch from one fixed device array
+ * inside the library instead of the cache's WORKSPACE buffer, and allocates
+ * nothing.  The array is QWM_NOALLOC_SCRATCH_BYTES long and stays allocated on
+ * every GPU that loads the library until the process exits; the call needs
+ * 4*H*C*d bytes (rounded up to 256) + 4*H*n bytes of it and returns
+ * QWM_ERR_CAPACITY when that exceeds the array.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device
+ * current), so make that first call before any stream capture.  No scratch
+ * entry needs to start at zero (each is written before it is read).  All calls
+ * share the one array and it keeps the last call's contents: calls whose
+ * kernels can overlap on the GPU (several streams of one device) race, and the
+ * caller must order them.  Arguments and other errors as for
+ * qwm_build_centroids: INVALID_ARG, ALIGNMENT, CAPACITY, CUDA. */
+QWM_API qwm_status qwm_build_centroids_noalloc(qwm_cache* c, const void* K, const void* V,
+                                               int64_t n, int32_t iters, void* stream);
+
 /* Device-side health check: synchronizes the current device, then reads and
  * clears the flag that the tensor-core kernels set when one of their bounded
  * waits gave up (about one second per wait) instead of hanging.  *flags = 1 and
