@@ -21,7 +21,7 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
           "-fvisibility=hidden", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 # Files whose floating-point decisions must follow the canonical operation
 # order exactly: no contraction of a*b+c beyond the explicit __fmaf_rn calls.
-NO_FMAD = {"append.cu", "kmeans.cu", "stats.cu"}
+NO_FMAD = {"append.cu", "append_tc.cu", "kmeans.cu", "stats.cu"}
 
 
 def sources():

@@ -218,7 +218,9 @@ qwm_status qwm_device_status(int32_t* flags) {
   if (!flags) return QWM_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return QWM_ERR_CUDA;
   int v = read_and_clear_tc_timeout();
-  if (v < 0) return QWM_ERR_CUDA;
+  int v2 = read_and_clear_append_timeout();
+  if (v < 0 || v2 < 0) return QWM_ERR_CUDA;
+  v = v | v2;
   *flags = v;
   return v ? QWM_ERR_TIMEOUT : QWM_OK;
 }

@@ -265,8 +265,19 @@ cudaError_t run(const AppendArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_t* K,
+                               const uint16_t* V, int64_t n, int64_t t0, int version,
+                               cudaStream_t s);
+
 cudaError_t launch_append(const Dims& Dm, const CacheView& v, const uint16_t* K, const uint16_t* V,
                           int64_t n, int64_t t0, int version, cudaStream_t s) {
+  if (append_tc_supported(Dm)) return launch_append_tc(Dm, v, K, V, n, t0, version, s);
+  return launch_append_simt(Dm, v, K, V, n, t0, version, s);
+}
+
+cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_t* K,
+                               const uint16_t* V, int64_t n, int64_t t0, int version,
+                               cudaStream_t s) {
   AppendArgs a{};
   a.n = n;
   a.t0 = t0;

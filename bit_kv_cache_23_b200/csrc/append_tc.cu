@@ -1,0 +1,528 @@
+// append_tc.cu -- the append with a tensor-core prefilter for the centroid
+// search (head_dim 128, C a multiple of 16, C <= 512).
+//
+// The codes written are exactly those of the canonical fp32 definition in
+// append.cu (QSAC shortlist by (D_i, i), QSAC score, INT2 groups, PSAC INT8);
+// only the search for candidates changes:
+//
+//   D_i = A_t + d_i,  d_i = B_i - 2 X_ti,  A_t = sum_j s_j k_j^2,
+//   B_i = sum_j s_j c_ij^2,  X_ti = sum_j (s_j k_tj) c_ij      (s = 1 for Values)
+//
+// The tensor cores compute the approximation d~_i for all C centroids at once
+// (s*k split into bf16 hi + lo, centroid rows as -2c in bf16, plus one K step
+// adding B_i as bf16 hi + lo) into TMEM.  With a bound E >= |d~_i - d_i|
+// (representation 2^-17 and fp32-accumulation error, Cauchy-Schwarz:
+// sum |s k c| <= sqrt(A_t B_i)) and the canonical fold's relative error
+// gamma, every index of the exact top-M must satisfy d~_i <= theta (derived
+// below); those survivors, usually about M, are rescored with the canonical fp32
+// fold and ranked by (D, i).  A token with more than SURV_MAX survivors is
+// rescored over all C centroids.
+//
+// One CTA per (head, 128 tokens), 128 threads: thread t owns token t and TMEM
+// lane t.  Thread 0 issues the MMAs.  Phases are separated by __syncthreads;
+// the single mbarrier wait is bounded.
+//
+// This file is compiled with --fmad=false; all fused multiply-adds of the
+// canonical definition are explicit __fmaf_rn calls.
+#include <math.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace qwm {
+
+__device__ int g_append_timeout;
+
+namespace {
+using namespace tc;
+
+constexpr int TT = 128;        // tokens per CTA
+constexpr int DH = 128;        // head_dim
+constexpr int NCH = 256;       // centroids per MMA chunk (N)
+constexpr int SURV_MAX = 24;   // survivors kept per token before falling back
+constexpr int KROW = 130;      // padded bf16 row of the token tile (conflict-free)
+
+constexpr uint32_t TILE_A = 128 * 128 * 2;           // A hi / lo (SW128 K-major)
+constexpr uint32_t TILE_B = NCH * 128 * 2;           // -2c chunk (SW128 K-major)
+constexpr uint32_t OFF_AHI = 0;
+constexpr uint32_t OFF_ALO = OFF_AHI + TILE_A;
+constexpr uint32_t OFF_B = OFF_ALO + TILE_A;
+constexpr uint32_t OFF_AEXT = OFF_B + TILE_B;                 // [128][16] bf16 no swizzle
+constexpr uint32_t OFF_BEXT = OFF_AEXT + 128 * 16 * 2;        // [256][16]
+constexpr uint32_t OFF_KROW = OFF_BEXT + NCH * 16 * 2;        // [128][130] bf16
+constexpr uint32_t OFF_BSUM = OFF_KROW + TT * KROW * 2;       // [512] fp32
+constexpr uint32_t OFF_SURV = OFF_BSUM + 512 * 4;             // [128][SURV_MAX] u16
+constexpr uint32_t OFF_S = OFF_SURV + TT * SURV_MAX * 2;      // [128] s
+constexpr uint32_t OFF_W = OFF_S + 128 * 4;                   // [8] w
+constexpr uint32_t OFF_U = OFF_W + 8 * 4;                     // [128][16] U
+constexpr uint32_t OFF_RED = OFF_U + 128 * 16 * 4;            // [8]
+constexpr uint32_t OFF_BAR = OFF_RED + 8 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 16 + 16 + 1024;
+// PSAC residual scratch [128 channels][128 tokens] fp32 reuses A hi/lo (64 KB)
+constexpr uint32_t OFF_E = OFF_AHI;
+
+struct ApArgs {
+  const uint16_t* X;      // [n][H][d] bf16
+  const uint16_t* cent;   // [H][C][d] bf16
+  const float* sens;      // [H][d]
+  const float* wgroup;    // [H][ng]
+  const float* basis;     // [H][d][r] (slot in force)
+  uint8_t* codes;
+  uint16_t* params;
+  void* idx;
+  int8_t* coef;
+  uint16_t* cscale;
+  uint16_t* tokver;
+  int64_t n, t0, tcap;
+  int H, C, G, M, r, idx_bytes, version;
+};
+
+__device__ __forceinline__ bool lex_less(float a, int ia, float b, int ib) {
+  return a < b || (a == b && ia < ib);
+}
+
+__device__ __forceinline__ uint16_t bf16_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// canonical distance of token row k (padded smem row) to centroid row c (global)
+template <bool KEY>
+__device__ __forceinline__ float canon_dist(const uint16_t* krow, const uint16_t* crow,
+                                            const float* s) {
+  float acc = 0.0f;
+  const uint4* c4 = reinterpret_cast<const uint4*>(crow);
+#pragma unroll 2
+  for (int q = 0; q < DH / 8; ++q) {
+    const uint4 cw = __ldg(c4 + q);
+    const uint32_t cv[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = q * 8 + e;
+      const float cj = __uint_as_float(e & 1 ? (cv[e / 2] & 0xffff0000u) : (cv[e / 2] << 16));
+      const float dl = __fsub_rn(bf2f(krow[j]), cj);
+      if (KEY) acc = __fmaf_rn(s[j], __fmul_rn(dl, dl), acc);
+      else acc = __fmaf_rn(dl, dl, acc);
+    }
+  }
+  return acc;
+}
+
+template <bool KEY>
+__global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8);
+  uint16_t* krow = reinterpret_cast<uint16_t*>(smem + OFF_KROW);
+  float* bsum = reinterpret_cast<float*>(smem + OFF_BSUM);
+  uint16_t* surv = reinterpret_cast<uint16_t*>(smem + OFF_SURV);
+  float* s_s = reinterpret_cast<float*>(smem + OFF_S);
+  float* w_s = reinterpret_cast<float*>(smem + OFF_W);
+  float* U_s = reinterpret_cast<float*>(smem + OFF_U);
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const int C = A.C, G = A.G, r = A.r, ng = DH / A.G;
+  const int64_t tok = (int64_t)blockIdx.x * TT + tid;
+  const bool valid = tok < A.n;
+  const uint16_t* cent = A.cent + (size_t)h * C * DH;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  // ---- P0: statistics in force; B_i for every centroid; Bmax
+  for (int j = tid; j < DH; j += TT) s_s[j] = KEY ? A.sens[(size_t)h * DH + j] : 1.0f;
+  if (KEY) {
+    if (tid < ng) w_s[tid] = A.wgroup[(size_t)h * ng + tid];
+    for (int e = tid; e < DH * r; e += TT) U_s[e] = A.basis[(size_t)h * DH * r + e];
+  }
+  __syncthreads();
+  float bmax = 0.0f;
+  for (int i = tid; i < C; i += TT) {
+    const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
+    float acc = 0.0f;
+    for (int q = 0; q < DH / 8; ++q) {
+      const uint4 cw = __ldg(c4 + q);
+      const uint32_t cv[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float cj = __uint_as_float(e & 1 ? (cv[e / 2] & 0xffff0000u) : (cv[e / 2] << 16));
+        acc = __fmaf_rn(s_s[q * 8 + e], __fmul_rn(cj, cj), acc);
+      }
+    }
+    bsum[i] = acc;
+    bmax = fmaxf(bmax, acc);
+  }
+  for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+  if (lane == 0) red[warp] = bmax;
+  // ---- P1: token row -> padded smem row, A hi/lo (s*k split), A_t
+  float At = 0.0f;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(A.X + ((size_t)tok * A.H + h) * DH);
+    uint8_t* ahi = smem + OFF_AHI;
+    uint8_t* alo = smem + OFF_ALO;
+#pragma unroll 2
+    for (int c = 0; c < 16; ++c) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (valid) w = __ldg(src + c);
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        reinterpret_cast<uint32_t*>(krow + tid * KROW)[c * 4 + e2] = wv[e2];
+        float sk[2], hv[2];
+        uint16_t hb[2], lb[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int j = c * 8 + e2 * 2 + u;
+          const float kj = __uint_as_float(u ? (wv[e2] & 0xffff0000u) : (wv[e2] << 16));
+          At = __fmaf_rn(s_s[j], __fmul_rn(kj, kj), At);
+          sk[u] = KEY ? __fmul_rn(s_s[j], kj) : kj;
+          hb[u] = bf16_rn(sk[u]);
+          hv[u] = bf2f(hb[u]);
+          lb[u] = bf16_rn(__fsub_rn(sk[u], hv[u]));
+        }
+        hi[e2] = (uint32_t)hb[0] | ((uint32_t)hb[1] << 16);
+        lo[e2] = (uint32_t)lb[0] | ((uint32_t)lb[1] << 16);
+      }
+      *reinterpret_cast<uint4*>(ahi + sw128_off(tid, c, 128)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (KEY)
+        *reinterpret_cast<uint4*>(alo + sw128_off(tid, c, 128)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    // extra K step: A row = [1, 1, 0 ...]
+    uint8_t* aext = smem + OFF_AEXT;
+    const uint32_t one2 = 0x3F803F80u;  // bf16 1.0, 1.0
+    *reinterpret_cast<uint4*>(aext + (tid >> 3) * 256 + (tid & 7) * 16) = make_uint4(one2, 0, 0, 0);
+    *reinterpret_cast<uint4*>(aext + (tid >> 3) * 256 + 128 + (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  bmax = 0.0f;
+  for (int wv = 0; wv < TT / 32; ++wv) bmax = fmaxf(bmax, red[wv]);
+
+  // ---- P2/P3: per chunk of 256 centroids: B operand, MMAs into TMEM columns
+  const int nchunk = (C + NCH - 1) / NCH;
+  bool ok = true;
+  for (int ch = 0; ch < nchunk; ++ch) {
+    const int c0 = ch * NCH, nc = min(NCH, C - c0);
+    uint8_t* bt = smem + OFF_B;
+    uint8_t* bext = smem + OFF_BEXT;
+    for (int rr = tid; rr < NCH; rr += TT) {
+      const int i = c0 + rr;
+      const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (rr < nc) w = __ldg(c4 + c);
+        // -2c is exact in bf16: flip the sign, add one to the exponent (0 stays 0)
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          uint32_t x = wv[e2], y = 0;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t hbits = (x >> (16 * u)) & 0xffffu;
+            const float f = __uint_as_float(hbits << 16);
+            const uint16_t m2 = bf16_rn(-2.0f * f);
+            y |= (uint32_t)m2 << (16 * u);
+          }
+          o[e2] = y;
+        }
+        *reinterpret_cast<uint4*>(bt + sw128_off(rr, c, NCH)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      const float b = (rr < nc) ? bsum[i] : 0.0f;
+      const uint16_t bh = bf16_rn(b);
+      const uint16_t bl = bf16_rn(__fsub_rn(b, bf2f(bh)));
+      *reinterpret_cast<uint4*>(bext + (rr >> 3) * 256 + (rr & 7) * 16) =
+          make_uint4((uint32_t)bh | ((uint32_t)bl << 16), 0, 0, 0);
+      *reinterpret_cast<uint4*>(bext + (rr >> 3) * 256 + 128 + (rr & 7) * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16(128, NCH, false, false);
+      const uint32_t sa = smem_u32(smem + OFF_AHI), sl = smem_u32(smem + OFF_ALO);
+      const uint32_t sb = smem_u32(smem + OFF_B);
+      const uint32_t d_t = tmem + ch * NCH;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t ko = (k >> 2) * (128 * 128) + (k & 3) * 32;
+        const uint32_t kb = (k >> 2) * (NCH * 128) + (k & 3) * 32;
+        mma_bf16_ss(d_t, desc_sw128(sa + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, k > 0);
+      }
+      if (KEY) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t ko = (k >> 2) * (128 * 128) + (k & 3) * 32;
+          const uint32_t kb = (k >> 2) * (NCH * 128) + (k & 3) * 32;
+          mma_bf16_ss(d_t, desc_sw128(sl + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, 1u);
+        }
+      }
+      mma_bf16_ss(d_t, desc_noswz(smem_u32(smem + OFF_AEXT), 128, 256),
+                  desc_noswz(smem_u32(smem + OFF_BEXT), 128, 256), idesc, 1u);
+      mma_commit(bar);
+    }
+    ok = ok && mbar_wait(bar, ch & 1);
+    tc_fence_after();
+    __syncthreads();
+  }
+  if (!__syncthreads_and(ok)) {
+    if (tid == 0) atomicExch(&g_append_timeout, 1);
+  }
+
+  // ---- P4: selection from the approximations (thread t, TMEM lane t)
+  const int Mc = KEY ? A.M : 1;
+  // |d~ - d| <= (2^-16.9 + 2^-14) sqrt(A_t B_i) + (2^-15 + 2^-17 + 2^-18) B_i: bf16 hi+lo
+  // representation of s*k (2^-17.9 per term, Cauchy-Schwarz), fp32 accumulation of
+  // 258 terms (<= 258 * 2^-23 of the sum of magnitudes), B_i's fp32 fold and its
+  // hi+lo split.  E doubles both coefficients.  The canonical fold of 128
+  // positive terms is within (n + 3) 2^-24 < 2^-16.9 relative; gamma = 2^-15.
+  const float E = 2.4414062e-4f * sqrtf(At * bmax) + 1.2207031e-4f * bmax;  // 2^-12, 2^-13
+  const float gam = 3.0517578e-5f;                                           // 2^-15
+  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+  float topv[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) topv[m] = INFINITY;
+  for (int c0 = 0; c0 < nchunk * NCH; c0 += 32) {
+    float v[32];
+    tmem_ld32(trow + c0, v);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if (c0 + e < C && v[e] < topv[7]) {
+        float x = v[e];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {  // insertion into the sorted list
+          const float lo = fminf(topv[m], x);
+          x = fmaxf(topv[m], x);
+          topv[m] = lo;
+        }
+      }
+    }
+  }
+  float dM = topv[0];
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+    if (m == Mc - 1) dM = topv[m];
+  const float tau = dM + E + gam * (At + fabsf(dM) + E);
+  float theta = (tau + E + gam * (At + E)) / (1.0f - gam);
+  theta += 1e-6f * (fabsf(theta) + At) + 1e-30f;
+  int cnt = 0;
+  for (int c0 = 0; c0 < nchunk * NCH; c0 += 32) {
+    float v[32];
+    tmem_ld32(trow + c0, v);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if (c0 + e < C && v[e] <= theta) {
+        if (cnt < SURV_MAX) surv[tid * SURV_MAX + cnt] = (uint16_t)(c0 + e);
+        ++cnt;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+
+  // ---- P5: exact (canonical) distances of the survivors; top-M by (D, i)
+  const uint16_t* kr = krow + tid * KROW;
+  int cand[8];
+  float candD[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) { cand[m] = -1; candD[m] = INFINITY; }
+  if (valid) {
+    const bool all = cnt > SURV_MAX || cnt < Mc;  // overflow, or no usable approximation
+    const int nloop = all ? C : cnt;
+    for (int q = 0; q < nloop; ++q) {
+      const int i = all ? q : (int)surv[tid * SURV_MAX + q];
+      const float D = canon_dist<KEY>(kr, cent + (size_t)i * DH, s_s);
+      // insert (D, i) into the sorted candidate list (total order on (D, i))
+      float xd = D;
+      int xi = i;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        if (m < Mc) {
+          const bool sw = (candD[m] == INFINITY && cand[m] < 0) || lex_less(xd, xi, candD[m], cand[m]);
+          if (sw) {
+            const float td = candD[m];
+            const int ti = cand[m];
+            candD[m] = xd;
+            cand[m] = xi;
+            xd = td;
+            xi = ti;
+          }
+        }
+      }
+    }
+  }
+  if (!valid) return;
+
+  // ---- P6: QSAC stage 2 (keys): expected squared logit perturbation
+  int a = cand[0];
+  if (KEY && Mc > 1) {
+    float best = 0.0f;
+    int bm = -1;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      if (m < Mc) {
+        const uint16_t* crow = cent + (size_t)cand[m] * DH;
+        float score = 0.0f;
+        for (int g = 0; g < ng; ++g) {
+          float lo = 0.0f, hi = 0.0f;
+          for (int jj = 0; jj < G; ++jj) {
+            const int j = g * G + jj;
+            const float rho = __fsub_rn(bf2f(kr[j]), bf2f(__ldg(crow + j)));
+            lo = (jj == 0) ? rho : fminf(lo, rho);
+            hi = (jj == 0) ? rho : fmaxf(hi, rho);
+          }
+          const float R = __fsub_rn(hi, lo);
+          score = __fmaf_rn(w_s[g], __fmul_rn(R, R), score);
+        }
+        if (bm < 0 || score < best) { best = score; bm = m; }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (m == bm) a = cand[m];
+  }
+
+  // ---- P7: INT2 residual, PSAC coefficients, stores
+  const size_t slot = (size_t)h * A.tcap + (size_t)(A.t0 + tok);
+  const uint16_t* crow = cent + (size_t)a * DH;
+  float* e_s = reinterpret_cast<float*>(smem + OFF_E);  // [channel][token]
+  for (int g = 0; g < ng; ++g) {
+    float lo = 0.0f, hi = 0.0f;
+    for (int jj = 0; jj < G; ++jj) {
+      const int j = g * G + jj;
+      const float rho = __fsub_rn(bf2f(kr[j]), bf2f(__ldg(crow + j)));
+      lo = (jj == 0) ? rho : fminf(lo, rho);
+      hi = (jj == 0) ? rho : fmaxf(hi, rho);
+    }
+    uint16_t mnh, sch;
+    float mn, sc;
+    int2_params(lo, hi, mnh, sch, mn, sc);
+    reinterpret_cast<uint32_t*>(A.params)[slot * ng + g] = (uint32_t)mnh | ((uint32_t)sch << 16);
+    for (int jb = 0; jb < G; jb += 4) {
+      uint32_t byte = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = g * G + jb + u;
+        const float cj = bf2f(__ldg(crow + j));
+        const float kj = bf2f(kr[j]);
+        const float rho = __fsub_rn(kj, cj);
+        const int code = int2_code(rho, mn, sc);
+        byte |= (uint32_t)code << (2 * u);
+        if (KEY) {
+          const float deq = __fmaf_rn((float)code, sc, mn);
+          e_s[j * TT + tid] = __fsub_rn(kj, __fadd_rn(cj, deq));
+        }
+      }
+      A.codes[slot * (DH / 4) + (g * G + jb) / 4] = (uint8_t)byte;
+    }
+  }
+  if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
+  else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
+  if (KEY) {
+    if (h == 0) A.tokver[A.t0 + tok] = (uint16_t)A.version;
+    float cq[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      cq[q] = 0.0f;
+      if (q < r) {
+        float acc = 0.0f;
+        for (int j = 0; j < DH; ++j) acc = __fmaf_rn(U_s[j * r + q], e_s[j * TT + tid], acc);
+        cq[q] = acc;
+        amax = fmaxf(amax, fabsf(acc));
+      }
+    }
+    const uint16_t csh = f2h_ru(__fdiv_rn(amax, 127.0f));
+    const float cs = h2f(csh);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if (q < r) {
+        int q8 = 0;
+        if (cs != 0.0f) {
+          q8 = __float2int_rn(__fdiv_rn(cq[q], cs));
+          q8 = max(-127, min(127, q8));
+        }
+        A.coef[slot * r + q] = (int8_t)q8;
+      }
+    }
+    A.cscale[slot] = csh;
+  }
+}
+
+template <bool KEY>
+cudaError_t run_tc(const ApArgs& a, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((a.n + TT - 1) / TT), a.H);
+  append_tc_kernel<KEY><<<grid, TT, SMEM_BYTES, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int read_and_clear_append_timeout() {
+  int v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_append_timeout, sizeof(int)) != cudaSuccess) return -1;
+  cudaMemcpyToSymbol(g_append_timeout, &z, sizeof(int));
+  return v;
+}
+
+bool append_tc_supported(const Dims& D) {
+  return D.d == DH && D.C % 16 == 0 && D.C <= 512 && D.M <= 8 && D.r <= 16;
+}
+
+cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t* K,
+                             const uint16_t* V, int64_t n, int64_t t0, int version,
+                             cudaStream_t s) {
+  ApArgs a{};
+  a.n = n;
+  a.t0 = t0;
+  a.tcap = Dm.tcap;
+  a.H = Dm.H;
+  a.C = Dm.C;
+  a.G = Dm.G;
+  a.M = Dm.M;
+  a.r = Dm.r;
+  a.idx_bytes = Dm.idx_bytes;
+  a.version = version;
+  a.X = K;
+  a.cent = v.cent_k;
+  a.sens = v.sens;
+  a.wgroup = v.wgroup;
+  a.basis = v.basis + (size_t)version * Dm.H * Dm.d * (Dm.r > 0 ? Dm.r : 1);
+  a.codes = v.k_codes;
+  a.params = v.k_params;
+  a.idx = v.k_idx;
+  a.coef = v.k_coef;
+  a.cscale = v.k_cscale;
+  a.tokver = v.tokver;
+  cudaError_t e = run_tc<true>(a, s);
+  if (e != cudaSuccess) return e;
+  a.X = V;
+  a.cent = v.cent_v;
+  a.codes = v.v_codes;
+  a.params = v.v_params;
+  a.idx = v.v_idx;
+  a.coef = nullptr;
+  a.cscale = nullptr;
+  return run_tc<false>(a, s);
+}
+
+}  // namespace qwm

@@ -53,22 +53,20 @@ constexpr uint32_t XSLAB = 128 * 32 * 2;   // [128][<=32] bf16 compensation slab
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE;         // 2 slots
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE;     // 2 slots
-constexpr uint32_t OFF_P = OFF_V + 2 * TILE;     // 1 buffer
-constexpr uint32_t OFF_AX = OFF_P + TILE;        // 2 buffers (by tile parity)
+constexpr uint32_t OFF_AX = OFF_V + 2 * TILE;    // 2 buffers (by tile parity)
 constexpr uint32_t OFF_BX = OFF_AX + 2 * XSLAB;  // 2 slots (with K-hat/V')
 constexpr uint32_t OFF_BAR = OFF_BX + 2 * XSLAB;
 constexpr int NBAR = 16;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 
 enum {
-  B_KV_FULL = 0,  // [2] dequant (256) -> MMA
+  B_KV_FULL = 0,  // [2] dequant (one arrival per warp) -> MMA
   B_KV_EMPTY = 2, // [2] MMA commit -> dequant
   B_S_FULL = 4,   // [2] MMA commit -> softmax
-  B_S_FREE = 6,   // [2] softmax (128) -> MMA
-  B_AX_FULL = 8,  // [2] softmax (128) -> MMA: slab for the tile of that parity
-  B_P_FULL = 10,  // softmax (128) -> MMA
+  B_P_FULL = 6,   // [2] softmax (per warp) -> MMA: P of that parity is in TMEM
+  B_AX_FULL = 8,  // [2] softmax (per warp) -> MMA: slab for the tile of that parity
   B_O_FULL = 11,  // MMA commit after each P V'
-  B_Q_READY = 12, // softmax (128) -> MMA
+  B_Q_READY = 12, // softmax (per warp) -> MMA
   B_DONE = 13,    // MMA commit -> MMA (drain before exit)
   B_O_LAST = 14   // MMA commit after the last P V'
 };
@@ -90,12 +88,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// {a, b} -> bf16x2 with a in the low half (round to nearest even)
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
 }
 
 __device__ __forceinline__ void timeout_flag() { atomicExch(&g_tc_timeout, 1); }
+
+// One arrival per warp: every lane has ordered its own writes (proxy fence or
+// tcgen05 fence) before calling; __syncwarp orders the lanes, then lane 0
+// arrives with release semantics.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 
 // byte offset of 16-byte chunk c (8 bf16) of row r in a no-swizzle K-major slab
 // with kx columns: core matrices of 8 rows x 16 B, K-adjacent cores 128 B apart,
@@ -203,10 +211,10 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     }
   }
   fence_proxy_async_smem();
-  mbar_arrive(&bars[B_Q_READY]);
+  warp_arrive(&bars[B_Q_READY]);
   if (A.kx) {
-    mbar_arrive(&bars[B_AX_FULL + 0]);
-    if (ntile > 1) mbar_arrive(&bars[B_AX_FULL + 1]);
+    warp_arrive(&bars[B_AX_FULL + 0]);
+    if (ntile > 1) warp_arrive(&bars[B_AX_FULL + 1]);
   }
 
   float m_used = -INFINITY, l = 0.0f;
@@ -234,15 +242,15 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     if (j == 0) {
       m_used = m_row;
     } else {
-      // P V' of tile j-1 must be done before P is overwritten and before O is
-      // touched.  S_FULL(j) implies P V' of tile j-2 is done (commits track all
-      // earlier MMAs) and P V' of tile j cannot start before P_FULL(j), so
-      // O_FULL sits in phase j-1 or j and the parity test is exact.
-      bool w2 = mbar_wait(&bars[B_O_FULL], (j - 1) & 1);
-      if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-      tc_fence_after();
       const bool need = m_row > m_used + TAU;
       if (__any_sync(0xffffffffu, need)) {
+        // O holds P V' of tiles < j: wait for the last of them, then rescale.
+        // S_FULL(j) implies P V' of tile j-2 is done (commits track all earlier
+        // MMAs) and P V' of tile j cannot start before P_FULL(j), so O_FULL sits
+        // in phase j-1 or j and the parity test is exact.
+        bool w2 = mbar_wait(&bars[B_O_FULL], (j - 1) & 1);
+        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+        tc_fence_after();
         const float f = need ? ex2(m_used - m_row) : 1.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -256,32 +264,28 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
         if (need) m_used = m_row;
       }
     }
+    // P (bf16 pairs) overwrites the S columns already read: keys 2i, 2i+1 of
+    // the tile go to column i of the same TMEM buffer (the A-operand layout of
+    // the P V' MMA).
     float lsum = 0.0f;
-    uint8_t* pb = smem + OFF_P;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float s[32];
+      tmem_ld32(trow + b * 128 + c * 32, s);
+      uint32_t pk[16];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      float s[64];
-      tmem_ld64(trow + b * 128 + c * 64, s);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int col = c * 64 + k * 8 + e;
-          const float p0 = (col < nvalid) ? ex2(fmaf(s[k * 8 + e], sl2, -m_used)) : 0.0f;
-          const float p1 = (col + 1 < nvalid) ? ex2(fmaf(s[k * 8 + e + 1], sl2, -m_used)) : 0.0f;
-          lsum += p0 + p1;
-          pk[e / 2] = pack_bf16(p0, p1);
-        }
-        *reinterpret_cast<uint4*>(pb + sw128_off(row, c * 8 + k, BQ)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < 32; e += 2) {
+        const int col = c * 32 + e;
+        const float p0 = (col < nvalid) ? ex2(fmaf(s[e], sl2, -m_used)) : 0.0f;
+        const float p1 = (col + 1 < nvalid) ? ex2(fmaf(s[e + 1], sl2, -m_used)) : 0.0f;
+        lsum += p0 + p1;
+        pk[e / 2] = pack_bf16(p0, p1);
       }
+      tmem_st16u(trow + b * 128 + c * 16, pk);
     }
     l += lsum;
     tc_fence_before();
-    mbar_arrive(&bars[B_S_FREE + b]);
-    fence_proxy_async_smem();
-    mbar_arrive(&bars[B_P_FULL]);
+    warp_arrive(&bars[B_P_FULL + b]);
     // slab for tile j+2 into buffer b (QK^T of tile j, its last reader, is done)
     if (A.kx && j + 2 < ntile) {
       int va, vb;
@@ -293,7 +297,7 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
         else ax_pair0 = pair;
         fence_proxy_async_smem();
       }
-      mbar_arrive(&bars[B_AX_FULL + b]);
+      warp_arrive(&bars[B_AX_FULL + b]);
     }
   }
   if (ok) {
@@ -339,9 +343,12 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
   const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
   for (int j = 0; j < ntile; ++j) {
     const int slot = j & 1;
-    if (j >= 2 && !mbar_wait_sleep(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1)) {
-      timeout_flag();
-      return;
+    if (j >= 2) {
+      const bool w = mbar_wait_sleep(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1);
+      if (!__all_sync(0xffffffffu, w)) {
+        timeout_flag();
+        return;
+      }
     }
     uint8_t* kb = smem + OFF_K + slot * TILE;
     uint8_t* vb = smem + OFF_V + slot * TILE;
@@ -456,7 +463,7 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
       }
     }
     fence_proxy_async_smem();
-    mbar_arrive(&bars[B_KV_FULL + slot]);
+    warp_arrive(&bars[B_KV_FULL + slot]);
   }
 }
 
@@ -469,7 +476,8 @@ __device__ __forceinline__ bool issue_qk(uint64_t* bars, uint32_t sbase, uint32_
   const int slot = j & 1;
   if (!mbar_wait(&bars[B_KV_FULL + slot], (j >> 1) & 1)) return false;
   if (kx && !mbar_wait(&bars[B_AX_FULL + slot], (j >> 1) & 1)) return false;
-  if (j >= 2 && !mbar_wait(&bars[B_S_FREE + slot], ((j - 2) >> 1) & 1)) return false;
+  // S[slot] of tile j-2 held P of that tile; its P V' was issued before this
+  // QK^T by the same thread, and the tensor pipe executes them in order.
   tc_fence_after();
   const uint32_t sq = sbase + OFF_Q, sk = sbase + OFF_K + slot * TILE;
 #pragma unroll
@@ -490,19 +498,19 @@ __device__ __forceinline__ void mma_role(uint8_t* smem, uint64_t* bars, uint32_t
                                          int kx) {
   constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sv = sbase + OFF_V, sp = sbase + OFF_P;
+  const uint32_t sv = sbase + OFF_V;
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
   if (ok) ok = issue_qk(bars, sbase, tmem, 0, kx);
   for (int j = 0; ok && j < ntile; ++j) {
     if (j + 1 < ntile && !(ok = issue_qk(bars, sbase, tmem, j + 1, kx))) break;
     const int b = j & 1;
-    if (!mbar_wait(&bars[B_P_FULL], j & 1)) { ok = false; break; }
+    if (!mbar_wait(&bars[B_P_FULL + b], (j >> 1) & 1)) { ok = false; break; }
     tc_fence_after();
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint64_t da = desc_sw128(sp + (k >> 2) * (BQ * 128) + (k & 3) * 32, 16, 1024);
+      // P of keys 16k..16k+15: TMEM columns b*128 + 8k .. +7 (bf16 pairs)
       const uint64_t db = desc_sw128(sv + b * TILE + k * 2048, KT * 128, 1024);
-      mma_bf16_ss(tmem + 256, da, db, IDP, (j > 0 || k > 0) ? 1u : 0u);
+      mma_bf16_ts(tmem + 256, tmem + b * 128 + k * 8, db, IDP, (j > 0 || k > 0) ? 1u : 0u);
     }
     mma_commit(&bars[B_O_FULL]);
     mma_commit(&bars[B_KV_EMPTY + b]);
@@ -523,15 +531,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   const int ntile = (int)((A.T + KT - 1) / KT);
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[B_KV_FULL + i], NDQ);
+      mbar_init(&bars[B_KV_FULL + i], NDQ / 32);
       mbar_init(&bars[B_KV_EMPTY + i], 1);
       mbar_init(&bars[B_S_FULL + i], 1);
-      mbar_init(&bars[B_S_FREE + i], 128);
-      mbar_init(&bars[B_AX_FULL + i], 128);
+      mbar_init(&bars[B_P_FULL + i], 4);
+      mbar_init(&bars[B_AX_FULL + i], 4);
     }
-    mbar_init(&bars[B_P_FULL], 128);
     mbar_init(&bars[B_O_FULL], 1);
-    mbar_init(&bars[B_Q_READY], 128);
+    mbar_init(&bars[B_Q_READY], 4);
     mbar_init(&bars[B_DONE], 1);
     mbar_init(&bars[B_O_LAST], 1);
     fence_mbar_init();

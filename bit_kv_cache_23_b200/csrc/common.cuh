@@ -7,7 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/qwm.h"
+#include "qwm.h"
 
 namespace qwm {
 
@@ -117,5 +117,10 @@ cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, co
 cudaError_t launch_attention_simt(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
                                   int64_t nq, float scale, uint16_t* O, cudaStream_t s);
 int read_and_clear_tc_timeout();
+int read_and_clear_append_timeout();
+bool append_tc_supported(const Dims& D);
+cudaError_t launch_append_tc(const Dims& D, const CacheView& v, const uint16_t* K,
+                             const uint16_t* V, int64_t n, int64_t t0, int version,
+                             cudaStream_t s);
 
 }  // namespace qwm
