@@ -344,7 +344,7 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
   for (int j = 0; j < ntile; ++j) {
     const int slot = j & 1;
     if (j >= 2) {
-      const bool w = mbar_wait_sleep(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1);
+      const bool w = mbar_wait(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1);
       if (!__all_sync(0xffffffffu, w)) {
         timeout_flag();
         return;
@@ -470,15 +470,10 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
 // ------------------------------------------------------------------ MMA role
 // S[j&1] = Q K-hat_j^T (8 K16 steps over head_dim, two 64-wide swizzled blocks)
 // + the compensation steps [Q U_va | Q U_vb] [c slots]^T.
-__device__ __forceinline__ bool issue_qk(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
+__device__ __forceinline__ void issue_qk(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
                                          int kx) {
   constexpr uint32_t IDQ = idesc_bf16(128, 128, false, false);
   const int slot = j & 1;
-  if (!mbar_wait(&bars[B_KV_FULL + slot], (j >> 1) & 1)) return false;
-  if (kx && !mbar_wait(&bars[B_AX_FULL + slot], (j >> 1) & 1)) return false;
-  // S[slot] of tile j-2 held P of that tile; its P V' was issued before this
-  // QK^T by the same thread, and the tensor pipe executes them in order.
-  tc_fence_after();
   const uint32_t sq = sbase + OFF_Q, sk = sbase + OFF_K + slot * TILE;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -491,30 +486,60 @@ __device__ __forceinline__ bool issue_qk(uint64_t* bars, uint32_t sbase, uint32_
     mma_bf16_ss(tmem + slot * 128, desc_noswz(sa + k * 256, 128, kx * 16),
                 desc_noswz(sb + k * 256, 128, kx * 16), IDQ, 1u);
   mma_commit(&bars[B_S_FULL + slot]);
-  return true;
 }
 
+// O += P_j V'_j with P read from TMEM (the S buffer of tile j).
+__device__ __forceinline__ void issue_pv(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
+                                         int ntile) {
+  constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);
+  const int b = j & 1;
+  const uint32_t sv = sbase + OFF_V + b * TILE;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    // P of keys 16k..16k+15: TMEM columns b*128 + 8k .. +7 (bf16 pairs)
+    mma_bf16_ts(tmem + 256, tmem + b * 128 + k * 8, desc_sw128(sv + k * 2048, KT * 128, 1024),
+                IDP, (j > 0 || k > 0) ? 1u : 0u);
+  }
+  mma_commit(&bars[B_O_FULL]);
+  mma_commit(&bars[B_KV_EMPTY + b]);
+  if (j == ntile - 1) mma_commit(&bars[B_O_LAST]);
+}
+
+// ------------------------------------------------------------------ MMA role
+// Issues whichever MMA group is ready.  Constraints: QK^T of tile j after P V'
+// of tile j-2 has been issued (S/P buffer j&1 is reused; the tensor pipe runs
+// in issue order); P V' of tile j after its P is in TMEM.
 __device__ __forceinline__ void mma_role(uint8_t* smem, uint64_t* bars, uint32_t tmem, int ntile,
                                          int kx) {
-  constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sv = sbase + OFF_V;
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
-  if (ok) ok = issue_qk(bars, sbase, tmem, 0, kx);
-  for (int j = 0; ok && j < ntile; ++j) {
-    if (j + 1 < ntile && !(ok = issue_qk(bars, sbase, tmem, j + 1, kx))) break;
-    const int b = j & 1;
-    if (!mbar_wait(&bars[B_P_FULL + b], (j >> 1) & 1)) { ok = false; break; }
-    tc_fence_after();
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      // P of keys 16k..16k+15: TMEM columns b*128 + 8k .. +7 (bf16 pairs)
-      const uint64_t db = desc_sw128(sv + b * TILE + k * 2048, KT * 128, 1024);
-      mma_bf16_ts(tmem + 256, tmem + b * 128 + k * 8, db, IDP, (j > 0 || k > 0) ? 1u : 0u);
+  int qn = 0, pn = 0;  // next QK^T tile, next P V' tile
+  long long t_idle = 0;
+  while (ok && pn < ntile) {
+    bool progress = false;
+    if (qn < ntile && qn < pn + 2) {
+      const int slot = qn & 1;
+      if (mbar_test(&bars[B_KV_FULL + slot], (qn >> 1) & 1) &&
+          (!kx || mbar_test(&bars[B_AX_FULL + slot], (qn >> 1) & 1))) {
+        tc_fence_after();
+        issue_qk(bars, sbase, tmem, qn, kx);
+        ++qn;
+        progress = true;
+      }
     }
-    mma_commit(&bars[B_O_FULL]);
-    mma_commit(&bars[B_KV_EMPTY + b]);
-    if (j == ntile - 1) mma_commit(&bars[B_O_LAST]);
+    if (pn < qn && mbar_test(&bars[B_P_FULL + (pn & 1)], (pn >> 1) & 1)) {
+      tc_fence_after();
+      issue_pv(bars, sbase, tmem, pn, ntile);
+      ++pn;
+      progress = true;
+    }
+    if (progress) {
+      t_idle = 0;
+    } else if (t_idle == 0) {
+      t_idle = clock64();
+    } else if (clock64() - t_idle > (1ll << 31)) {
+      ok = false;
+    }
   }
   mma_commit(&bars[B_DONE]);
   if (!mbar_wait(&bars[B_DONE], 0)) ok = false;
