@@ -1,5 +1,5 @@
 // attention_tc.cu -- attention over the packed QuantWM cache on the sm_100a
-// tensor cores (tcgen05.mma, accumulators in TMEM).
+// tensor cores (tcgen05.mma; Q, S/P and O live in TMEM).
 //
 // O = softmax(scale Q K'^T) V' with K' = C_K[a] + deq(R) + U_v (c8 cs) and
 // V' = C_V[b] + deq(R_V) reconstructed on the fly (QuantWM, "Flickering after
@@ -9,28 +9,34 @@
 //
 // The compensation term runs on the tensor cores instead of per element:
 //   q . (U_v c_t) = (U_v^T q) . c_t,
-// so each QK^T gains one extra K16 step (two for r > 8) whose A operand holds
-// [Q U_va | Q U_vb] for the (at most two) basis versions va, vb of the tile and
-// whose B operand holds each key's c8 cs in the slot of its version.  A key whose
-// version is neither (a tile spanning more than two versions) is compensated
-// element-wise by the dequant thread instead.
+// so each Q K^T gains one extra K16 step (two for r > 8) whose A operand holds
+// AX = [Q U_va | Q U_vb] for the (at most two) basis versions va, vb of the key
+// tile and whose B operand holds each key's c8 cs in the slot of its version.
+// AX itself is a tensor-core product (Q from TMEM times [U_va | U_vb] in bf16),
+// recomputed only when the version pair changes from one key tile to the next;
+// a key whose version is neither (a tile spanning three versions) is
+// compensated element-wise by its dequant thread instead.
 //
-// One CTA per (head, 128 query rows); 416 threads in three roles:
-//   warps 0-3  softmax: warp w owns TMEM lanes 32w..32w+31 = query rows; loads
-//              S from TMEM, online softmax in the log2 domain, writes P (bf16)
-//              to shared memory; rescales O in TMEM when a row max moves; builds
-//              the [Q U_va | Q U_vb] slab two tiles ahead.
-//   warps 4-11 dequant: two threads per key row of each 128-key tile (64
-//              channels each) issue all their loads first, then write K-hat and
-//              V' (bf16) straight into the 128B-swizzled layout the UMMA
-//              descriptors read, plus the key's compensation slab row.
-//   warp 12    MMA: one thread issues S = Q K'^T and O += P V' (V' read
-//              MN-major) and commits to mbarriers.
-// K-hat/V' tiles, the slabs and S are double-buffered, so the QK^T of tile j+1
-// runs while the softmax works on tile j.  TMEM: S[2] at columns 0/128, O at
-// 256 (512 columns; one CTA per SM by shared memory).  Every mbarrier wait is
-// bounded (about 1 s); a timeout sets a device flag that qwm_device_status()
-// reports, and every role then leaves its loop.
+// One CTA per (head, 256 query rows = two 128-row Q tiles); 576 threads:
+//   warps 0-7   softmax: warp w serves Q tile w/4, TMEM lanes 32(w%4)..+31 =
+//               query rows; online softmax in the log2 domain with a lazy
+//               rescale of O, P written back into TMEM over S (bf16 pairs).
+//   warps 8-15  dequant: four threads per key row of each 64-key tile gather
+//               their centroid chunks with 16-byte async copies two tiles
+//               ahead, then rewrite them in place as K-hat / V' (bf16, the
+//               128B-swizzled layouts the UMMA descriptors read).
+//   warp 16     MMA: one thread issues, per key tile and Q tile, S = Q K^T
+//               (+ AX BX^T) and O += P V', alternating the two Q tiles so the
+//               tensor pipe works on one while the softmax works on the other.
+//   warp 17     producer: bulk-copies (TMA engine) the tile's packed codes,
+//               group parameters, coefficients, versions and centroid indices
+//               into the stage, and builds [U_va | U_vb] in bf16 on changes.
+// TMEM (512 columns): per Q tile p, Q at 256p (64 columns of bf16 pairs), S/P
+// at 256p+64, O at 256p+128.  Shared memory: a ring of 4 stages of K-hat, V',
+// packed fields and the compensation slab.  Every mbarrier wait is bounded
+// (about 1 s); a timeout sets a device flag that qwm_device_status() reports,
+// every role then leaves its loop, and in-flight copies and MMAs are drained
+// (bounded) before the TMEM is freed.
 #include <math.h>
 
 #include "dequant.cuh"
@@ -43,32 +49,44 @@ __device__ int g_tc_timeout;
 namespace {
 using namespace tc;
 
-constexpr int BQ = 128;        // query rows per CTA
-constexpr int KT = 128;        // keys per tile
 constexpr int DH = 128;        // head_dim handled here
-constexpr int NTHREADS = 416;  // 4 softmax + 8 dequant + 1 MMA warps
-constexpr int NDQ = 256;       // dequant threads: two per key row
-constexpr uint32_t TILE = 128 * 128 * 2;   // one bf16 128x128 tile
-constexpr uint32_t XSLAB = 128 * 32 * 2;   // [128][<=32] bf16 compensation slab
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + TILE;         // 2 slots
-constexpr uint32_t OFF_V = OFF_K + 2 * TILE;     // 2 slots
-constexpr uint32_t OFF_AX = OFF_V + 2 * TILE;    // 2 buffers (by tile parity)
-constexpr uint32_t OFF_BX = OFF_AX + 2 * XSLAB;  // 2 slots (with K-hat/V')
-constexpr uint32_t OFF_BAR = OFF_BX + 2 * XSLAB;
-constexpr int NBAR = 16;
+constexpr int KT = 64;         // keys per tile
+constexpr int QT = 128;        // query rows per Q tile (TMEM lanes)
+constexpr int BQ = 2 * QT;     // query rows per CTA
+constexpr int NST = 4;         // pipeline stages
+constexpr int NTHREADS = 576;  // 8 softmax + 8 dequant + MMA + producer warps
+constexpr int W_MMA = 16;
+constexpr int NDQW = 8;        // dequant warps
+
+// ---- shared memory (bytes); K-hat and V' tiles 1024-aligned for the swizzle
+constexpr uint32_t KV_TILE = KT * DH * 2;  // [2 column halves][64 rows][128 B]
+constexpr uint32_t PK_KCODE = 0, PK_VCODE = 2048, PK_KPAR = 4096, PK_VPAR = 6144,
+                   PK_KCOEF = 8192, PK_KCS = 9216, PK_TV = 9344, PK_KIDX = 9472,
+                   PK_VIDX = 9600, PK_BYTES = 9728;
+constexpr uint32_t ST_K = 0, ST_V = KV_TILE, ST_PK = 2 * KV_TILE, ST_BX = ST_PK + PK_BYTES;
+constexpr uint32_t BX_BYTES = KT * 32 * 2;  // [64 keys][<= 32] bf16
+constexpr uint32_t STAGE = (ST_BX + BX_BYTES + 1023) / 1024 * 1024;
+constexpr uint32_t AX_BYTES = QT * 32 * 2;  // [128 rows][<= 32] bf16 per Q tile
+constexpr uint32_t UB_BYTES = 32 * DH * 2;  // [<= 32 rows][128] bf16 per buffer
+constexpr uint32_t OFF_AX = NST * STAGE;
+constexpr uint32_t OFF_UB = OFF_AX + 2 * AX_BYTES;
+constexpr uint32_t OFF_BAR = OFF_UB + 2 * UB_BYTES;
+constexpr int NBAR = 28;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 
 enum {
-  B_KV_FULL = 0,  // [2] dequant (one arrival per warp) -> MMA
-  B_KV_EMPTY = 2, // [2] MMA commit -> dequant
-  B_S_FULL = 4,   // [2] MMA commit -> softmax
-  B_P_FULL = 6,   // [2] softmax (per warp) -> MMA: P of that parity is in TMEM
-  B_AX_FULL = 8,  // [2] softmax (per warp) -> MMA: slab for the tile of that parity
-  B_O_FULL = 11,  // MMA commit after each P V'
-  B_Q_READY = 12, // softmax (per warp) -> MMA
-  B_DONE = 13,    // MMA commit -> MMA (drain before exit)
-  B_O_LAST = 14   // MMA commit after the last P V'
+  B_LOAD_FULL = 0,   // [NST] producer bulk copies (tx bytes) -> dequant
+  B_KV_FULL = 4,     // [NST] dequant (one arrival per warp) -> MMA
+  B_KV_EMPTY = 8,    // [NST] MMA commit after the tile's last P V' -> producer
+  B_S_FULL = 12,     // [2] MMA commit after Q K^T -> softmax of that Q tile
+  B_P_FULL = 14,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
+  B_AXD_FULL = 16,   // [2] MMA commit after Q [U_va | U_vb] -> softmax
+  B_AX_FULL = 18,    // [2] softmax (per warp) -> MMA: AX slab in shared memory
+  B_UB_FULL = 20,    // [2] producer -> MMA: [U_va | U_vb] in buffer
+  B_UB_EMPTY = 22,   // [2] MMA commit after both AX products -> producer
+  B_Q_READY = 24,    // softmax (per warp) -> MMA: Q in TMEM
+  B_O_LAST = 25,     // [2] MMA commit after the last P V' of that Q tile
+  B_DONE = 27        // MMA commit -> MMA (drain before exit)
 };
 
 struct TcArgs {
@@ -105,35 +123,32 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// byte offset of 16-byte chunk c (8 bf16) of row r in a no-swizzle K-major slab
-// with kx columns: core matrices of 8 rows x 16 B, K-adjacent cores 128 B apart,
-// 8-row groups kx*16 B apart.
-__device__ __forceinline__ uint32_t xslab_off(int r, int c, int kx) {
-  return (uint32_t)((r >> 3) * (kx * 16) + c * 128 + (r & 7) * 16);
+// Bounded wait taken by a whole warp; false (on every lane) if any lane gave up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  const bool w = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, w);
 }
 
-// versions in force for the first and the last key of tile j
-__device__ __forceinline__ void tile_versions(const uint16_t* tokver, int64_t T, int j, int& va,
-                                              int& vb) {
+// Versions in force for the first and the last key of tile j, packed as
+// first | last << 16 (read from global memory).
+__device__ __forceinline__ uint32_t tile_pair_global(const uint16_t* tokver, int64_t T, int j) {
   const int64_t t0 = (int64_t)j * KT;
   const int64_t t1 = ((t0 + KT) < T ? (t0 + KT) : T) - 1;
-  va = tokver[t0];
-  vb = tokver[t1];
+  return (uint32_t)tokver[t0] | ((uint32_t)tokver[t1] << 16);
 }
 
-// 32 lanes x 32 fp32 columns to TMEM (the store wait is part of the statement).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
-      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
-      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
-      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
-      "f"(v[29]), "f"(v[30]), "f"(v[31])
-      : "memory");
+// Slab layouts (no swizzle, K-major core matrices of 8 rows x 16 B):
+//   AX  [128 rows][kx]: core (row group g, K column kc) at kc*2048 + g*128
+//   BX  [64 keys][kx] : core (g, kc) at kc*1024 + g*128
+//   UB  [kx rows][128]: core (g, kc) at g*2048 + kc*128
+__device__ __forceinline__ uint32_t ax_off(int m, int kc) {
+  return (uint32_t)(kc * 2048 + (m >> 3) * 128 + (m & 7) * 16);
+}
+__device__ __forceinline__ uint32_t bx_off(int n, int kc) {
+  return (uint32_t)(kc * 1024 + (n >> 3) * 128 + (n & 7) * 16);
+}
+__device__ __forceinline__ uint32_t ub_off(int n, int kc) {
+  return (uint32_t)((n >> 3) * 2048 + kc * 128 + (n & 7) * 16);
 }
 
 // ------------------------------------------------------------------ softmax role
@@ -142,101 +157,99 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 // accumulates in TMEM across tiles, is rescaled in place only on such moves.
 constexpr float TAU = 8.0f;
 
-// Slot `sl` (columns [sl*sw, sl*sw + sw), sw = kx/2) of row `row` of the slab
-// [Q U_va | Q U_vb] for one tile: (U_v^T q) for version v, zeros when v < 0 or
-// past r.
-__device__ __forceinline__ void build_ax(const TcArgs& A, uint8_t* slab, int row, int64_t q,
-                                         int v, int sl) {
-  const Dims& Dm = A.Dm;
-  const int r = Dm.r, kx = A.kx, sw = kx / 2, h = blockIdx.y;
-  float acc[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
-  if (q < A.nq && v >= 0) {
-    const uint4* qrow = reinterpret_cast<const uint4*>(A.Q + ((size_t)q * Dm.H + h) * DH);
-    const float* Uv = basis_of(A.v, Dm, v, h);
-    for (int c = 0; c < 16; ++c) {
-      const uint4 w = __ldg(qrow + c);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float qv = __uint_as_float(e & 1 ? (ww[e / 2] & 0xffff0000u) : (ww[e / 2] << 16));
-        const float* Uj = Uv + (c * 8 + e) * r;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (k < r) acc[k] = fmaf(qv, __ldg(Uj + k), acc[k]);
-      }
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    if (c < sw / 8)
-      *reinterpret_cast<uint4*>(slab + xslab_off(row, sl * (sw / 8) + c, kx)) = make_uint4(
-          pack_bf16(acc[8 * c], acc[8 * c + 1]), pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
-          pack_bf16(acc[8 * c + 4], acc[8 * c + 5]), pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
-  }
-}
-
-__device__ __forceinline__ void build_ax_pair(const TcArgs& A, uint8_t* slab, int row, int64_t q,
-                                              int va, int vb) {
-  build_ax(A, slab, row, q, va, 0);
-  build_ax(A, slab, row, q, vb != va ? vb : -1, 1);
-}
-
 __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
-                                             uint32_t tmem, int ntile) {
-  const int row = threadIdx.x;  // 0..127
-  const int warp = row / 32;
+                                             uint32_t tmem, int ntile, int nqt) {
+  const int warp = threadIdx.x >> 5;
+  const int p = warp >> 2;          // Q tile
+  const int m = threadIdx.x & 127;  // row in the Q tile = TMEM lane
   const int h = blockIdx.y;
   const int H = A.Dm.H;
-  const int64_t q = (int64_t)blockIdx.x * BQ + row;
+  const int kx = A.kx;
+  const int64_t q = (int64_t)blockIdx.x * BQ + p * QT + m;
+  const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  const uint32_t tq = trow + 256 * p, ts = tq + 64, to = tq + 128;
   {
+    // Q row -> TMEM as bf16 pairs (dims 2i, 2i+1 in column i)
     const uint4* src = reinterpret_cast<const uint4*>(A.Q + ((size_t)q * H + h) * DH);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (q < A.nq) val = __ldg(src + c);
-      *reinterpret_cast<uint4*>(smem + OFF_Q + sw128_off(row, c, BQ)) = val;
+    for (int hlf = 0; hlf < 2; ++hlf) {
+      uint32_t w[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (q < A.nq) val = __ldg(src + hlf * 8 + c);
+        w[4 * c] = val.x;
+        w[4 * c + 1] = val.y;
+        w[4 * c + 2] = val.z;
+        w[4 * c + 3] = val.w;
+      }
+      tmem_st32u(tq + 32 * hlf, w);
     }
   }
-  // (va, vb) pair held by slab buffer 0 and 1, packed as va | vb << 16
-  uint32_t ax_pair0 = 0xffffffffu, ax_pair1 = 0xffffffffu;
-  if (A.kx) {
-    for (int j = 0; j < 2 && j < ntile; ++j) {
-      int va, vb;
-      tile_versions(A.v.tokver, A.T, j, va, vb);
-      build_ax_pair(A, smem + OFF_AX + j * XSLAB, row, q, va, vb);
-      if (j == 0) ax_pair0 = (uint32_t)va | ((uint32_t)vb << 16);
-      else ax_pair1 = (uint32_t)va | ((uint32_t)vb << 16);
-    }
-  }
-  fence_proxy_async_smem();
+  tc_fence_before();
   warp_arrive(&bars[B_Q_READY]);
-  if (A.kx) {
-    warp_arrive(&bars[B_AX_FULL + 0]);
-    if (ntile > 1) warp_arrive(&bars[B_AX_FULL + 1]);
-  }
+  if (p >= nqt) return;
 
+  uint8_t* ax = smem + OFF_AX + p * AX_BYTES;
+  // version pairs of tiles j, j+1, j+2 (loaded ahead; only with compensation)
+  uint32_t pr0 = 0, pr1 = 0, pr2 = 0;
+  if (kx) {
+    pr0 = tile_pair_global(A.v.tokver, A.T, 0);
+    if (ntile > 1) pr1 = tile_pair_global(A.v.tokver, A.T, 1);
+    if (ntile > 2) pr2 = tile_pair_global(A.v.tokver, A.T, 2);
+  }
+  uint32_t prev = 0xffffffffu;
+  int nchg = 0;
   float m_used = -INFINITY, l = 0.0f;
-  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-  const uint32_t to = trow + 256;  // O accumulator columns
   const float sl2 = A.scale_log2;
   bool ok = true;
   for (int j = 0; j < ntile; ++j) {
-    const int b = j & 1;
-    bool w = mbar_wait(&bars[B_S_FULL + b], (j >> 1) & 1);
-    if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+    if (kx) {
+      const uint32_t pr = pr0;
+      pr0 = pr1;
+      pr1 = pr2;
+      if (j + 3 < ntile) pr2 = tile_pair_global(A.v.tokver, A.T, j + 3);
+      if (pr != prev) {
+        // AX = Q [U_va | U_vb] (fp32 in the S columns) -> bf16 slab
+        if (!warp_wait(&bars[B_AXD_FULL + p], nchg & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t w[16];
+        if (kx == 16) {
+          float a[16];
+          tmem_ld16(ts, a);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = pack_bf16(a[2 * e], a[2 * e + 1]);
+#pragma unroll
+          for (int e = 8; e < 16; ++e) w[e] = 0u;
+        } else {
+          float a[32];
+          tmem_ld32(ts, a);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = pack_bf16(a[2 * e], a[2 * e + 1]);
+        }
+#pragma unroll
+        for (int kc = 0; kc < 4; ++kc)
+          if (kc < kx / 8)
+            *reinterpret_cast<uint4*>(ax + ax_off(m, kc)) =
+                make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        warp_arrive(&bars[B_AX_FULL + p]);
+        prev = pr;
+        ++nchg;
+      }
+    }
+    if (!warp_wait(&bars[B_S_FULL + p], j & 1)) { ok = false; break; }
     tc_fence_after();
     const int64_t kb = (int64_t)j * KT;
     const int nvalid = (int)((A.T - kb) < KT ? (A.T - kb) : KT);
     float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    {
       float s[64];
-      tmem_ld64(trow + b * 128 + c * 64, s);
+      tmem_ld64(ts, s);
 #pragma unroll
       for (int e = 0; e < 64; ++e)
-        if (c * 64 + e < nvalid) mx = fmaxf(mx, s[e]);
+        if (e < nvalid) mx = fmaxf(mx, s[e]);
     }
     const float m_row = mx * sl2;
     if (j == 0) {
@@ -244,34 +257,29 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     } else {
       const bool need = m_row > m_used + TAU;
       if (__any_sync(0xffffffffu, need)) {
-        // O holds P V' of tiles < j: wait for the last of them, then rescale.
-        // S_FULL(j) implies P V' of tile j-2 is done (commits track all earlier
-        // MMAs) and P V' of tile j cannot start before P_FULL(j), so O_FULL sits
-        // in phase j-1 or j and the parity test is exact.
-        bool w2 = mbar_wait(&bars[B_O_FULL], (j - 1) & 1);
-        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-        tc_fence_after();
+        // O holds P V' of tiles < j, all complete: the commit behind S_FULL(j)
+        // tracks every MMA issued before Q K^T of tile j.
         const float f = need ? ex2(m_used - m_row) : 1.0f;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
           tmem_ld32(to + c * 32, o);
+          uint32_t ou[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(to + c * 32, o);
+          for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e] * f);
+          tmem_st32u(to + c * 32, ou);
         }
         l *= f;
         if (need) m_used = m_row;
       }
     }
-    // P (bf16 pairs) overwrites the S columns already read: keys 2i, 2i+1 of
-    // the tile go to column i of the same TMEM buffer (the A-operand layout of
-    // the P V' MMA).
+    // P (bf16 pairs) over the S columns already read: keys 2i, 2i+1 of the tile
+    // in column i (the A-operand layout of the P V' MMA).
     float lsum = 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float s[32];
-      tmem_ld32(trow + b * 128 + c * 32, s);
+      tmem_ld32(ts + c * 32, s);
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
@@ -281,37 +289,21 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
         lsum += p0 + p1;
         pk[e / 2] = pack_bf16(p0, p1);
       }
-      tmem_st16u(trow + b * 128 + c * 16, pk);
+      tmem_st16u(ts + c * 16, pk);
     }
     l += lsum;
     tc_fence_before();
-    warp_arrive(&bars[B_P_FULL + b]);
-    // slab for tile j+2 into buffer b (QK^T of tile j, its last reader, is done)
-    if (A.kx && j + 2 < ntile) {
-      int va, vb;
-      tile_versions(A.v.tokver, A.T, j + 2, va, vb);
-      const uint32_t pair = (uint32_t)va | ((uint32_t)vb << 16);
-      if (pair != (b ? ax_pair1 : ax_pair0)) {
-        build_ax_pair(A, smem + OFF_AX + b * XSLAB, row, q, va, vb);
-        if (b) ax_pair1 = pair;
-        else ax_pair0 = pair;
-        fence_proxy_async_smem();
-      }
-      warp_arrive(&bars[B_AX_FULL + b]);
-    }
+    warp_arrive(&bars[B_P_FULL + p]);
   }
-  if (ok) {
-    bool w = mbar_wait(&bars[B_O_LAST], 0);
-    ok = __all_sync(0xffffffffu, w);
-  }
+  if (ok) ok = warp_wait(&bars[B_O_LAST + p], 0);
   if (!ok) {
-    if (row == 0) timeout_flag();
+    if ((threadIdx.x & 31) == 0) timeout_flag();
     return;
   }
   tc_fence_after();
   const float inv = 1.0f / l;
   uint4* dst = reinterpret_cast<uint4*>(A.O + ((size_t)q * H + h) * DH);
-#pragma unroll
+#pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     float o[32];
     tmem_ld32(to + c * 32, o);
@@ -332,213 +324,360 @@ __device__ __forceinline__ float code_f(uint32_t bits, int e) {
   return __uint_as_float(0x4B000000u | ((bits >> (2 * e)) & 3u)) - 8388608.0f;
 }
 
+__device__ __forceinline__ int staged_idx(const uint8_t* pk, uint32_t off, int k, int ib) {
+  return ib == 1 ? (int)pk[off + k] : (int)reinterpret_cast<const uint16_t*>(pk + off)[k];
+}
+
+// Issue this thread's 16-byte centroid-chunk copies for tile jj (key row k,
+// channel chunks 4qq..4qq+3 of K and V); one commit group per tile.
+__device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, const PackedHead& ph,
+                                             int jj, int k, int qq) {
+  uint8_t* st = smem + (jj % NST) * STAGE;
+  const int64_t t = (int64_t)jj * KT + k;
+  if (t < A.T) {
+    const int ib = A.Dm.idx_bytes;
+    const int a = staged_idx(st + ST_PK, PK_KIDX, k, ib);
+    const int b = staged_idx(st + ST_PK, PK_VIDX, k, ib);
+    const uint16_t* ck = ph.cent_k + (size_t)a * DH;
+    const uint16_t* cv = ph.cent_v + (size_t)b * DH;
+    const uint32_t sk = smem_u32(st + ST_K), sv = smem_u32(st + ST_V);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = 4 * qq + cc;
+      cp_async16(sk + sw128_off(k, c, KT), ck + c * 8);
+      cp_async16(sv + sw128_off(k, c, KT), cv + c * 8);
+    }
+  }
+  cp_async_commit();
+}
+
 __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              int ntile) {
-  const int dq = threadIdx.x - 128;  // 0..255
-  const int dt = dq >> 1;            // key row in the tile
-  const int hf = dq & 1;             // channel half [64 hf, 64 hf + 64)
+  const int dq = threadIdx.x - 256;  // 0..255
+  const int k = dq >> 2;             // key row in the tile
+  const int qq = dq & 3;             // channel quarter [32 qq, 32 qq + 32)
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
-  const PackedHead p = packed_head(A.v, Dm, h);
+  const PackedHead ph = packed_head(A.v, Dm, h);
   const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
-  for (int j = 0; j < ntile; ++j) {
-    const int slot = j & 1;
-    if (j >= 2) {
-      const bool w = mbar_wait(&bars[B_KV_EMPTY + slot], ((j - 2) >> 1) & 1);
-      if (!__all_sync(0xffffffffu, w)) {
-        timeout_flag();
-        return;
-      }
+  bool ok = true;
+  // prologue: gathers of tiles 0 and 1
+  for (int jj = 0; jj < 2 && jj < ntile; ++jj) {
+    if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
+    issue_gather(A, smem, ph, jj, k, qq);
+  }
+  for (int j = 0; ok && j < ntile; ++j) {
+    const int s = j % NST;
+    if (j + 2 < ntile) {
+      const int j2 = j + 2;
+      if (!warp_wait(&bars[B_LOAD_FULL + j2 % NST], (j2 / NST) & 1)) { ok = false; break; }
+      issue_gather(A, smem, ph, j2, k, qq);
+      cp_async_wait<2>();
+    } else if (j + 1 < ntile) {
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    uint8_t* kb = smem + OFF_K + slot * TILE;
-    uint8_t* vb = smem + OFF_V + slot * TILE;
-    uint8_t* xb = smem + OFF_BX + slot * XSLAB;
-    const int64_t t = (int64_t)j * KT + dt;
+    uint8_t* st = smem + s * STAGE;
+    uint8_t* kb = st + ST_K;
+    uint8_t* vb = st + ST_V;
+    const uint8_t* pk = st + ST_PK;
+    uint8_t* xb = st + ST_BX;
+    const int64_t t0 = (int64_t)j * KT;
+    const int64_t t = t0 + k;
+    const int nvalid = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
     if (t < A.T) {
-      // ---- all loads of this half-row first (memory-level parallelism)
-      const int a = load_idx(p.k_idx, t, Dm.idx_bytes);
-      const int bi = load_idx(p.v_idx, t, Dm.idx_bytes);
-      const uint4* ck = reinterpret_cast<const uint4*>(p.cent_k + (size_t)a * DH) + hf * 8;
-      const uint4* cv = reinterpret_cast<const uint4*>(p.cent_v + (size_t)bi * DH) + hf * 8;
-      uint4 kc[8], vc[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        kc[c] = __ldg(ck + c);
-        vc[c] = __ldg(cv + c);
-      }
-      const uint4 kw4 = __ldg(reinterpret_cast<const uint4*>(p.k_codes + t * (DH / 4)) + hf);
-      const uint4 vw4 = __ldg(reinterpret_cast<const uint4*>(p.v_codes + t * (DH / 4)) + hf);
-      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(p.k_params) + t * ng;
-      const uint32_t* vpar = reinterpret_cast<const uint32_t*>(p.v_params) + t * ng;
-      const int ver = A.v.tokver[t];
+      const uint2 kw = *reinterpret_cast<const uint2*>(pk + PK_KCODE + k * 32 + qq * 8);
+      const uint2 vw = *reinterpret_cast<const uint2*>(pk + PK_VCODE + k * 32 + qq * 8);
+      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(pk + PK_KPAR) + k * ng;
+      const uint32_t* vpar = reinterpret_cast<const uint32_t*>(pk + PK_VPAR) + k * ng;
       bool fallback = false;
       float chat[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) chat[k] = 0.0f;
+      for (int i = 0; i < 16; ++i) chat[i] = 0.0f;
+      int ver = 0;
       if (r > 0) {
-        int va, vbv;
-        tile_versions(A.v.tokver, A.T, j, va, vbv);
+        const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
+        ver = tv[k];
+        const int va = tv[0], vbv = tv[nvalid - 1];
         fallback = (ver != va) && (ver != vbv);
-        if (hf == 0 || fallback) {
-          const float cs = h2f(p.k_cscale[t]);
+        if (qq == 0 || fallback) {
+          const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
+          const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (k < r) chat[k] = (float)p.k_coef[t * r + k] * cs;
+          for (int i = 0; i < 16; ++i)
+            if (i < r) chat[i] = (float)cf[i] * cs;
         }
-        if (hf == 0) {
+        if (qq == 0) {
           // compensation slab row: c8 cs in the slot of the key's version
-          const int sw = kx / 2;
+          // (slot = K columns [0, kx/2) for va, [kx/2, kx) for vb)
           const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c < kx / 8) {
-              const int cs0 = c - (sl >= 0 ? sl * (sw / 8) : 0);
-              const bool mine = sl >= 0 && cs0 >= 0 && cs0 < sw / 8;
+          for (int kc = 0; kc < 4; ++kc) {
+            const bool wide = kx == 32;  // two core columns per slot
+            if (kc < kx / 8) {
+              const int slot = wide ? (kc >> 1) : kc;
+              const bool mine = slot == sl;
               float x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                float v = 0.0f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                  if (mine && m == cs0 * 8 + e) v = chat[m];
-                x[e] = v;
-              }
-              *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) =
+              for (int e = 0; e < 8; ++e)
+                x[e] = mine ? ((wide && (kc & 1)) ? chat[8 + e] : chat[e]) : 0.0f;
+              *reinterpret_cast<uint4*>(xb + bx_off(k, kc)) =
                   make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                              pack_bf16(x[6], x[7]));
             }
           }
         }
       }
-      const float* U = basis_of(A.v, Dm, ver, h);
-      const uint32_t kwv[4] = {kw4.x, kw4.y, kw4.z, kw4.w};
-      const uint32_t vwv[4] = {vw4.x, vw4.y, vw4.z, vw4.w};
+      const float* U = fallback ? basis_of(A.v, Dm, ver, h) : nullptr;
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const int c = hf * 8 + cc;  // chunk of 8 channels within the row
+      for (int cc = 0; cc < 4; ++cc) {
+        // rotating by the quarter keeps the 8 threads of a shared-memory phase
+        // on distinct 16-byte bank groups
+        const int lc = (cc + qq) & 3;  // chunk within the quarter
+        const int c = 4 * qq + lc;     // chunk of 8 channels within the row
         const int j0 = c * 8;
         const int g = j0 / G;
-        const uint32_t kp = __ldg(kpar + g), vp = __ldg(vpar + g);
+        const uint32_t kp = kpar[g], vp = vpar[g];
         const float kmn = h2f((uint16_t)(kp & 0xffff)), ksc = h2f((uint16_t)(kp >> 16));
         const float vmn = h2f((uint16_t)(vp & 0xffff)), vsc = h2f((uint16_t)(vp >> 16));
-        const uint32_t kbits = (kwv[cc / 2] >> (16 * (cc & 1))) & 0xffff;
-        const uint32_t vbits = (vwv[cc / 2] >> (16 * (cc & 1))) & 0xffff;
-        const uint32_t kw[4] = {kc[cc].x, kc[cc].y, kc[cc].z, kc[cc].w};
-        const uint32_t vw[4] = {vc[cc].x, vc[cc].y, vc[cc].z, vc[cc].w};
+        const uint32_t kbits = ((lc < 2 ? kw.x : kw.y) >> (16 * (lc & 1))) & 0xffff;
+        const uint32_t vbits = ((lc < 2 ? vw.x : vw.y) >> (16 * (lc & 1))) & 0xffff;
+        const uint32_t off = sw128_off(k, c, KT);
+        const uint4 kc4 = *reinterpret_cast<const uint4*>(kb + off);
+        const uint4 vc4 = *reinterpret_cast<const uint4*>(vb + off);
+        const uint32_t kwd[4] = {kc4.x, kc4.y, kc4.z, kc4.w};
+        const uint32_t vwd[4] = {vc4.x, vc4.y, vc4.z, vc4.w};
         float kxv[8], vxv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float kcf = __uint_as_float(e & 1 ? (kw[e / 2] & 0xffff0000u) : (kw[e / 2] << 16));
-          const float vcf = __uint_as_float(e & 1 ? (vw[e / 2] & 0xffff0000u) : (vw[e / 2] << 16));
+          const float kcf =
+              __uint_as_float(e & 1 ? (kwd[e / 2] & 0xffff0000u) : (kwd[e / 2] << 16));
+          const float vcf =
+              __uint_as_float(e & 1 ? (vwd[e / 2] & 0xffff0000u) : (vwd[e / 2] << 16));
           kxv[e] = kcf + fmaf(code_f(kbits, e), ksc, kmn);
           vxv[e] = vcf + fmaf(code_f(vbits, e), vsc, vmn);
         }
         if (fallback) {  // a third basis version in this tile: compensate here
+#pragma unroll
           for (int e = 0; e < 8; ++e) {
             float corr = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-              if (k < r) corr = fmaf(__ldg(U + (size_t)(j0 + e) * r + k), chat[k], corr);
+            for (int i = 0; i < 16; ++i)
+              if (i < r) corr = fmaf(__ldg(U + (size_t)(j0 + e) * r + i), chat[i], corr);
             kxv[e] += corr;
           }
         }
-        *reinterpret_cast<uint4*>(kb + sw128_off(dt, c, KT)) =
+        *reinterpret_cast<uint4*>(kb + off) =
             make_uint4(pack_bf16(kxv[0], kxv[1]), pack_bf16(kxv[2], kxv[3]),
                        pack_bf16(kxv[4], kxv[5]), pack_bf16(kxv[6], kxv[7]));
-        *reinterpret_cast<uint4*>(vb + sw128_off(dt, c, KT)) =
+        *reinterpret_cast<uint4*>(vb + off) =
             make_uint4(pack_bf16(vxv[0], vxv[1]), pack_bf16(vxv[2], vxv[3]),
                        pack_bf16(vxv[4], vxv[5]), pack_bf16(vxv[6], vxv[7]));
       }
     } else {
+      // past the end of the cache: zero rows (finite V' under P = 0)
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        *reinterpret_cast<uint4*>(kb + sw128_off(dt, hf * 8 + cc, KT)) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(vb + sw128_off(dt, hf * 8 + cc, KT)) = make_uint4(0, 0, 0, 0);
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t off = sw128_off(k, 4 * qq + cc, KT);
+        *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
       }
-      if (hf == 0) {
+      if (qq == 0) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < kx / 8)
-            *reinterpret_cast<uint4*>(xb + xslab_off(dt, c, kx)) = make_uint4(0, 0, 0, 0);
+        for (int kc = 0; kc < 4; ++kc)
+          if (kc < kx / 8)
+            *reinterpret_cast<uint4*>(xb + bx_off(k, kc)) = make_uint4(0, 0, 0, 0);
       }
     }
     fence_proxy_async_smem();
-    warp_arrive(&bars[B_KV_FULL + slot]);
+    warp_arrive(&bars[B_KV_FULL + s]);
   }
+  cp_async_wait<0>();
+  if (!ok && (threadIdx.x & 31) == 0) timeout_flag();
 }
 
-// ------------------------------------------------------------------ MMA role
-// S[j&1] = Q K-hat_j^T (8 K16 steps over head_dim, two 64-wide swizzled blocks)
-// + the compensation steps [Q U_va | Q U_vb] [c slots]^T.
-__device__ __forceinline__ void issue_qk(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
-                                         int kx) {
-  constexpr uint32_t IDQ = idesc_bf16(128, 128, false, false);
-  const int slot = j & 1;
-  const uint32_t sq = sbase + OFF_Q, sk = sbase + OFF_K + slot * TILE;
+// ------------------------------------------------------------------ producer role
+__device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
+                                              int ntile) {
+  const int lane = threadIdx.x & 31;
+  const Dims& Dm = A.Dm;
+  const int h = blockIdx.y;
+  const PackedHead ph = packed_head(A.v, Dm, h);
+  const int ng = Dm.ng, r = Dm.r, kx = A.kx, ib = Dm.idx_bytes;
+  const uint32_t par_bytes = KT * ng * 4, coef_bytes = KT * r, idx_bytes = KT * ib;
+  const uint32_t tx = 2 * (KT * DH / 4) + 2 * par_bytes + (r > 0 ? coef_bytes + KT * 2 : 0) +
+                      KT * 2 + 2 * idx_bytes;
+  const uint16_t* tokver = A.v.tokver;
+  uint32_t prev = 0xffffffffu;
+  int nchg = 0;
+  bool ok = true;
+  int issued = 0;
+  for (int j = 0; j < ntile; ++j) {
+    const int s = j % NST;
+    if (j >= NST) {
+      if (!warp_wait(&bars[B_KV_EMPTY + s], ((j / NST) - 1) & 1)) { ok = false; break; }
+    }
+    uint8_t* pk = smem + s * STAGE + ST_PK;
+    const int64_t t0 = (int64_t)j * KT;
+    if (lane == 0) {
+      uint64_t* bar = &bars[B_LOAD_FULL + s];
+      mbar_arrive_expect_tx(bar, tx);
+      bulk_g2s(smem_u32(pk + PK_KCODE), ph.k_codes + t0 * (DH / 4), KT * DH / 4, bar);
+      bulk_g2s(smem_u32(pk + PK_VCODE), ph.v_codes + t0 * (DH / 4), KT * DH / 4, bar);
+      bulk_g2s(smem_u32(pk + PK_KPAR), ph.k_params + t0 * ng * 2, par_bytes, bar);
+      bulk_g2s(smem_u32(pk + PK_VPAR), ph.v_params + t0 * ng * 2, par_bytes, bar);
+      if (r > 0) {
+        bulk_g2s(smem_u32(pk + PK_KCOEF), ph.k_coef + t0 * r, coef_bytes, bar);
+        bulk_g2s(smem_u32(pk + PK_KCS), ph.k_cscale + t0, KT * 2, bar);
+      }
+      bulk_g2s(smem_u32(pk + PK_TV), tokver + t0, KT * 2, bar);
+      bulk_g2s(smem_u32(pk + PK_KIDX), (const uint8_t*)ph.k_idx + t0 * ib, idx_bytes, bar);
+      bulk_g2s(smem_u32(pk + PK_VIDX), (const uint8_t*)ph.v_idx + t0 * ib, idx_bytes, bar);
+    }
+    __syncwarp();
+    ++issued;
+    if (kx) {
+      const uint32_t pr = tile_pair_global(tokver, A.T, j);
+      if (pr != prev) {
+        const int b = nchg & 1;
+        if (nchg >= 2) {
+          if (!warp_wait(&bars[B_UB_EMPTY + b], ((nchg >> 1) - 1) & 1)) { ok = false; break; }
+        }
+        // [U_va | U_vb]^T in bf16: row n = slot * sw + i holds column i of the
+        // slot's basis (zeros past r, and slot 1 is zero when va == vb)
+        const int va = (int)(pr & 0xffff), vbv = (int)(pr >> 16);
+        const int sw = kx / 2;
+        uint8_t* ub = smem + OFF_UB + b * UB_BYTES;
+        const int kc = lane & 15;
+        for (int n = lane >> 4; n < kx; n += 2) {
+          const int sl = n / sw, i = n % sw;
+          const int ver = sl == 0 ? va : (vbv != va ? vbv : -1);
+          float x[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t koff = (k >> 2) * (128 * 128) + (k & 3) * 32;
-    mma_bf16_ss(tmem + slot * 128, desc_sw128(sq + koff, 16, 1024),
-                desc_sw128(sk + koff, 16, 1024), IDQ, k > 0);
-  }
-  const uint32_t sa = sbase + OFF_AX + slot * XSLAB, sb = sbase + OFF_BX + slot * XSLAB;
-  for (int k = 0; k < kx / 16; ++k)
-    mma_bf16_ss(tmem + slot * 128, desc_noswz(sa + k * 256, 128, kx * 16),
-                desc_noswz(sb + k * 256, 128, kx * 16), IDQ, 1u);
-  mma_commit(&bars[B_S_FULL + slot]);
-}
-
-// O += P_j V'_j with P read from TMEM (the S buffer of tile j).
-__device__ __forceinline__ void issue_pv(uint64_t* bars, uint32_t sbase, uint32_t tmem, int j,
-                                         int ntile) {
-  constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);
-  const int b = j & 1;
-  const uint32_t sv = sbase + OFF_V + b * TILE;
+          for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+          if (ver >= 0 && i < r) {
+            const float* U = basis_of(A.v, Dm, ver, h);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    // P of keys 16k..16k+15: TMEM columns b*128 + 8k .. +7 (bf16 pairs)
-    mma_bf16_ts(tmem + 256, tmem + b * 128 + k * 8, desc_sw128(sv + k * 2048, KT * 128, 1024),
-                IDP, (j > 0 || k > 0) ? 1u : 0u);
-  }
-  mma_commit(&bars[B_O_FULL]);
-  mma_commit(&bars[B_KV_EMPTY + b]);
-  if (j == ntile - 1) mma_commit(&bars[B_O_LAST]);
-}
-
-// ------------------------------------------------------------------ MMA role
-// Issues whichever MMA group is ready.  Constraints: QK^T of tile j after P V'
-// of tile j-2 has been issued (S/P buffer j&1 is reused; the tensor pipe runs
-// in issue order); P V' of tile j after its P is in TMEM.
-__device__ __forceinline__ void mma_role(uint8_t* smem, uint64_t* bars, uint32_t tmem, int ntile,
-                                         int kx) {
-  const uint32_t sbase = smem_u32(smem);
-  bool ok = mbar_wait(&bars[B_Q_READY], 0);
-  int qn = 0, pn = 0;  // next QK^T tile, next P V' tile
-  long long t_idle = 0;
-  while (ok && pn < ntile) {
-    bool progress = false;
-    if (qn < ntile && qn < pn + 2) {
-      const int slot = qn & 1;
-      if (mbar_test(&bars[B_KV_FULL + slot], (qn >> 1) & 1) &&
-          (!kx || mbar_test(&bars[B_AX_FULL + slot], (qn >> 1) & 1))) {
-        tc_fence_after();
-        issue_qk(bars, sbase, tmem, qn, kx);
-        ++qn;
-        progress = true;
+            for (int e = 0; e < 8; ++e) x[e] = __ldg(U + (size_t)(kc * 8 + e) * r + i);
+          }
+          *reinterpret_cast<uint4*>(ub + ub_off(n, kc)) =
+              make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                         pack_bf16(x[6], x[7]));
+        }
+        fence_proxy_async_smem();
+        warp_arrive(&bars[B_UB_FULL + b]);
+        prev = pr;
+        ++nchg;
       }
     }
-    if (pn < qn && mbar_test(&bars[B_P_FULL + (pn & 1)], (pn >> 1) & 1)) {
+  }
+  // drain: every bulk copy issued has landed before the CTA may exit
+  for (int jj = (issued > NST ? issued - NST : 0); jj < issued; ++jj)
+    if (!warp_wait(&bars[B_LOAD_FULL + jj % NST], (jj / NST) & 1)) ok = false;
+  if (!ok && lane == 0) timeout_flag();
+}
+
+// ------------------------------------------------------------------ MMA role
+// S_p = Q_p K-hat^T (8 K16 steps, A from TMEM) + AX_p BX^T for the tile in stage s.
+__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int p, int s, int kx) {
+  constexpr uint32_t IDQ = idesc_bf16(128, KT, false, false);
+  const uint32_t tq = tmem + 256 * p, ts = tq + 64;
+  const uint32_t sk = sbase + s * STAGE + ST_K;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t koff = (k >> 2) * (KT * 128) + (k & 3) * 32;
+    mma_bf16_ts(ts, tq + 8 * k, desc_sw128(sk + koff, 16, 1024), IDQ, k > 0);
+  }
+  const uint32_t sa = sbase + OFF_AX + p * AX_BYTES, sb = sbase + s * STAGE + ST_BX;
+  for (int k = 0; k < kx / 16; ++k)
+    mma_bf16_ss(ts, desc_noswz(sa + k * 4096, 2048, 128), desc_noswz(sb + k * 2048, 1024, 128),
+                IDQ, 1u);
+}
+
+// O_p += P_p V' (stage s) with P read from TMEM (the S columns of Q tile p).
+__device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int p, int s, bool first) {
+  constexpr uint32_t IDP = idesc_bf16(128, DH, false, true);
+  const uint32_t ts = tmem + 256 * p + 64, to = tmem + 256 * p + 128;
+  const uint32_t sv = sbase + s * STAGE + ST_V;
+#pragma unroll
+  for (int k = 0; k < KT / 16; ++k)
+    mma_bf16_ts(to, ts + 8 * k, desc_sw128(sv + k * 2048, KT * 128, 1024), IDP,
+                (!first || k > 0) ? 1u : 0u);
+}
+
+// AX_p = Q_p [U_va | U_vb] into the S columns of Q tile p.
+__device__ __forceinline__ void issue_ax(uint32_t sbase, uint32_t tmem, int p, int b, int kx) {
+  const uint32_t idx = idesc_bf16(128, kx, false, false);
+  const uint32_t tq = tmem + 256 * p, ts = tq + 64;
+  const uint32_t su = sbase + OFF_UB + b * UB_BYTES;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mma_bf16_ts(ts, tq + 8 * k, desc_noswz(su + 2 * k * 128, 128, 2048), idx, k > 0);
+}
+
+// Issue order per key tile j: P V' of tile j-1, then Q K^T of tile j, for Q
+// tile 0 and then for Q tile 1, so that the tensor pipe runs one Q tile while
+// the softmax works on the other.  When the version pair changes at tile j, both
+// P V'(j-1) and both AX products are issued first, then each Q K^T once its AX
+// slab is in shared memory.  The tensor pipe executes in issue order, so an MMA
+// that overwrites the S/P columns never overtakes the P V' that reads them.
+__device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
+                                         uint32_t tmem, int ntile, int nqt) {
+  const uint32_t sbase = smem_u32(smem);
+  const int kx = A.kx;
+  bool ok = mbar_wait(&bars[B_Q_READY], 0);
+  tc_fence_after();
+  uint32_t prev = 0xffffffffu;
+  int nchg = 0;
+  for (int j = 0; ok && j <= ntile; ++j) {
+    const int s = j % NST, sp = (j + NST - 1) % NST;
+    bool change = false;
+    int b = 0;
+    if (j < ntile) {
+      if (!mbar_wait(&bars[B_KV_FULL + s], (j / NST) & 1)) { ok = false; break; }
       tc_fence_after();
-      issue_pv(bars, sbase, tmem, pn, ntile);
-      ++pn;
-      progress = true;
+      if (kx) {
+        const uint16_t* tv = reinterpret_cast<const uint16_t*>(smem + s * STAGE + ST_PK + PK_TV);
+        const int64_t t0 = (int64_t)j * KT;
+        const int nvalid = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
+        const uint32_t pr = (uint32_t)tv[0] | ((uint32_t)tv[nvalid - 1] << 16);
+        change = pr != prev;
+        prev = pr;
+        if (change) {
+          b = nchg & 1;
+          if (!mbar_wait(&bars[B_UB_FULL + b], (nchg >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+        }
+      }
     }
-    if (progress) {
-      t_idle = 0;
-    } else if (t_idle == 0) {
-      t_idle = clock64();
-    } else if (clock64() - t_idle > (1ll << 31)) {
-      ok = false;
+    for (int p = 0; p < nqt; ++p) {
+      if (j > 0) {
+        if (!mbar_wait(&bars[B_P_FULL + p], (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(sbase, tmem, p, sp, j == 1);
+        if (p == nqt - 1) mma_commit(&bars[B_KV_EMPTY + sp]);
+        if (j == ntile) mma_commit(&bars[B_O_LAST + p]);
+      }
+      if (j < ntile) {
+        if (change) {
+          issue_ax(sbase, tmem, p, b, kx);
+          mma_commit(&bars[B_AXD_FULL + p]);
+          if (p == nqt - 1) mma_commit(&bars[B_UB_EMPTY + b]);
+        } else {
+          issue_qk(sbase, tmem, p, s, kx);
+          mma_commit(&bars[B_S_FULL + p]);
+        }
+      }
+    }
+    if (ok && change) {
+      for (int p = 0; p < nqt; ++p) {
+        if (!mbar_wait(&bars[B_AX_FULL + p], nchg & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_qk(sbase, tmem, p, s, kx);
+        mma_commit(&bars[B_S_FULL + p]);
+      }
+      ++nchg;
     }
   }
   mma_commit(&bars[B_DONE]);
@@ -554,21 +693,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBAR * 8);
   const int warp = threadIdx.x / 32;
   const int ntile = (int)((A.T + KT - 1) / KT);
+  const int nqt = ((int64_t)blockIdx.x * BQ + QT < A.nq) ? 2 : 1;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[B_KV_FULL + i], NDQ / 32);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&bars[B_LOAD_FULL + i], 1);
+      mbar_init(&bars[B_KV_FULL + i], NDQW);
       mbar_init(&bars[B_KV_EMPTY + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[B_S_FULL + i], 1);
       mbar_init(&bars[B_P_FULL + i], 4);
+      mbar_init(&bars[B_AXD_FULL + i], 1);
       mbar_init(&bars[B_AX_FULL + i], 4);
+      mbar_init(&bars[B_UB_FULL + i], 1);
+      mbar_init(&bars[B_UB_EMPTY + i], 1);
+      mbar_init(&bars[B_O_LAST + i], 1);
     }
-    mbar_init(&bars[B_O_FULL], 1);
-    mbar_init(&bars[B_Q_READY], 4);
+    mbar_init(&bars[B_Q_READY], 8);
     mbar_init(&bars[B_DONE], 1);
-    mbar_init(&bars[B_O_LAST], 1);
     fence_mbar_init();
   }
-  if (warp == 12) {
+  if (warp == W_MMA) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -576,17 +721,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  if (warp < 4) {
-    softmax_role(A, smem, bars, tmem, ntile);
-  } else if (warp < 12) {
+  if (warp < 8) {
+    softmax_role(A, smem, bars, tmem, ntile, nqt);
+  } else if (warp < 8 + NDQW) {
     dequant_role(A, smem, bars, ntile);
-  } else if ((threadIdx.x & 31) == 0) {
-    mma_role(smem, bars, tmem, ntile, A.kx);
+  } else if (warp == W_MMA) {
+    if ((threadIdx.x & 31) == 0) mma_role(A, smem, bars, tmem, ntile, nqt);
+    __syncwarp();
+  } else {
+    producer_role(A, smem, bars, ntile);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
-    __syncwarp();
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
