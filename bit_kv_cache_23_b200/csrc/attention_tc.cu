@@ -53,40 +53,46 @@ constexpr int DH = 128;        // head_dim handled here
 constexpr int KT = 64;         // keys per tile
 constexpr int QT = 128;        // query rows per Q tile (TMEM lanes)
 constexpr int BQ = 2 * QT;     // query rows per CTA
-constexpr int NST = 4;         // pipeline stages
-constexpr int NTHREADS = 576;  // 8 softmax + 8 dequant + MMA + producer warps
-constexpr int W_MMA = 16;
+constexpr int NKV = 4;         // K-hat / V' stages (released by the MMA)
+constexpr int NPK = 5;         // packed-field stages (released by the dequant)
+constexpr int NTHREADS = 608;  // 8 softmax + 8 dequant + 2 MMA + producer warps
+constexpr int W_MMA = 16;      // warps 16, 17 issue the MMAs of Q tiles 0, 1
+constexpr int W_PROD = 18;
 constexpr int NDQW = 8;        // dequant warps
 
 // ---- shared memory (bytes); K-hat and V' tiles 1024-aligned for the swizzle
 constexpr uint32_t KV_TILE = KT * DH * 2;  // [2 column halves][64 rows][128 B]
+constexpr uint32_t ST_K = 0, ST_V = KV_TILE, ST_BX = 2 * KV_TILE;
+constexpr uint32_t BX_BYTES = KT * 32 * 2;  // [64 keys][<= 32] bf16
+constexpr uint32_t KVST = ST_BX + BX_BYTES;  // 36 KB
 constexpr uint32_t PK_KCODE = 0, PK_VCODE = 2048, PK_KPAR = 4096, PK_VPAR = 6144,
                    PK_KCOEF = 8192, PK_KCS = 9216, PK_TV = 9344, PK_KIDX = 9472,
                    PK_VIDX = 9600, PK_BYTES = 9728;
-constexpr uint32_t ST_K = 0, ST_V = KV_TILE, ST_PK = 2 * KV_TILE, ST_BX = ST_PK + PK_BYTES;
-constexpr uint32_t BX_BYTES = KT * 32 * 2;  // [64 keys][<= 32] bf16
-constexpr uint32_t STAGE = (ST_BX + BX_BYTES + 1023) / 1024 * 1024;
 constexpr uint32_t AX_BYTES = QT * 32 * 2;  // [128 rows][<= 32] bf16 per Q tile
 constexpr uint32_t UB_BYTES = 32 * DH * 2;  // [<= 32 rows][128] bf16 per buffer
-constexpr uint32_t OFF_AX = NST * STAGE;
+constexpr uint32_t OFF_KV = 0;
+constexpr uint32_t OFF_PK = OFF_KV + NKV * KVST;
+constexpr uint32_t OFF_AX = (OFF_PK + NPK * PK_BYTES + 1023) / 1024 * 1024;
 constexpr uint32_t OFF_UB = OFF_AX + 2 * AX_BYTES;
-constexpr uint32_t OFF_BAR = OFF_UB + 2 * UB_BYTES;
-constexpr int NBAR = 28;
+constexpr uint32_t OFF_INFO = OFF_UB + 2 * UB_BYTES;  // [NKV] version pair of the tile in stage
+constexpr uint32_t OFF_BAR = OFF_INFO + 128;
+constexpr int NBAR = 35;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 
 enum {
-  B_LOAD_FULL = 0,   // [NST] producer bulk copies (tx bytes) -> dequant
-  B_KV_FULL = 4,     // [NST] dequant (one arrival per warp) -> MMA
-  B_KV_EMPTY = 8,    // [NST] MMA commit after the tile's last P V' -> producer
-  B_S_FULL = 12,     // [2] MMA commit after Q K^T -> softmax of that Q tile
-  B_P_FULL = 14,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
-  B_AXD_FULL = 16,   // [2] MMA commit after Q [U_va | U_vb] -> softmax
-  B_AX_FULL = 18,    // [2] softmax (per warp) -> MMA: AX slab in shared memory
-  B_UB_FULL = 20,    // [2] producer -> MMA: [U_va | U_vb] in buffer
-  B_UB_EMPTY = 22,   // [2] MMA commit after both AX products -> producer
-  B_Q_READY = 24,    // softmax (per warp) -> MMA: Q in TMEM
-  B_O_LAST = 25,     // [2] MMA commit after the last P V' of that Q tile
-  B_DONE = 27        // MMA commit -> MMA (drain before exit)
+  B_LOAD_FULL = 0,   // [NPK] producer bulk copies (tx bytes) -> dequant
+  B_PK_EMPTY = 5,    // [NPK] dequant (one arrival per warp) -> producer
+  B_KV_FULL = 10,    // [NKV] dequant (one arrival per warp) -> MMA
+  B_KV_EMPTY = 14,   // [NKV] MMA commit after each Q tile's P V' -> dequant
+  B_S_FULL = 18,     // [2] MMA commit after Q K^T, or after AX on a version change
+  B_P_FULL = 20,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
+  // 22, 23 unused
+  B_AX_FULL = 24,    // [2] softmax (per warp) -> MMA: AX slab in shared memory
+  B_UB_FULL = 26,    // [2] producer -> MMA: [U_va | U_vb] in buffer
+  B_UB_EMPTY = 28,   // [2] MMA commit after the AX products -> producer
+  B_Q_READY = 30,    // softmax (per warp) -> MMA: Q in TMEM
+  B_O_LAST = 31,     // [2] MMA commit after the last P V' of that Q tile
+  B_DONE = 33        // [2] MMA commit -> MMA (drain before exit)
 };
 
 struct TcArgs {
@@ -157,6 +163,25 @@ __device__ __forceinline__ uint32_t ub_off(int n, int kc) {
 // accumulates in TMEM across tiles, is rescaled in place only on such moves.
 constexpr float TAU = 8.0f;
 
+// Row maximum of the first n of 64 scores (n = 64 on all but the last tile).
+__device__ __forceinline__ float row_max(const float (&s)[64], int n) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+  if (n == KT) {
+#pragma unroll
+    for (int e = 0; e < 64; e += 8) {
+      m0 = fmax3(m0, s[e], s[e + 1]);
+      m1 = fmax3(m1, s[e + 2], s[e + 3]);
+      m2 = fmax3(m2, s[e + 4], s[e + 5]);
+      m3 = fmax3(m3, s[e + 6], s[e + 7]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+      if (e < n) m0 = fmaxf(m0, s[e]);
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
 __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              uint32_t tmem, int ntile, int nqt) {
   const int warp = threadIdx.x >> 5;
@@ -191,28 +216,24 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
   if (p >= nqt) return;
 
   uint8_t* ax = smem + OFF_AX + p * AX_BYTES;
-  // version pairs of tiles j, j+1, j+2 (loaded ahead; only with compensation)
-  uint32_t pr0 = 0, pr1 = 0, pr2 = 0;
-  if (kx) {
-    pr0 = tile_pair_global(A.v.tokver, A.T, 0);
-    if (ntile > 1) pr1 = tile_pair_global(A.v.tokver, A.T, 1);
-    if (ntile > 2) pr2 = tile_pair_global(A.v.tokver, A.T, 2);
-  }
+  const uint32_t* kvinfo = reinterpret_cast<const uint32_t*>(smem + OFF_INFO);
   uint32_t prev = 0xffffffffu;
-  int nchg = 0;
-  float m_used = -INFINITY, l = 0.0f;
+  int sph = 0;  // phases of S_FULL seen: one per tile, two when the tile brings AX
+  float m_used = -INFINITY;
+  uint64_t l2 = 0;  // running row sum, as a pair of partial sums
   const float sl2 = A.scale_log2;
+  const uint64_t sc2 = f2pack(sl2, sl2);
   bool ok = true;
   for (int j = 0; j < ntile; ++j) {
+    if (!warp_wait(&bars[B_S_FULL + p], sph & 1)) { ok = false; break; }
+    ++sph;
+    tc_fence_after();
     if (kx) {
-      const uint32_t pr = pr0;
-      pr0 = pr1;
-      pr1 = pr2;
-      if (j + 3 < ntile) pr2 = tile_pair_global(A.v.tokver, A.T, j + 3);
+      // the version pair of the tile (written by the dequant before the stage
+      // was handed to the MMA); on a change the S columns hold AX = Q [U_va | U_vb]
+      const uint32_t pr = kvinfo[j % NKV];
       if (pr != prev) {
-        // AX = Q [U_va | U_vb] (fp32 in the S columns) -> bf16 slab
-        if (!warp_wait(&bars[B_AXD_FULL + p], nchg & 1)) { ok = false; break; }
-        tc_fence_after();
+        prev = pr;
         uint32_t w[16];
         if (kx == 16) {
           float a[16];
@@ -235,23 +256,19 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
         fence_proxy_async_smem();
         tc_fence_before();
         warp_arrive(&bars[B_AX_FULL + p]);
-        prev = pr;
-        ++nchg;
+        if (!warp_wait(&bars[B_S_FULL + p], sph & 1)) { ok = false; break; }
+        ++sph;
+        tc_fence_after();
       }
     }
-    if (!warp_wait(&bars[B_S_FULL + p], j & 1)) { ok = false; break; }
-    tc_fence_after();
     const int64_t kb = (int64_t)j * KT;
     const int nvalid = (int)((A.T - kb) < KT ? (A.T - kb) : KT);
-    float mx = -INFINITY;
+    float m_row;
     {
       float s[64];
       tmem_ld64(ts, s);
-#pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (e < nvalid) mx = fmaxf(mx, s[e]);
+      m_row = row_max(s, nvalid) * sl2;
     }
-    const float m_row = mx * sl2;
     if (j == 0) {
       m_used = m_row;
     } else {
@@ -269,13 +286,13 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
           for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e] * f);
           tmem_st32u(to + c * 32, ou);
         }
-        l *= f;
+        l2 = ffma2(l2, f2pack(f, f), 0ull);
         if (need) m_used = m_row;
       }
     }
     // P (bf16 pairs) over the S columns already read: keys 2i, 2i+1 of the tile
     // in column i (the A-operand layout of the P V' MMA).
-    float lsum = 0.0f;
+    const uint64_t nm2 = f2pack(-m_used, -m_used);
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       float s[32];
@@ -283,15 +300,20 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const int col = c * 32 + e;
-        const float p0 = (col < nvalid) ? ex2(fmaf(s[e], sl2, -m_used)) : 0.0f;
-        const float p1 = (col + 1 < nvalid) ? ex2(fmaf(s[e + 1], sl2, -m_used)) : 0.0f;
-        lsum += p0 + p1;
+        float x0, x1;
+        f2unpack(ffma2(f2pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (nvalid < KT) {
+          const int col = c * 32 + e;
+          if (col >= nvalid) p0 = 0.0f;
+          if (col + 1 >= nvalid) p1 = 0.0f;
+        }
+        const uint64_t pp = f2pack(p0, p1);
+        l2 = fadd2(l2, pp);
         pk[e / 2] = pack_bf16(p0, p1);
       }
       tmem_st16u(ts + c * 16, pk);
     }
-    l += lsum;
     tc_fence_before();
     warp_arrive(&bars[B_P_FULL + p]);
   }
@@ -301,7 +323,9 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
     return;
   }
   tc_fence_after();
-  const float inv = 1.0f / l;
+  float la, lb;
+  f2unpack(l2, la, lb);
+  const float inv = 1.0f / (la + lb);
   uint4* dst = reinterpret_cast<uint4*>(A.O + ((size_t)q * H + h) * DH);
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
@@ -319,33 +343,122 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
 }
 
 // ------------------------------------------------------------------ dequant role
-// exact float of a 2-bit code: (2^23 + code) - 2^23
-__device__ __forceinline__ float code_f(uint32_t bits, int e) {
-  return __uint_as_float(0x4B000000u | ((bits >> (2 * e)) & 3u)) - 8388608.0f;
+// Residual decode without an int-to-float conversion: for the code c of
+// position i (0..3) of a code byte shifted to bits 15..22, OR-ing the masked
+// bits into 1.0f gives exactly 1 + c 2^(2i-8); with S_i = sc 2^(8-2i) and
+// M_i = mn - S_i one fma then yields mn + c sc (S_i is exact, and M_i is exact
+// whenever mn and S_i lie within 2^13 of each other).  Pairs of positions share
+// one f32x2 fma; the centroid is added with one f32x2 add.
+struct GroupConst {
+  uint64_t s01, s23, m01, m23;  // {S_0, S_1}, {S_2, S_3}, {M_0, M_1}, {M_2, M_3}
+};
+
+__device__ __forceinline__ GroupConst group_const(uint32_t par) {
+  const float mn = h2f((uint16_t)(par & 0xffff)), sc = h2f((uint16_t)(par >> 16));
+  const float s0 = sc * 256.0f, s1 = sc * 64.0f, s2 = sc * 16.0f, s3 = sc * 4.0f;
+  GroupConst g;
+  g.s01 = f2pack(s0, s1);
+  g.s23 = f2pack(s2, s3);
+  g.m01 = f2pack(__fsub_rn(mn, s0), __fsub_rn(mn, s1));
+  g.m23 = f2pack(__fsub_rn(mn, s2), __fsub_rn(mn, s3));
+  return g;
+}
+
+__device__ __forceinline__ float magic_code(uint32_t x, int i) {
+  return __uint_as_float((x & (3u << (15 + 2 * i))) | 0x3F800000u);
+}
+
+// Eight channels: centroid chunk cw (bf16 x 8) plus the residual of the 16-bit
+// code word `bits` (channel e at bits 2e), as fp32 pairs.
+__device__ __forceinline__ void deq_chunk_f32(uint4 cw, uint32_t bits, const GroupConst& g,
+                                              uint64_t (&v)[4]) {
+  const uint32_t x0 = bits << 15, x1 = bits << 7;  // channels 0-3, 4-7 at bits 15..22
+  const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+  for (int pi = 0; pi < 4; ++pi) {
+    const uint32_t x = pi < 2 ? x0 : x1;
+    const int i0 = (2 * pi) & 3;
+    const uint64_t mm = f2pack(magic_code(x, i0), magic_code(x, i0 + 1));
+    const uint64_t r = ffma2(mm, i0 == 0 ? g.s01 : g.s23, i0 == 0 ? g.m01 : g.m23);
+    const uint64_t c = f2pack(__uint_as_float(w[pi] << 16), __uint_as_float(w[pi] & 0xffff0000u));
+    v[pi] = fadd2(r, c);
+  }
+}
+
+__device__ __forceinline__ uint4 pack_chunk(const uint64_t (&v)[4]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int pi = 0; pi < 4; ++pi) {
+    float a, b;
+    f2unpack(v[pi], a, b);
+    o[pi] = pack_bf16(a, b);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ int staged_idx(const uint8_t* pk, uint32_t off, int k, int ib) {
   return ib == 1 ? (int)pk[off + k] : (int)reinterpret_cast<const uint16_t*>(pk + off)[k];
 }
 
+// Element-wise compensation U (c8 cs) of channels j0..j0+7 (rare path).
+__device__ __forceinline__ void compensate_chunk(uint64_t (&v2)[4], const float* U, const uint8_t* pk,
+                                              int k, int r, int j0) {
+  const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
+  const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
+  for (int pi = 0; pi < 4; ++pi) {
+    float a, b, ca = 0.0f, cb = 0.0f;
+    f2unpack(v2[pi], a, b);
+    for (int i = 0; i < r; ++i) {
+      const float ch = (float)cf[i] * cs;
+      ca = fmaf(__ldg(U + (size_t)(j0 + 2 * pi) * r + i), ch, ca);
+      cb = fmaf(__ldg(U + (size_t)(j0 + 2 * pi + 1) * r + i), ch, cb);
+    }
+    v2[pi] = f2pack(a + ca, b + cb);
+  }
+}
+
+// One tensor (K or V) of this thread's quarter row: centroid chunks read from
+// the stage, residual added, bf16 written back in place.  U != nullptr adds the
+// element-wise compensation U (c8 cs) (a key whose basis version is not one of
+// the tile's two slots).
+__device__ __forceinline__ void deq_quarter(uint8_t* base, const uint32_t (&offs)[4], uint2 w,
+                                            const uint32_t* par, int G, int qq, const float* U,
+                                            const uint8_t* pk, int k, int r) {
+  uint4 cv[4];
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) cv[cc] = *reinterpret_cast<const uint4*>(base + offs[cc]);
+  GroupConst g;
+  if (G == 32) g = group_const(par[qq]);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int lc = (cc + qq) & 3;  // chunk within the quarter
+    if (G != 32) g = group_const(par[(4 * qq + lc) * 8 / G]);
+    const uint32_t bits = (lc < 2 ? w.x : w.y) >> (16 * (lc & 1));
+    uint64_t v2[4];
+    deq_chunk_f32(cv[cc], bits, g, v2);
+    if (U) compensate_chunk(v2, U, pk, k, r, (4 * qq + lc) * 8);
+    *reinterpret_cast<uint4*>(base + offs[cc]) = pack_chunk(v2);
+  }
+}
+
 // Issue this thread's 16-byte centroid-chunk copies for tile jj (key row k,
 // channel chunks 4qq..4qq+3 of K and V); one commit group per tile.
 __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, const PackedHead& ph,
                                              int jj, int k, int qq) {
-  uint8_t* st = smem + (jj % NST) * STAGE;
+  const uint8_t* pk = smem + OFF_PK + (jj % NPK) * PK_BYTES;
+  const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
   const int64_t t = (int64_t)jj * KT + k;
   if (t < A.T) {
     const int ib = A.Dm.idx_bytes;
-    const int a = staged_idx(st + ST_PK, PK_KIDX, k, ib);
-    const int b = staged_idx(st + ST_PK, PK_VIDX, k, ib);
+    const int a = staged_idx(pk, PK_KIDX, k, ib);
+    const int b = staged_idx(pk, PK_VIDX, k, ib);
     const uint16_t* ck = ph.cent_k + (size_t)a * DH;
     const uint16_t* cv = ph.cent_v + (size_t)b * DH;
-    const uint32_t sk = smem_u32(st + ST_K), sv = smem_u32(st + ST_V);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      const int c = 4 * qq + cc;
-      cp_async16(sk + sw128_off(k, c, KT), ck + c * 8);
-      cp_async16(sv + sw128_off(k, c, KT), cv + c * 8);
+      const int c = 4 * qq + ((cc + qq) & 3);  // same bank-group rotation as the rewrite
+      cp_async16(st + ST_K + sw128_off(k, c, KT), ck + c * 8);
+      cp_async16(st + ST_V + sw128_off(k, c, KT), cv + c * 8);
     }
   }
   cp_async_commit();
@@ -360,17 +473,19 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
   const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
+  uint32_t* kvinfo = reinterpret_cast<uint32_t*>(smem + OFF_INFO);
   bool ok = true;
-  // prologue: gathers of tiles 0 and 1
+  // prologue: gathers of tiles 0 and 1 (their K-hat / V' stages start free)
   for (int jj = 0; jj < 2 && jj < ntile; ++jj) {
     if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
     issue_gather(A, smem, ph, jj, k, qq);
   }
   for (int j = 0; ok && j < ntile; ++j) {
-    const int s = j % NST;
     if (j + 2 < ntile) {
       const int j2 = j + 2;
-      if (!warp_wait(&bars[B_LOAD_FULL + j2 % NST], (j2 / NST) & 1)) { ok = false; break; }
+      if (!warp_wait(&bars[B_LOAD_FULL + j2 % NPK], (j2 / NPK) & 1)) { ok = false; break; }
+      if (j2 >= NKV &&
+          !warp_wait(&bars[B_KV_EMPTY + j2 % NKV], ((j2 / NKV) - 1) & 1)) { ok = false; break; }
       issue_gather(A, smem, ph, j2, k, qq);
       cp_async_wait<2>();
     } else if (j + 1 < ntile) {
@@ -378,103 +493,56 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
     } else {
       cp_async_wait<0>();
     }
-    uint8_t* st = smem + s * STAGE;
+    const int s = j % NKV, sp = j % NPK;
+    uint8_t* st = smem + OFF_KV + s * KVST;
     uint8_t* kb = st + ST_K;
     uint8_t* vb = st + ST_V;
-    const uint8_t* pk = st + ST_PK;
     uint8_t* xb = st + ST_BX;
+    const uint8_t* pk = smem + OFF_PK + sp * PK_BYTES;
     const int64_t t0 = (int64_t)j * KT;
     const int64_t t = t0 + k;
     const int nvalid = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
+    const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
+    const int va = tv[0], vbv = tv[nvalid - 1];
     if (t < A.T) {
       const uint2 kw = *reinterpret_cast<const uint2*>(pk + PK_KCODE + k * 32 + qq * 8);
       const uint2 vw = *reinterpret_cast<const uint2*>(pk + PK_VCODE + k * 32 + qq * 8);
       const uint32_t* kpar = reinterpret_cast<const uint32_t*>(pk + PK_KPAR) + k * ng;
       const uint32_t* vpar = reinterpret_cast<const uint32_t*>(pk + PK_VPAR) + k * ng;
       bool fallback = false;
-      float chat[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) chat[i] = 0.0f;
       int ver = 0;
       if (r > 0) {
-        const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
         ver = tv[k];
-        const int va = tv[0], vbv = tv[nvalid - 1];
         fallback = (ver != va) && (ver != vbv);
-        if (qq == 0 || fallback) {
-          const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
-          const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < r) chat[i] = (float)cf[i] * cs;
-        }
-        if (qq == 0) {
+        if (qq < kx / 8) {
           // compensation slab row: c8 cs in the slot of the key's version
-          // (slot = K columns [0, kx/2) for va, [kx/2, kx) for vb)
+          // (slot = K columns [0, kx/2) for va, [kx/2, kx) for vb); thread qq
+          // writes core column qq (8 columns)
+          const int per = kx / 16;  // core columns per slot: 1 or 2
+          const int slot = qq / per, i0 = (qq % per) * 8;
           const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
+          if (slot == sl) {
+            const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
+            const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
 #pragma unroll
-          for (int kc = 0; kc < 4; ++kc) {
-            const bool wide = kx == 32;  // two core columns per slot
-            if (kc < kx / 8) {
-              const int slot = wide ? (kc >> 1) : kc;
-              const bool mine = slot == sl;
-              float x[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                x[e] = mine ? ((wide && (kc & 1)) ? chat[8 + e] : chat[e]) : 0.0f;
-              *reinterpret_cast<uint4*>(xb + bx_off(k, kc)) =
-                  make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                             pack_bf16(x[6], x[7]));
+            for (int e = 0; e < 8; e += 2) {
+              const float x0 = (i0 + e < r) ? (float)cf[i0 + e] * cs : 0.0f;
+              const float x1 = (i0 + e + 1 < r) ? (float)cf[i0 + e + 1] * cs : 0.0f;
+              w[e / 2] = pack_bf16(x0, x1);
             }
           }
+          *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+      // rotating the chunk order by the quarter keeps the 8 threads of a
+      // shared-memory phase on distinct 16-byte bank groups
+      uint32_t offs[4];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) offs[cc] = sw128_off(k, 4 * qq + ((cc + qq) & 3), KT);
       const float* U = fallback ? basis_of(A.v, Dm, ver, h) : nullptr;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        // rotating by the quarter keeps the 8 threads of a shared-memory phase
-        // on distinct 16-byte bank groups
-        const int lc = (cc + qq) & 3;  // chunk within the quarter
-        const int c = 4 * qq + lc;     // chunk of 8 channels within the row
-        const int j0 = c * 8;
-        const int g = j0 / G;
-        const uint32_t kp = kpar[g], vp = vpar[g];
-        const float kmn = h2f((uint16_t)(kp & 0xffff)), ksc = h2f((uint16_t)(kp >> 16));
-        const float vmn = h2f((uint16_t)(vp & 0xffff)), vsc = h2f((uint16_t)(vp >> 16));
-        const uint32_t kbits = ((lc < 2 ? kw.x : kw.y) >> (16 * (lc & 1))) & 0xffff;
-        const uint32_t vbits = ((lc < 2 ? vw.x : vw.y) >> (16 * (lc & 1))) & 0xffff;
-        const uint32_t off = sw128_off(k, c, KT);
-        const uint4 kc4 = *reinterpret_cast<const uint4*>(kb + off);
-        const uint4 vc4 = *reinterpret_cast<const uint4*>(vb + off);
-        const uint32_t kwd[4] = {kc4.x, kc4.y, kc4.z, kc4.w};
-        const uint32_t vwd[4] = {vc4.x, vc4.y, vc4.z, vc4.w};
-        float kxv[8], vxv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float kcf =
-              __uint_as_float(e & 1 ? (kwd[e / 2] & 0xffff0000u) : (kwd[e / 2] << 16));
-          const float vcf =
-              __uint_as_float(e & 1 ? (vwd[e / 2] & 0xffff0000u) : (vwd[e / 2] << 16));
-          kxv[e] = kcf + fmaf(code_f(kbits, e), ksc, kmn);
-          vxv[e] = vcf + fmaf(code_f(vbits, e), vsc, vmn);
-        }
-        if (fallback) {  // a third basis version in this tile: compensate here
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float corr = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (i < r) corr = fmaf(__ldg(U + (size_t)(j0 + e) * r + i), chat[i], corr);
-            kxv[e] += corr;
-          }
-        }
-        *reinterpret_cast<uint4*>(kb + off) =
-            make_uint4(pack_bf16(kxv[0], kxv[1]), pack_bf16(kxv[2], kxv[3]),
-                       pack_bf16(kxv[4], kxv[5]), pack_bf16(kxv[6], kxv[7]));
-        *reinterpret_cast<uint4*>(vb + off) =
-            make_uint4(pack_bf16(vxv[0], vxv[1]), pack_bf16(vxv[2], vxv[3]),
-                       pack_bf16(vxv[4], vxv[5]), pack_bf16(vxv[6], vxv[7]));
-      }
+      deq_quarter(kb, offs, kw, kpar, G, qq, U, pk, k, r);
+      deq_quarter(vb, offs, vw, vpar, G, qq, nullptr, pk, k, r);
     } else {
       // past the end of the cache: zero rows (finite V' under P = 0)
 #pragma unroll
@@ -483,15 +551,12 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
         *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
       }
-      if (qq == 0) {
-#pragma unroll
-        for (int kc = 0; kc < 4; ++kc)
-          if (kc < kx / 8)
-            *reinterpret_cast<uint4*>(xb + bx_off(k, kc)) = make_uint4(0, 0, 0, 0);
-      }
+      if (qq < kx / 8) *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(0, 0, 0, 0);
     }
+    if (dq == 0) kvinfo[s] = (uint32_t)va | ((uint32_t)vbv << 16);
     fence_proxy_async_smem();
     warp_arrive(&bars[B_KV_FULL + s]);
+    warp_arrive(&bars[B_PK_EMPTY + sp]);
   }
   cp_async_wait<0>();
   if (!ok && (threadIdx.x & 31) == 0) timeout_flag();
@@ -514,11 +579,11 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
   bool ok = true;
   int issued = 0;
   for (int j = 0; j < ntile; ++j) {
-    const int s = j % NST;
-    if (j >= NST) {
-      if (!warp_wait(&bars[B_KV_EMPTY + s], ((j / NST) - 1) & 1)) { ok = false; break; }
+    const int s = j % NPK;
+    if (j >= NPK) {
+      if (!warp_wait(&bars[B_PK_EMPTY + s], ((j / NPK) - 1) & 1)) { ok = false; break; }
     }
-    uint8_t* pk = smem + s * STAGE + ST_PK;
+    uint8_t* pk = smem + OFF_PK + s * PK_BYTES;
     const int64_t t0 = (int64_t)j * KT;
     if (lane == 0) {
       uint64_t* bar = &bars[B_LOAD_FULL + s];
@@ -540,6 +605,8 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
     if (kx) {
       const uint32_t pr = tile_pair_global(tokver, A.T, j);
       if (pr != prev) {
+        // two buffers: the wait is for the change before last, whose tile
+        // precedes this one by at least two, so the MMA can always reach it
         const int b = nchg & 1;
         if (nchg >= 2) {
           if (!warp_wait(&bars[B_UB_EMPTY + b], ((nchg >> 1) - 1) & 1)) { ok = false; break; }
@@ -573,115 +640,109 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
     }
   }
   // drain: every bulk copy issued has landed before the CTA may exit
-  for (int jj = (issued > NST ? issued - NST : 0); jj < issued; ++jj)
-    if (!warp_wait(&bars[B_LOAD_FULL + jj % NST], (jj / NST) & 1)) ok = false;
+  for (int jj = (issued > NPK ? issued - NPK : 0); jj < issued; ++jj)
+    if (!warp_wait(&bars[B_LOAD_FULL + jj % NPK], (jj / NPK) & 1)) ok = false;
   if (!ok && lane == 0) timeout_flag();
 }
 
 // ------------------------------------------------------------------ MMA role
+// Descriptors are built once; a stage or K-step offset is added to the start
+// address field (bytes / 16; no carry out of the 14-bit field in 227 KB).
+struct MmaDesc {
+  uint64_t k, v, bx, ax, ub;
+};
+
 // S_p = Q_p K-hat^T (8 K16 steps, A from TMEM) + AX_p BX^T for the tile in stage s.
-__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int p, int s, int kx) {
+__device__ __forceinline__ void issue_qk(const MmaDesc& D, uint32_t tmem, int p, int s, int kx) {
   constexpr uint32_t IDQ = idesc_bf16(128, KT, false, false);
   const uint32_t tq = tmem + 256 * p, ts = tq + 64;
-  const uint32_t sk = sbase + s * STAGE + ST_K;
+  const uint64_t kd = D.k + (uint64_t)((s * KVST) >> 4);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint32_t koff = (k >> 2) * (KT * 128) + (k & 3) * 32;
-    mma_bf16_ts(ts, tq + 8 * k, desc_sw128(sk + koff, 16, 1024), IDQ, k > 0);
+    const uint32_t koff = ((k >> 2) * (KT * 128) + (k & 3) * 32) >> 4;
+    mma_bf16_ts(ts, tq + 8 * k, kd + koff, IDQ, k > 0);
   }
-  const uint32_t sa = sbase + OFF_AX + p * AX_BYTES, sb = sbase + s * STAGE + ST_BX;
-  for (int k = 0; k < kx / 16; ++k)
-    mma_bf16_ss(ts, desc_noswz(sa + k * 4096, 2048, 128), desc_noswz(sb + k * 2048, 1024, 128),
-                IDQ, 1u);
+  if (kx) {
+    const uint64_t ad = D.ax + (uint64_t)((p * AX_BYTES) >> 4);
+    const uint64_t bd = D.bx + (uint64_t)((s * KVST) >> 4);
+    mma_bf16_ss(ts, ad, bd, IDQ, 1u);
+    if (kx == 32) mma_bf16_ss(ts, ad + (4096 >> 4), bd + (2048 >> 4), IDQ, 1u);
+  }
 }
 
 // O_p += P_p V' (stage s) with P read from TMEM (the S columns of Q tile p).
-__device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int p, int s, bool first) {
+__device__ __forceinline__ void issue_pv(const MmaDesc& D, uint32_t tmem, int p, int s,
+                                         bool first) {
   constexpr uint32_t IDP = idesc_bf16(128, DH, false, true);
   const uint32_t ts = tmem + 256 * p + 64, to = tmem + 256 * p + 128;
-  const uint32_t sv = sbase + s * STAGE + ST_V;
+  const uint64_t vd = D.v + (uint64_t)((s * KVST) >> 4);
 #pragma unroll
   for (int k = 0; k < KT / 16; ++k)
-    mma_bf16_ts(to, ts + 8 * k, desc_sw128(sv + k * 2048, KT * 128, 1024), IDP,
+    mma_bf16_ts(to, ts + 8 * k, vd + (uint64_t)((k * 2048) >> 4), IDP,
                 (!first || k > 0) ? 1u : 0u);
 }
 
 // AX_p = Q_p [U_va | U_vb] into the S columns of Q tile p.
-__device__ __forceinline__ void issue_ax(uint32_t sbase, uint32_t tmem, int p, int b, int kx) {
+__device__ __forceinline__ void issue_ax(const MmaDesc& D, uint32_t tmem, int p, int b, int kx) {
   const uint32_t idx = idesc_bf16(128, kx, false, false);
   const uint32_t tq = tmem + 256 * p, ts = tq + 64;
-  const uint32_t su = sbase + OFF_UB + b * UB_BYTES;
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    mma_bf16_ts(ts, tq + 8 * k, desc_noswz(su + 2 * k * 128, 128, 2048), idx, k > 0);
+    mma_bf16_ts(ts, tq + 8 * k, D.ub + (uint64_t)((b * UB_BYTES + 2 * k * 128) >> 4), idx, k > 0);
 }
 
-// Issue order per key tile j: P V' of tile j-1, then Q K^T of tile j, for Q
-// tile 0 and then for Q tile 1, so that the tensor pipe runs one Q tile while
-// the softmax works on the other.  When the version pair changes at tile j, both
-// P V'(j-1) and both AX products are issued first, then each Q K^T once its AX
-// slab is in shared memory.  The tensor pipe executes in issue order, so an MMA
-// that overwrites the S/P columns never overtakes the P V' that reads them.
+// One issuing thread per Q tile p (warps 16 and 17), each running
+//   Q K^T(p, t) [after AX(p) when the version pair changes at t]
+//     -> wait for the softmax -> P V'(p, t) -> Q K^T(p, t + 1) -> ...
+// with blocking waits; the two threads interleave on the tensor pipe, which
+// works on one Q tile while the softmax works on the other.  Q K^T(p, t + 1) and
+// AX(p) come after P V'(p, t) in the thread's issue order, so an MMA that
+// overwrites the S/P columns never overtakes the P V' that reads them.  A stage
+// is released after both threads' P V' (one commit each).
 __device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
-                                         uint32_t tmem, int ntile, int nqt) {
+                                         uint32_t tmem, int ntile, int p) {
   const uint32_t sbase = smem_u32(smem);
   const int kx = A.kx;
+  MmaDesc D;
+  D.k = desc_sw128(sbase + OFF_KV + ST_K, 16, 1024);
+  D.v = desc_sw128(sbase + OFF_KV + ST_V, KT * 128, 1024);
+  D.bx = desc_noswz(sbase + OFF_KV + ST_BX, 1024, 128);
+  D.ax = desc_noswz(sbase + OFF_AX, 2048, 128);
+  D.ub = desc_noswz(sbase + OFF_UB, 128, 2048);
+  const uint32_t* kvinfo = reinterpret_cast<const uint32_t*>(smem + OFF_INFO);
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
   tc_fence_after();
   uint32_t prev = 0xffffffffu;
   int nchg = 0;
-  for (int j = 0; ok && j <= ntile; ++j) {
-    const int s = j % NST, sp = (j + NST - 1) % NST;
-    bool change = false;
-    int b = 0;
-    if (j < ntile) {
-      if (!mbar_wait(&bars[B_KV_FULL + s], (j / NST) & 1)) { ok = false; break; }
-      tc_fence_after();
-      if (kx) {
-        const uint16_t* tv = reinterpret_cast<const uint16_t*>(smem + s * STAGE + ST_PK + PK_TV);
-        const int64_t t0 = (int64_t)j * KT;
-        const int nvalid = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
-        const uint32_t pr = (uint32_t)tv[0] | ((uint32_t)tv[nvalid - 1] << 16);
-        change = pr != prev;
-        prev = pr;
-        if (change) {
-          b = nchg & 1;
-          if (!mbar_wait(&bars[B_UB_FULL + b], (nchg >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-        }
-      }
-    }
-    for (int p = 0; p < nqt; ++p) {
-      if (j > 0) {
-        if (!mbar_wait(&bars[B_P_FULL + p], (j - 1) & 1)) { ok = false; break; }
+  for (int t = 0; ok && t < ntile; ++t) {
+    const int s = t % NKV;
+    if (!mbar_wait(&bars[B_KV_FULL + s], (t / NKV) & 1)) { ok = false; break; }
+    tc_fence_after();
+    if (kx) {
+      const uint32_t pr = kvinfo[s];
+      if (pr != prev) {
+        const int b = nchg & 1;
+        if (!mbar_wait(&bars[B_UB_FULL + b], (nchg >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        issue_pv(sbase, tmem, p, sp, j == 1);
-        if (p == nqt - 1) mma_commit(&bars[B_KV_EMPTY + sp]);
-        if (j == ntile) mma_commit(&bars[B_O_LAST + p]);
-      }
-      if (j < ntile) {
-        if (change) {
-          issue_ax(sbase, tmem, p, b, kx);
-          mma_commit(&bars[B_AXD_FULL + p]);
-          if (p == nqt - 1) mma_commit(&bars[B_UB_EMPTY + b]);
-        } else {
-          issue_qk(sbase, tmem, p, s, kx);
-          mma_commit(&bars[B_S_FULL + p]);
-        }
-      }
-    }
-    if (ok && change) {
-      for (int p = 0; p < nqt; ++p) {
+        issue_ax(D, tmem, p, b, kx);
+        mma_commit(&bars[B_S_FULL + p]);
+        mma_commit(&bars[B_UB_EMPTY + b]);
         if (!mbar_wait(&bars[B_AX_FULL + p], nchg & 1)) { ok = false; break; }
         tc_fence_after();
-        issue_qk(sbase, tmem, p, s, kx);
-        mma_commit(&bars[B_S_FULL + p]);
+        ++nchg;
+        prev = pr;
       }
-      ++nchg;
     }
+    issue_qk(D, tmem, p, s, kx);
+    mma_commit(&bars[B_S_FULL + p]);
+    if (!mbar_wait(&bars[B_P_FULL + p], t & 1)) { ok = false; break; }
+    tc_fence_after();
+    issue_pv(D, tmem, p, s, t == 0);
+    mma_commit(&bars[B_KV_EMPTY + s]);
+    if (t == ntile - 1) mma_commit(&bars[B_O_LAST + p]);
   }
-  mma_commit(&bars[B_DONE]);
-  if (!mbar_wait(&bars[B_DONE], 0)) ok = false;
+  mma_commit(&bars[B_DONE + p]);
+  if (!mbar_wait(&bars[B_DONE + p], 0)) ok = false;
   if (!ok) timeout_flag();
 }
 
@@ -695,22 +756,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   const int ntile = (int)((A.T + KT - 1) / KT);
   const int nqt = ((int64_t)blockIdx.x * BQ + QT < A.nq) ? 2 : 1;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NST; ++i) {
+    for (int i = 0; i < NPK; ++i) {
       mbar_init(&bars[B_LOAD_FULL + i], 1);
+      mbar_init(&bars[B_PK_EMPTY + i], NDQW);
+    }
+    for (int i = 0; i < NKV; ++i) {
       mbar_init(&bars[B_KV_FULL + i], NDQW);
-      mbar_init(&bars[B_KV_EMPTY + i], 1);
+      mbar_init(&bars[B_KV_EMPTY + i], nqt);  // one commit per Q tile
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[B_S_FULL + i], 1);
       mbar_init(&bars[B_P_FULL + i], 4);
-      mbar_init(&bars[B_AXD_FULL + i], 1);
       mbar_init(&bars[B_AX_FULL + i], 4);
-      mbar_init(&bars[B_UB_FULL + i], 1);
-      mbar_init(&bars[B_UB_EMPTY + i], 1);
       mbar_init(&bars[B_O_LAST + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[B_UB_FULL + i], 1);
+      mbar_init(&bars[B_UB_EMPTY + i], nqt);  // one commit per Q tile
     }
     mbar_init(&bars[B_Q_READY], 8);
     mbar_init(&bars[B_DONE], 1);
+    mbar_init(&bars[B_DONE + 1], 1);
     fence_mbar_init();
   }
   if (warp == W_MMA) {
@@ -725,8 +791,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
     softmax_role(A, smem, bars, tmem, ntile, nqt);
   } else if (warp < 8 + NDQW) {
     dequant_role(A, smem, bars, ntile);
-  } else if (warp == W_MMA) {
-    if ((threadIdx.x & 31) == 0) mma_role(A, smem, bars, tmem, ntile, nqt);
+  } else if (warp < W_PROD) {
+    const int p = warp - W_MMA;
+    if ((threadIdx.x & 31) == 0 && p < nqt) mma_role(A, smem, bars, tmem, ntile, p);
     __syncwarp();
   } else {
     producer_role(A, smem, bars, ntile);
