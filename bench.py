@@ -21,13 +21,13 @@ whole job (all ranks); each rank runs its own replica (weak scaling).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 import numpy as np
@@ -55,52 +55,108 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled during the timed region.
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    Reads NVML from a background thread every 5 ms (read-only queries; nothing
+    is changed on the GPU), so that even a timed region of a few tens of
+    milliseconds is covered; reports None when NVML is not available.
+    """
+
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap")]
+
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []
+        self.thread = None
+        self.stop_flag = threading.Event()
+        self.handle = None
+        self.nv = None
+        self.error = None
+
+    def _open(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        want = str(getattr(props, "uuid", "")).lower().replace("gpu-", "")
+        bus = getattr(props, "pci_bus_id", None)
+        for i in range(nv.nvmlDeviceGetCount()):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            u = nv.nvmlDeviceGetUUID(h)
+            u = (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "")
+            if want and u == want:
+                self.handle = h
+                break
+            if bus is not None and nv.nvmlDeviceGetPciInfo(h).bus == bus:
+                self.handle = h
+        if self.handle is None:
+            raise RuntimeError("no NVML device matches the CUDA device")
+        self.nv = nv
+
+    def _run(self):
+        nv, h = self.nv, self.handle
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, mx, rs))
+            except Exception as e:  # noqa: BLE001 - reported when no sample succeeds
+                self.error = f"{type(e).__name__}: {e}"
+            self.stop_flag.wait(0.005)
 
     def start(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            self._open()
+        except Exception as e:  # noqa: BLE001 - reported in the JSON line
+            self.handle = None
+            self.error = f"{type(e).__name__}: {e}"
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 2.0:  # sampling is live before timing
+            time.sleep(0.001)
+        self.samples.clear()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        if self.thread is None:
+            return {"error": self.error} if self.error else None
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return {"error": self.error or "no sample during the timed region"}
+        nv = self.nv
+        reasons = sorted({name for _, _, rs in self.samples for name, attr in self.REASONS
+                          if hasattr(nv, attr) and rs & getattr(nv, attr)})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml, 5 ms"}
+
+
+# DRAM bytes (read + write) per attention launch on the 480p workload (24 cached
+# frames): ncu dram__bytes_read.sum + dram__bytes_write.sum captured at 6 cached
+# frames and scaled to 24 by the packed-cache bytes (see the attention profile
+# summary).  Valid only for the kernel source it was taken on (hash below).
+ATTN_TRAFFIC = {"sha256_16": "68c66f22ad7c8be4", "config": "480p", "frames": 24,
+                "bytes_per_launch": 62.96e6 + 1.93e6 + (161.7e6 - 40.4e6)}
+
+
+def attention_traffic(cfg) -> float | None:
+    import hashlib
+
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_kv_cache_23_b200", "csrc",
+                       "attention_tc.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if (h != ATTN_TRAFFIC["sha256_16"] or cfg.name != ATTN_TRAFFIC["config"]
+            or cfg.frames != ATTN_TRAFFIC["frames"]):
+        return None
+    return ATTN_TRAFFIC["bytes_per_launch"]
 
 
 # ----------------------------------------------------------------------------- workload
@@ -248,11 +304,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-top1", action="store_true")
+    ap.add_argument("--cache-frames", type=int, default=0,
+                    help="cache length in frames (default: the configuration's); smaller "
+                         "values give the short runs used for ncu captures")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = syn.get_config(args.config)
+    if args.cache_frames > 0:
+        cfg = dataclasses.replace(cfg, frames=args.cache_frames)
     workload_name = (f"{cfg.name} layer: {cfg.heads} heads x {cfg.head_dim}, cache "
                      f"{cfg.frames} latent frames x {cfg.tokens_per_frame} tokens, "
                      f"{cfg.q_rows}-query chunk, C={cfg.n_centroids}, G={cfg.group}, "
@@ -311,10 +372,11 @@ def main():
     # ---- timed region (device time, CUDA events on the launching stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(device)
     clocks.start()
     barrier()
     torch.cuda.synchronize(device)
+    nstep0 = wl.nstep
     start.record()
     for i in range(K):
         wl.step(i, evs[i])
@@ -328,6 +390,9 @@ def main():
     stats_ms, app_ms, att_ms = (float(x) for x in seg.mean(0))
     ms_step = total_ms / K
     value = world * cfg.q_rows / (ms_step * 1e-3)
+    # our kernels in the timed region: per step statistics, append K and V and
+    # attention, plus the refresh kernel on the steps that refresh the basis
+    n_launches = 4 * K + sum(1 for n in range(nstep0, nstep0 + K) if n % cfg.refresh_every == 0)
 
     # ---- end to end through the public API from pinned host memory
     e2e = None
@@ -375,11 +440,14 @@ def main():
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_name,
-                   "l2": "inputs larger than L2: 161 MB packed cache read per step, step inputs rotate over 4 HBM-resident frames",
+                   "l2": (f"packed cache of {T * c.heads * per_tok / 1e6:.0f} MB read per step "
+                          f"({'larger' if T * c.heads * per_tok > 126e6 else 'smaller'} than "
+                          "the 126 MB L2), step inputs rotate over 4 HBM-resident frames"),
                    "parallelism": f"replicas x{world}"},
-        "gpu_launches": 6 * K,
+        "gpu_launches": n_launches,
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16"],
-                     "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"], "traffic": None,
+                     "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
+                     "traffic": attention_traffic(cfg), "traffic_unit": "bytes per launch",
                      "kernel": "qwm_attention", "peak_source": f"{peaks['source']} bf16 burst"},
         "append": {"ms": app_ms, "tokens_per_s": c.tokens_per_frame / (app_ms * 1e-3),
                    "GB_per_s": app_gbs, "frac_hbm": app_gbs / peaks["hbm"],
