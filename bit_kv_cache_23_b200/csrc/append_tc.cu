@@ -19,8 +19,13 @@
 // rescored over all C centroids.
 //
 // One CTA per (head, 128 tokens), 128 threads: thread t owns token t and TMEM
-// lane t.  Thread 0 issues the MMAs.  Phases are separated by __syncthreads;
-// the single mbarrier wait is bounded.
+// lane t and keeps its token row in registers.  Thread 0 issues the MMAs.
+// After the MMAs the -2c tile stays in shared memory and serves as the
+// centroid table for the exact passes (c = -0.5 * (-2c) is exact), so that the
+// rescoring, the QSAC score, the INT2 codes and the PSAC coefficients read
+// centroid rows from shared memory (from global memory only when C exceeds
+// one 256-row tile).  Phases are separated by __syncthreads; the single
+// mbarrier wait is bounded.
 //
 // This file is compiled with --fmad=false; all fused multiply-adds of the
 // canonical definition are explicit __fmaf_rn calls.
@@ -40,7 +45,6 @@ constexpr int TT = 128;        // tokens per CTA
 constexpr int DH = 128;        // head_dim
 constexpr int NCH = 256;       // centroids per MMA chunk (N)
 constexpr int SURV_MAX = 24;   // survivors kept per token before falling back
-constexpr int KROW = 130;      // padded bf16 row of the token tile (conflict-free)
 
 constexpr uint32_t TILE_A = 128 * 128 * 2;           // A hi / lo (SW128 K-major)
 constexpr uint32_t TILE_B = NCH * 128 * 2;           // -2c chunk (SW128 K-major)
@@ -49,8 +53,7 @@ constexpr uint32_t OFF_ALO = OFF_AHI + TILE_A;
 constexpr uint32_t OFF_B = OFF_ALO + TILE_A;
 constexpr uint32_t OFF_AEXT = OFF_B + TILE_B;                 // [128][16] bf16 no swizzle
 constexpr uint32_t OFF_BEXT = OFF_AEXT + 128 * 16 * 2;        // [256][16]
-constexpr uint32_t OFF_KROW = OFF_BEXT + NCH * 16 * 2;        // [128][130] bf16
-constexpr uint32_t OFF_BSUM = OFF_KROW + TT * KROW * 2;       // [512] fp32
+constexpr uint32_t OFF_BSUM = OFF_BEXT + NCH * 16 * 2;        // [512] fp32
 constexpr uint32_t OFF_SURV = OFF_BSUM + 512 * 4;             // [128][SURV_MAX] u16
 constexpr uint32_t OFF_S = OFF_SURV + TT * SURV_MAX * 2;      // [128] s
 constexpr uint32_t OFF_W = OFF_S + 128 * 4;                   // [8] w
@@ -58,8 +61,6 @@ constexpr uint32_t OFF_U = OFF_W + 8 * 4;                     // [128][16] U
 constexpr uint32_t OFF_RED = OFF_U + 128 * 16 * 4;            // [8]
 constexpr uint32_t OFF_BAR = OFF_RED + 8 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 16 + 16 + 1024;
-// PSAC residual scratch [128 channels][128 tokens] fp32 reuses A hi/lo (64 KB)
-constexpr uint32_t OFF_E = OFF_AHI;
 
 struct ApArgs {
   const uint16_t* X;      // [n][H][d] bf16
@@ -85,21 +86,47 @@ __device__ __forceinline__ uint16_t bf16_rn(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-// canonical distance of token row k (padded smem row) to centroid row c (global)
+__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Channels 8q..8q+7 of centroid i as fp32.  With the whole table in the -2c tile
+// (C <= NCH) they come from shared memory: -0.5 * (-2c) restores c exactly,
+// signed zeros included; otherwise from global memory.
+__device__ __forceinline__ void cent_chunk(const uint8_t* bt, const uint16_t* cent, int C, int i,
+                                           int q, float (&c)[8]) {
+  if (C <= NCH) {
+    const uint4 w = *reinterpret_cast<const uint4*>(bt + sw128_off(i, q, NCH));
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      c[2 * e] = __fmul_rn(-0.5f, lo_f(wv[e]));
+      c[2 * e + 1] = __fmul_rn(-0.5f, hi_f(wv[e]));
+    }
+  } else {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(cent + (size_t)i * DH) + q);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      c[2 * e] = lo_f(wv[e]);
+      c[2 * e + 1] = hi_f(wv[e]);
+    }
+  }
+}
+
+// canonical distance of the token (packed bf16 row in registers) to centroid i
 template <bool KEY>
-__device__ __forceinline__ float canon_dist(const uint16_t* krow, const uint16_t* crow,
-                                            const float* s) {
+__device__ __forceinline__ float canon_dist(const uint32_t (&kr)[64], const uint8_t* bt,
+                                            const uint16_t* cent, int C, int i, const float* s) {
   float acc = 0.0f;
-  const uint4* c4 = reinterpret_cast<const uint4*>(crow);
-#pragma unroll 2
+#pragma unroll
   for (int q = 0; q < DH / 8; ++q) {
-    const uint4 cw = __ldg(c4 + q);
-    const uint32_t cv[4] = {cw.x, cw.y, cw.z, cw.w};
+    float c[8];
+    cent_chunk(bt, cent, C, i, q, c);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int j = q * 8 + e;
-      const float cj = __uint_as_float(e & 1 ? (cv[e / 2] & 0xffff0000u) : (cv[e / 2] << 16));
-      const float dl = __fsub_rn(bf2f(krow[j]), cj);
+      const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
+      const float dl = __fsub_rn(kj, c[e]);
       if (KEY) acc = __fmaf_rn(s[j], __fmul_rn(dl, dl), acc);
       else acc = __fmaf_rn(dl, dl, acc);
     }
@@ -107,24 +134,24 @@ __device__ __forceinline__ float canon_dist(const uint16_t* krow, const uint16_t
   return acc;
 }
 
-template <bool KEY>
+template <bool KEY, int G>
 __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8);
-  uint16_t* krow = reinterpret_cast<uint16_t*>(smem + OFF_KROW);
   float* bsum = reinterpret_cast<float*>(smem + OFF_BSUM);
   uint16_t* surv = reinterpret_cast<uint16_t*>(smem + OFF_SURV);
   float* s_s = reinterpret_cast<float*>(smem + OFF_S);
   float* w_s = reinterpret_cast<float*>(smem + OFF_W);
   float* U_s = reinterpret_cast<float*>(smem + OFF_U);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  const uint8_t* bt = smem + OFF_B;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y;
-  const int C = A.C, G = A.G, r = A.r, ng = DH / A.G;
+  const int C = A.C, r = A.r, ng = DH / G;
   const int64_t tok = (int64_t)blockIdx.x * TT + tid;
   const bool valid = tok < A.n;
   const uint16_t* cent = A.cent + (size_t)h * C * DH;
@@ -137,6 +164,20 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
+  // the token row, in registers for every later pass
+  uint32_t kr[64];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(A.X + ((size_t)tok * A.H + h) * DH);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (valid) w = __ldg(src + c);
+      kr[4 * c] = w.x;
+      kr[4 * c + 1] = w.y;
+      kr[4 * c + 2] = w.z;
+      kr[4 * c + 3] = w.w;
+    }
+  }
   // ---- P0: statistics in force; B_i for every centroid; Bmax
   for (int j = tid; j < DH; j += TT) s_s[j] = KEY ? A.sens[(size_t)h * DH + j] : 1.0f;
   if (KEY) {
@@ -148,12 +189,13 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   for (int i = tid; i < C; i += TT) {
     const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
     float acc = 0.0f;
+#pragma unroll 4
     for (int q = 0; q < DH / 8; ++q) {
       const uint4 cw = __ldg(c4 + q);
       const uint32_t cv[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float cj = __uint_as_float(e & 1 ? (cv[e / 2] & 0xffff0000u) : (cv[e / 2] << 16));
+        const float cj = (e & 1) ? hi_f(cv[e / 2]) : lo_f(cv[e / 2]);
         acc = __fmaf_rn(s_s[q * 8 + e], __fmul_rn(cj, cj), acc);
       }
     }
@@ -162,32 +204,26 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   }
   for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
   if (lane == 0) red[warp] = bmax;
-  // ---- P1: token row -> padded smem row, A hi/lo (s*k split), A_t
+  // ---- P1: A hi/lo (s*k split), A_t
   float At = 0.0f;
   {
-    const uint4* src = reinterpret_cast<const uint4*>(A.X + ((size_t)tok * A.H + h) * DH);
     uint8_t* ahi = smem + OFF_AHI;
     uint8_t* alo = smem + OFF_ALO;
-#pragma unroll 2
+#pragma unroll
     for (int c = 0; c < 16; ++c) {
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (valid) w = __ldg(src + c);
-      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
-        reinterpret_cast<uint32_t*>(krow + tid * KROW)[c * 4 + e2] = wv[e2];
-        float sk[2], hv[2];
+        const uint32_t wv = kr[4 * c + e2];
         uint16_t hb[2], lb[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int j = c * 8 + e2 * 2 + u;
-          const float kj = __uint_as_float(u ? (wv[e2] & 0xffff0000u) : (wv[e2] << 16));
+          const float kj = u ? hi_f(wv) : lo_f(wv);
           At = __fmaf_rn(s_s[j], __fmul_rn(kj, kj), At);
-          sk[u] = KEY ? __fmul_rn(s_s[j], kj) : kj;
-          hb[u] = bf16_rn(sk[u]);
-          hv[u] = bf2f(hb[u]);
-          lb[u] = bf16_rn(__fsub_rn(sk[u], hv[u]));
+          const float sk = KEY ? __fmul_rn(s_s[j], kj) : kj;
+          hb[u] = bf16_rn(sk);
+          lb[u] = bf16_rn(__fsub_rn(sk, bf2f(hb[u])));
         }
         hi[e2] = (uint32_t)hb[0] | ((uint32_t)hb[1] << 16);
         lo[e2] = (uint32_t)lb[0] | ((uint32_t)lb[1] << 16);
@@ -214,7 +250,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   bool ok = true;
   for (int ch = 0; ch < nchunk; ++ch) {
     const int c0 = ch * NCH, nc = min(NCH, C - c0);
-    uint8_t* bt = smem + OFF_B;
+    uint8_t* btw = smem + OFF_B;
     uint8_t* bext = smem + OFF_BEXT;
     for (int rr = tid; rr < NCH; rr += TT) {
       const int i = c0 + rr;
@@ -238,7 +274,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
           }
           o[e2] = y;
         }
-        *reinterpret_cast<uint4*>(bt + sw128_off(rr, c, NCH)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(btw + sw128_off(rr, c, NCH)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       const float b = (rr < nc) ? bsum[i] : 0.0f;
       const uint16_t bh = bf16_rn(b);
@@ -337,7 +373,6 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   }
 
   // ---- P5: exact (canonical) distances of the survivors; top-M by (D, i)
-  const uint16_t* kr = krow + tid * KROW;
   int cand[8];
   float candD[8];
 #pragma unroll
@@ -345,9 +380,10 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   if (valid) {
     const bool all = cnt > SURV_MAX || cnt < Mc;  // overflow, or no usable approximation
     const int nloop = all ? C : cnt;
+#pragma unroll 1
     for (int q = 0; q < nloop; ++q) {
       const int i = all ? q : (int)surv[tid * SURV_MAX + q];
-      const float D = canon_dist<KEY>(kr, cent + (size_t)i * DH, s_s);
+      const float D = canon_dist<KEY>(kr, bt, cent, C, i, s_s);
       // insert (D, i) into the sorted candidate list (total order on (D, i))
       float xd = D;
       int xi = i;
@@ -369,110 +405,147 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   }
   if (!valid) return;
 
+  constexpr int NG = DH / G;     // groups per row
+  constexpr int QG = G / 8;      // 8-channel chunks per group
+
   // ---- P6: QSAC stage 2 (keys): expected squared logit perturbation
   int a = cand[0];
   if (KEY && Mc > 1) {
     float best = 0.0f;
     int bm = -1;
+#pragma unroll 1
+    for (int m = 0; m < Mc; ++m) {
+      int cm = cand[0];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      if (m < Mc) {
-        const uint16_t* crow = cent + (size_t)cand[m] * DH;
-        float score = 0.0f;
-        for (int g = 0; g < ng; ++g) {
-          float lo = 0.0f, hi = 0.0f;
-          for (int jj = 0; jj < G; ++jj) {
-            const int j = g * G + jj;
-            const float rho = __fsub_rn(bf2f(kr[j]), bf2f(__ldg(crow + j)));
-            lo = (jj == 0) ? rho : fminf(lo, rho);
-            hi = (jj == 0) ? rho : fmaxf(hi, rho);
+      for (int mm = 0; mm < 8; ++mm)
+        if (mm == m) cm = cand[mm];
+      float score = 0.0f;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+        for (int qi = 0; qi < QG; ++qi) {
+          const int q = g * QG + qi;
+          float c[8];
+          cent_chunk(bt, cent, C, cm, q, c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = q * 8 + e;
+            const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
+            const float rho = __fsub_rn(kj, c[e]);
+            lo = (qi == 0 && e == 0) ? rho : fminf(lo, rho);
+            hi = (qi == 0 && e == 0) ? rho : fmaxf(hi, rho);
           }
-          const float R = __fsub_rn(hi, lo);
-          score = __fmaf_rn(w_s[g], __fmul_rn(R, R), score);
         }
-        if (bm < 0 || score < best) { best = score; bm = m; }
+        const float R = __fsub_rn(hi, lo);
+        score = __fmaf_rn(w_s[g], __fmul_rn(R, R), score);
+      }
+      if (bm < 0 || score < best) {
+        best = score;
+        bm = m;
+        a = cm;
       }
     }
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-      if (m == bm) a = cand[m];
   }
 
-  // ---- P7: INT2 residual, PSAC coefficients, stores
+  // ---- P7: INT2 residual, PSAC coefficients (one pass over the channels), stores
   const size_t slot = (size_t)h * A.tcap + (size_t)(A.t0 + tok);
-  const uint16_t* crow = cent + (size_t)a * DH;
-  float* e_s = reinterpret_cast<float*>(smem + OFF_E);  // [channel][token]
-  for (int g = 0; g < ng; ++g) {
+  float mnv[NG], scv[NG];
+  uint32_t parw[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
     float lo = 0.0f, hi = 0.0f;
-    for (int jj = 0; jj < G; ++jj) {
-      const int j = g * G + jj;
-      const float rho = __fsub_rn(bf2f(kr[j]), bf2f(__ldg(crow + j)));
-      lo = (jj == 0) ? rho : fminf(lo, rho);
-      hi = (jj == 0) ? rho : fmaxf(hi, rho);
+#pragma unroll
+    for (int qi = 0; qi < QG; ++qi) {
+      const int q = g * QG + qi;
+      float c[8];
+      cent_chunk(bt, cent, C, a, q, c);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = q * 8 + e;
+        const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
+        const float rho = __fsub_rn(kj, c[e]);
+        lo = (qi == 0 && e == 0) ? rho : fminf(lo, rho);
+        hi = (qi == 0 && e == 0) ? rho : fmaxf(hi, rho);
+      }
     }
     uint16_t mnh, sch;
-    float mn, sc;
-    int2_params(lo, hi, mnh, sch, mn, sc);
-    reinterpret_cast<uint32_t*>(A.params)[slot * ng + g] = (uint32_t)mnh | ((uint32_t)sch << 16);
-    for (int jb = 0; jb < G; jb += 4) {
-      uint32_t byte = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = g * G + jb + u;
-        const float cj = bf2f(__ldg(crow + j));
-        const float kj = bf2f(kr[j]);
-        const float rho = __fsub_rn(kj, cj);
-        const int code = int2_code(rho, mn, sc);
-        byte |= (uint32_t)code << (2 * u);
-        if (KEY) {
-          const float deq = __fmaf_rn((float)code, sc, mn);
-          e_s[j * TT + tid] = __fsub_rn(kj, __fadd_rn(cj, deq));
-        }
-      }
-      A.codes[slot * (DH / 4) + (g * G + jb) / 4] = (uint8_t)byte;
-    }
+    int2_params(lo, hi, mnh, sch, mnv[g], scv[g]);
+    parw[g] = (uint32_t)mnh | ((uint32_t)sch << 16);
   }
+  float cq[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) cq[i] = 0.0f;
+  uint32_t codew[8];  // 2-bit codes, channel j at bit 2 (j % 16) of word j / 16
+#pragma unroll
+  for (int q = 0; q < DH / 8; ++q) {
+    const int g = q / QG;
+    float c[8];
+    cent_chunk(bt, cent, C, a, q, c);
+    uint32_t bits = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = q * 8 + e;
+      const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
+      const float rho = __fsub_rn(kj, c[e]);
+      const int code = int2_code(rho, mnv[g], scv[g]);
+      bits |= (uint32_t)code << (2 * e);
+      if (KEY) {
+        // PSAC: e_j = k_j - (c_j + deq_j); coef_i accumulates U_ji e_j in channel order
+        const float deq = __fmaf_rn((float)code, scv[g], mnv[g]);
+        const float ej = __fsub_rn(kj, __fadd_rn(c[e], deq));
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < r) cq[i] = __fmaf_rn(U_s[j * r + i], ej, cq[i]);
+      }
+    }
+    if (q & 1) codew[q / 2] |= bits << 16;
+    else codew[q / 2] = bits;
+  }
+  uint4* cdst = reinterpret_cast<uint4*>(A.codes + slot * (DH / 4));
+  cdst[0] = make_uint4(codew[0], codew[1], codew[2], codew[3]);
+  cdst[1] = make_uint4(codew[4], codew[5], codew[6], codew[7]);
+  uint4* pdst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(A.params) + slot * NG);
+#pragma unroll
+  for (int g = 0; g < NG; g += 4) pdst[g / 4] = make_uint4(parw[g], parw[g + 1], parw[g + 2], parw[g + 3]);
   if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
   else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
   if (KEY) {
     if (h == 0) A.tokver[A.t0 + tok] = (uint16_t)A.version;
-    float cq[16];
     float amax = 0.0f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      cq[q] = 0.0f;
-      if (q < r) {
-        float acc = 0.0f;
-        for (int j = 0; j < DH; ++j) acc = __fmaf_rn(U_s[j * r + q], e_s[j * TT + tid], acc);
-        cq[q] = acc;
-        amax = fmaxf(amax, fabsf(acc));
-      }
-    }
+    for (int i = 0; i < 16; ++i)
+      if (i < r) amax = fmaxf(amax, fabsf(cq[i]));
     const uint16_t csh = f2h_ru(__fdiv_rn(amax, 127.0f));
     const float cs = h2f(csh);
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      if (q < r) {
+    for (int i = 0; i < 16; ++i) {
+      if (i < r) {
         int q8 = 0;
         if (cs != 0.0f) {
-          q8 = __float2int_rn(__fdiv_rn(cq[q], cs));
+          q8 = __float2int_rn(__fdiv_rn(cq[i], cs));
           q8 = max(-127, min(127, q8));
         }
-        A.coef[slot * r + q] = (int8_t)q8;
+        A.coef[slot * r + i] = (int8_t)q8;
       }
     }
     A.cscale[slot] = csh;
   }
 }
 
-template <bool KEY>
+template <bool KEY, int G>
 cudaError_t run_tc(const ApArgs& a, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY>,
+  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((a.n + TT - 1) / TT), a.H);
-  append_tc_kernel<KEY><<<grid, TT, SMEM_BYTES, s>>>(a);
+  append_tc_kernel<KEY, G><<<grid, TT, SMEM_BYTES, s>>>(a);
   return cudaGetLastError();
+}
+
+template <bool KEY>
+cudaError_t run_tc_g(const ApArgs& a, cudaStream_t s) {
+  return a.G == 32 ? run_tc<KEY, 32>(a, s) : run_tc<KEY, 16>(a, s);
 }
 
 }  // namespace
@@ -485,7 +558,8 @@ int read_and_clear_append_timeout() {
 }
 
 bool append_tc_supported(const Dims& D) {
-  return D.d == DH && D.C % 16 == 0 && D.C <= 512 && D.M <= 8 && D.r <= 16;
+  return D.d == DH && (D.G == 16 || D.G == 32) && D.C % 16 == 0 && D.C <= 512 && D.M <= 8 &&
+         D.r <= 16;
 }
 
 cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t* K,
@@ -513,7 +587,7 @@ cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t*
   a.coef = v.k_coef;
   a.cscale = v.k_cscale;
   a.tokver = v.tokver;
-  cudaError_t e = run_tc<true>(a, s);
+  cudaError_t e = run_tc_g<true>(a, s);
   if (e != cudaSuccess) return e;
   a.X = V;
   a.cent = v.cent_v;
@@ -522,7 +596,7 @@ cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t*
   a.idx = v.v_idx;
   a.coef = nullptr;
   a.cscale = nullptr;
-  return run_tc<false>(a, s);
+  return run_tc_g<false>(a, s);
 }
 
 }  // namespace qwm

@@ -106,3 +106,47 @@ def test_degenerate_inputs():
     Oref = oc.attention(Q)
     err = np.abs(syn.bf16_bits_to_f32(u16(O)) - Oref)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3
+
+
+@pytest.mark.parametrize("G,C,M,r", [(16, 64, 4, 8), (32, 48, 3, 16), (16, 512, 8, 5)])
+def test_head128_shapes(G, C, M, r):
+    """head_dim 128 with groups of 16, C not a power of two, C = 512 (two MMA
+    chunks), M up to 8 and ranks other than 8: every packed field bit for bit,
+    attention within tolerance; keys with outlier channels and frame drift."""
+    from parity_util import compare_packed
+
+    H, d, n = 3, 128, 700
+    q = pytest.importorskip("bit_kv_cache_23_b200")
+    g = q.QuantKVCache(H, d, C, G, M, r, 3 * n, max_versions=8)
+    oc = oracle.OracleCache(H, d, C, G, M, r, 3 * n)
+    rng = np.random.default_rng(1000 + G + C + r)
+    w = np.ones(d)
+    w[rng.permutation(d)[:6]] = 6.0
+    Kf = [((rng.standard_normal((n, H, d)) + 0.3 * rng.standard_normal(d)) * w).astype(np.float32)
+          for _ in range(3)]
+    K = [syn.f32_to_bf16_bits(x) for x in Kf]
+    V = [syn.f32_to_bf16_bits(rng.standard_normal((n, H, d)).astype(np.float32)) for _ in range(3)]
+    basis = np.linalg.qr(rng.standard_normal((d, 8)))[0]
+    g.build_centroids(to_dev(K[0]), to_dev(V[0]), iters=4)
+    torch.cuda.synchronize()
+    CK = g.view("cent_k").cpu().numpy().view(np.uint16).copy()
+    CV = g.view("cent_v").cpu().numpy().view(np.uint16).copy()
+    oc.set_state(CK=CK, CV=CV)
+    for f in range(3):
+        Q = syn.f32_to_bf16_bits((3.3 * rng.standard_normal((200, H, 8)) @ basis.T
+                                  + 0.5 * rng.standard_normal((200, H, d))).astype(np.float32))
+        g.update_query_stats(to_dev(Q), refresh_basis=True)
+        torch.cuda.synchronize()
+        oc.set_state(s=g.view("sens").cpu().numpy(), w=g.view("wgroup").cpu().numpy(),
+                     U=g.view("basis")[g.version].cpu().numpy())
+        t0 = g.len
+        g.append_kv(to_dev(K[f]), to_dev(V[f]))
+        oc.append_kv(K[f], V[f])
+        assert compare_packed(g, oc, t0, g.len) == {}, f
+    O = g.attention(to_dev(Q))
+    torch.cuda.synchronize()
+    assert q.qwm_device_status() == 0
+    rows = np.arange(0, 200, 13)
+    Oref = oc.attention(Q, rows=rows)
+    err = np.abs(syn.bf16_bits_to_f32(u16(O))[rows] - Oref)
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
