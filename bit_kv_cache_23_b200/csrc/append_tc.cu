@@ -19,7 +19,8 @@
 // rescored over all C centroids.
 //
 // One CTA per (head, 128 tokens), 128 threads: thread t owns token t and TMEM
-// lane t and keeps its token row in registers.  Thread 0 issues the MMAs.
+// lane t; the token rows sit in shared memory (16-byte aligned, conflict-free
+// rows).  Thread 0 issues the MMAs.
 // After the MMAs the -2c tile stays in shared memory and serves as the
 // centroid table for the exact passes (c = -0.5 * (-2c) is exact), so that the
 // rescoring, the QSAC score, the INT2 codes and the PSAC coefficients read
@@ -53,13 +54,15 @@ constexpr uint32_t OFF_ALO = OFF_AHI + TILE_A;
 constexpr uint32_t OFF_B = OFF_ALO + TILE_A;
 constexpr uint32_t OFF_AEXT = OFF_B + TILE_B;                 // [128][16] bf16 no swizzle
 constexpr uint32_t OFF_BEXT = OFF_AEXT + 128 * 16 * 2;        // [256][16]
-constexpr uint32_t OFF_BSUM = OFF_BEXT + NCH * 16 * 2;        // [512] fp32
-constexpr uint32_t OFF_SURV = OFF_BSUM + 512 * 4;             // [128][SURV_MAX] u16
+constexpr uint32_t OFF_SURV = OFF_BEXT + NCH * 16 * 2;        // [128][SURV_MAX] u16
 constexpr uint32_t OFF_S = OFF_SURV + TT * SURV_MAX * 2;      // [128] s
 constexpr uint32_t OFF_W = OFF_S + 128 * 4;                   // [8] w
 constexpr uint32_t OFF_U = OFF_W + 8 * 4;                     // [128][16] U
 constexpr uint32_t OFF_RED = OFF_U + 128 * 16 * 4;            // [8]
-constexpr uint32_t OFF_BAR = OFF_RED + 8 * 4;
+constexpr int KROW = 136;                                     // bf16 row stride (16-B aligned)
+constexpr uint32_t OFF_KROW = OFF_RED + 8 * 4 + 16;           // [128][KROW] bf16 token rows
+constexpr uint32_t OFF_CODE = OFF_KROW + TT * KROW * 2;       // [128][8] u32 code words
+constexpr uint32_t OFF_BAR = OFF_CODE + TT * 8 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 16 + 16 + 1024;
 
 struct ApArgs {
@@ -113,25 +116,45 @@ __device__ __forceinline__ void cent_chunk(const uint8_t* bt, const uint16_t* ce
   }
 }
 
-// canonical distance of the token (packed bf16 row in registers) to centroid i
-template <bool KEY>
-__device__ __forceinline__ float canon_dist(const uint32_t (&kr)[64], const uint8_t* bt,
-                                            const uint16_t* cent, int C, int i, const float* s) {
-  float acc = 0.0f;
+// Channels 8q..8q+7 of this thread's token row (shared memory) as fp32.
+__device__ __forceinline__ void tok_chunk(const uint16_t* krow, int q, float (&k)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(krow + q * 8);
+  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    k[2 * e] = lo_f(wv[e]);
+    k[2 * e + 1] = hi_f(wv[e]);
+  }
+}
+
+// Canonical distances of the token to centroids i0 and i1 (two independent
+// channel-order folds interleaved for instruction-level parallelism).
+template <bool KEY>
+__device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t* bt,
+                                            const uint16_t* cent, int C, int i0, int i1,
+                                            const float* s, float& d0, float& d1) {
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 2
   for (int q = 0; q < DH / 8; ++q) {
-    float c[8];
-    cent_chunk(bt, cent, C, i, q, c);
+    float k[8], c0[8], c1[8];
+    tok_chunk(krow, q, k);
+    cent_chunk(bt, cent, C, i0, q, c0);
+    cent_chunk(bt, cent, C, i1, q, c1);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int j = q * 8 + e;
-      const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
-      const float dl = __fsub_rn(kj, c[e]);
-      if (KEY) acc = __fmaf_rn(s[j], __fmul_rn(dl, dl), acc);
-      else acc = __fmaf_rn(dl, dl, acc);
+      const float l0 = __fsub_rn(k[e], c0[e]), l1 = __fsub_rn(k[e], c1[e]);
+      if (KEY) {
+        a0 = __fmaf_rn(s[j], __fmul_rn(l0, l0), a0);
+        a1 = __fmaf_rn(s[j], __fmul_rn(l1, l1), a1);
+      } else {
+        a0 = __fmaf_rn(l0, l0, a0);
+        a1 = __fmaf_rn(l1, l1, a1);
+      }
     }
   }
-  return acc;
+  d0 = a0;
+  d1 = a1;
 }
 
 template <bool KEY, int G>
@@ -141,7 +164,6 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   uint8_t* smem = smem_raw + pad;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8);
-  float* bsum = reinterpret_cast<float*>(smem + OFF_BSUM);
   uint16_t* surv = reinterpret_cast<uint16_t*>(smem + OFF_SURV);
   float* s_s = reinterpret_cast<float*>(smem + OFF_S);
   float* w_s = reinterpret_cast<float*>(smem + OFF_W);
@@ -164,57 +186,37 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  // the token row, in registers for every later pass
-  uint32_t kr[64];
+  // the token row, in shared memory for every later pass
+  uint16_t* krow = reinterpret_cast<uint16_t*>(smem + OFF_KROW) + tid * KROW;
   {
     const uint4* src = reinterpret_cast<const uint4*>(A.X + ((size_t)tok * A.H + h) * DH);
-#pragma unroll
+#pragma unroll 4
     for (int c = 0; c < 16; ++c) {
       uint4 w = make_uint4(0, 0, 0, 0);
       if (valid) w = __ldg(src + c);
-      kr[4 * c] = w.x;
-      kr[4 * c + 1] = w.y;
-      kr[4 * c + 2] = w.z;
-      kr[4 * c + 3] = w.w;
+      *reinterpret_cast<uint4*>(krow + c * 8) = w;
     }
   }
-  // ---- P0: statistics in force; B_i for every centroid; Bmax
+  // ---- P0: statistics in force
   for (int j = tid; j < DH; j += TT) s_s[j] = KEY ? A.sens[(size_t)h * DH + j] : 1.0f;
   if (KEY) {
     if (tid < ng) w_s[tid] = A.wgroup[(size_t)h * ng + tid];
     for (int e = tid; e < DH * r; e += TT) U_s[e] = A.basis[(size_t)h * DH * r + e];
   }
   __syncthreads();
-  float bmax = 0.0f;
-  for (int i = tid; i < C; i += TT) {
-    const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
-    float acc = 0.0f;
-#pragma unroll 4
-    for (int q = 0; q < DH / 8; ++q) {
-      const uint4 cw = __ldg(c4 + q);
-      const uint32_t cv[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float cj = (e & 1) ? hi_f(cv[e / 2]) : lo_f(cv[e / 2]);
-        acc = __fmaf_rn(s_s[q * 8 + e], __fmul_rn(cj, cj), acc);
-      }
-    }
-    bsum[i] = acc;
-    bmax = fmaxf(bmax, acc);
-  }
-  for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
-  if (lane == 0) red[warp] = bmax;
   // ---- P1: A hi/lo (s*k split), A_t
   float At = 0.0f;
   {
     uint8_t* ahi = smem + OFF_AHI;
     uint8_t* alo = smem + OFF_ALO;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < 16; ++c) {
+      const uint4 w4 = *reinterpret_cast<const uint4*>(krow + c * 8);
+      const uint32_t wk[4] = {w4.x, w4.y, w4.z, w4.w};
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
-        const uint32_t wv = kr[4 * c + e2];
+        const uint32_t wv = wk[e2];
         uint16_t hb[2], lb[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -242,8 +244,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  bmax = 0.0f;
-  for (int wv = 0; wv < TT / 32; ++wv) bmax = fmaxf(bmax, red[wv]);
+  float bmax = 0.0f;  // max of B_i over this thread's centroid rows, then over all
 
   // ---- P2/P3: per chunk of 256 centroids: B operand, MMAs into TMEM columns
   const int nchunk = (C + NCH - 1) / NCH;
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     for (int rr = tid; rr < NCH; rr += TT) {
       const int i = c0 + rr;
       const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
+      float bacc = 0.0f;  // B_i = sum_j s_j c_ij^2, channel order
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {
         uint4 w = make_uint4(0, 0, 0, 0);
@@ -269,6 +271,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
           for (int u = 0; u < 2; ++u) {
             const uint32_t hbits = (x >> (16 * u)) & 0xffffu;
             const float f = __uint_as_float(hbits << 16);
+            bacc = __fmaf_rn(s_s[c * 8 + e2 * 2 + u], __fmul_rn(f, f), bacc);
             const uint16_t m2 = bf16_rn(-2.0f * f);
             y |= (uint32_t)m2 << (16 * u);
           }
@@ -276,7 +279,8 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
         }
         *reinterpret_cast<uint4*>(btw + sw128_off(rr, c, NCH)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      const float b = (rr < nc) ? bsum[i] : 0.0f;
+      const float b = (rr < nc) ? bacc : 0.0f;
+      bmax = fmaxf(bmax, b);
       const uint16_t bh = bf16_rn(b);
       const uint16_t bl = bf16_rn(__fsub_rn(b, bf2f(bh)));
       *reinterpret_cast<uint4*>(bext + (rr >> 3) * 256 + (rr & 7) * 16) =
@@ -316,6 +320,10 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   if (!__syncthreads_and(ok)) {
     if (tid == 0) atomicExch(&g_append_timeout, 1);
   }
+  for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+  if (lane == 0) red[warp] = bmax;
+  __syncthreads();
+  bmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
 
   // ---- P4: selection from the approximations (thread t, TMEM lane t)
   const int Mc = KEY ? A.M : 1;
@@ -327,22 +335,28 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   const float E = 2.4414062e-4f * sqrtf(At * bmax) + 1.2207031e-4f * bmax;  // 2^-12, 2^-13
   const float gam = 3.0517578e-5f;                                           // 2^-15
   const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+  // dM >= the M-th smallest d~: the M-th smallest of the minima of groups of 8
+  // columns (M groups hold an element no larger than it).  Group minima are
+  // four independent chains per 32 columns; only they enter the sorted list.
   float topv[8];
 #pragma unroll
   for (int m = 0; m < 8; ++m) topv[m] = INFINITY;
+#pragma unroll 1
   for (int c0 = 0; c0 < nchunk * NCH; c0 += 32) {
     float v[32];
     tmem_ld32(trow + c0, v);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      if (c0 + e < C && v[e] < topv[7]) {
-        float x = v[e];
+    for (int gq = 0; gq < 4; ++gq) {
+      float x = INFINITY;
+      if (c0 + 8 * gq < C) {  // C is a multiple of 16: groups are all valid or all not
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {  // insertion into the sorted list
-          const float lo = fminf(topv[m], x);
-          x = fmaxf(topv[m], x);
-          topv[m] = lo;
-        }
+        for (int e = 0; e < 8; ++e) x = fminf(x, v[8 * gq + e]);
+      }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {  // insertion into the sorted list
+        const float lo = fminf(topv[m], x);
+        x = fmaxf(topv[m], x);
+        topv[m] = lo;
       }
     }
   }
@@ -354,6 +368,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   float theta = (tau + E + gam * (At + E)) / (1.0f - gam);
   theta += 1e-6f * (fabsf(theta) + At) + 1e-30f;
   int cnt = 0;
+#pragma unroll 1
   for (int c0 = 0; c0 < nchunk * NCH; c0 += 32) {
     float v[32];
     tmem_ld32(trow + c0, v);
@@ -381,23 +396,31 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     const bool all = cnt > SURV_MAX || cnt < Mc;  // overflow, or no usable approximation
     const int nloop = all ? C : cnt;
 #pragma unroll 1
-    for (int q = 0; q < nloop; ++q) {
-      const int i = all ? q : (int)surv[tid * SURV_MAX + q];
-      const float D = canon_dist<KEY>(kr, bt, cent, C, i, s_s);
-      // insert (D, i) into the sorted candidate list (total order on (D, i))
-      float xd = D;
-      int xi = i;
+    for (int q = 0; q < nloop; q += 2) {
+      const int i0 = all ? q : (int)surv[tid * SURV_MAX + q];
+      const bool two = q + 1 < nloop;
+      const int i1 = two ? (all ? q + 1 : (int)surv[tid * SURV_MAX + q + 1]) : i0;
+      float D0, D1;
+      canon_dist2<KEY>(krow, bt, cent, C, i0, i1, s_s, D0, D1);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        if (m < Mc) {
-          const bool sw = (candD[m] == INFINITY && cand[m] < 0) || lex_less(xd, xi, candD[m], cand[m]);
-          if (sw) {
-            const float td = candD[m];
-            const int ti = cand[m];
-            candD[m] = xd;
-            cand[m] = xi;
-            xd = td;
-            xi = ti;
+      for (int u = 0; u < 2; ++u) {
+        if (u == 1 && !two) break;
+        // insert (D, i) into the sorted candidate list (total order on (D, i))
+        float xd = u ? D1 : D0;
+        int xi = u ? i1 : i0;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          if (m < Mc) {
+            const bool sw =
+                (candD[m] == INFINITY && cand[m] < 0) || lex_less(xd, xi, candD[m], cand[m]);
+            if (sw) {
+              const float td = candD[m];
+              const int ti = cand[m];
+              candD[m] = xd;
+              cand[m] = xi;
+              xd = td;
+              xi = ti;
+            }
           }
         }
       }
@@ -420,19 +443,18 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
       for (int mm = 0; mm < 8; ++mm)
         if (mm == m) cm = cand[mm];
       float score = 0.0f;
-#pragma unroll
+#pragma unroll 1
       for (int g = 0; g < NG; ++g) {
         float lo = 0.0f, hi = 0.0f;
 #pragma unroll
         for (int qi = 0; qi < QG; ++qi) {
           const int q = g * QG + qi;
-          float c[8];
+          float k[8], c[8];
+          tok_chunk(krow, q, k);
           cent_chunk(bt, cent, C, cm, q, c);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int j = q * 8 + e;
-            const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
-            const float rho = __fsub_rn(kj, c[e]);
+            const float rho = __fsub_rn(k[e], c[e]);
             lo = (qi == 0 && e == 0) ? rho : fminf(lo, rho);
             hi = (qi == 0 && e == 0) ? rho : fmaxf(hi, rho);
           }
@@ -448,66 +470,75 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     }
   }
 
-  // ---- P7: INT2 residual, PSAC coefficients (one pass over the channels), stores
+  // ---- P7: INT2 residual and PSAC coefficients, group by group in channel order
   const size_t slot = (size_t)h * A.tcap + (size_t)(A.t0 + tok);
-  float mnv[NG], scv[NG];
-  uint32_t parw[NG];
+  uint32_t* codew = reinterpret_cast<uint32_t*>(smem + OFF_CODE) + tid * 8;
+  uint32_t* pdst = reinterpret_cast<uint32_t*>(A.params) + slot * NG;
+  float cq[16];
 #pragma unroll
+  for (int i = 0; i < 16; ++i) cq[i] = 0.0f;
+#pragma unroll 1
   for (int g = 0; g < NG; ++g) {
     float lo = 0.0f, hi = 0.0f;
 #pragma unroll
     for (int qi = 0; qi < QG; ++qi) {
       const int q = g * QG + qi;
-      float c[8];
+      float k[8], c[8];
+      tok_chunk(krow, q, k);
       cent_chunk(bt, cent, C, a, q, c);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int j = q * 8 + e;
-        const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
-        const float rho = __fsub_rn(kj, c[e]);
+        const float rho = __fsub_rn(k[e], c[e]);
         lo = (qi == 0 && e == 0) ? rho : fminf(lo, rho);
         hi = (qi == 0 && e == 0) ? rho : fmaxf(hi, rho);
       }
     }
     uint16_t mnh, sch;
-    int2_params(lo, hi, mnh, sch, mnv[g], scv[g]);
-    parw[g] = (uint32_t)mnh | ((uint32_t)sch << 16);
-  }
-  float cq[16];
+    float mn, sc;
+    int2_params(lo, hi, mnh, sch, mn, sc);
+    pdst[g] = (uint32_t)mnh | ((uint32_t)sch << 16);
+#pragma unroll 1
+    for (int qi = 0; qi < QG; ++qi) {
+      const int q = g * QG + qi;
+      float k[8], c[8];
+      tok_chunk(krow, q, k);
+      cent_chunk(bt, cent, C, a, q, c);
+      uint32_t bits = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) cq[i] = 0.0f;
-  uint32_t codew[8];  // 2-bit codes, channel j at bit 2 (j % 16) of word j / 16
+      for (int e = 0; e < 8; ++e) {
+        const int j = q * 8 + e;
+        const float rho = __fsub_rn(k[e], c[e]);
+        const int code = int2_code(rho, mn, sc);
+        bits |= (uint32_t)code << (2 * e);
+        if (KEY) {
+          // PSAC: e_j = k_j - (c_j + deq_j); coefficient i accumulates U_ji e_j in channel order
+          const float deq = __fmaf_rn((float)code, sc, mn);
+          const float ej = __fsub_rn(k[e], __fadd_rn(c[e], deq));
+          const float* Uj = U_s + j * r;
+          if (r == 8) {
+            const float4 u0 = *reinterpret_cast<const float4*>(Uj);
+            const float4 u1 = *reinterpret_cast<const float4*>(Uj + 4);
+            cq[0] = __fmaf_rn(u0.x, ej, cq[0]);
+            cq[1] = __fmaf_rn(u0.y, ej, cq[1]);
+            cq[2] = __fmaf_rn(u0.z, ej, cq[2]);
+            cq[3] = __fmaf_rn(u0.w, ej, cq[3]);
+            cq[4] = __fmaf_rn(u1.x, ej, cq[4]);
+            cq[5] = __fmaf_rn(u1.y, ej, cq[5]);
+            cq[6] = __fmaf_rn(u1.z, ej, cq[6]);
+            cq[7] = __fmaf_rn(u1.w, ej, cq[7]);
+          } else {
 #pragma unroll
-  for (int q = 0; q < DH / 8; ++q) {
-    const int g = q / QG;
-    float c[8];
-    cent_chunk(bt, cent, C, a, q, c);
-    uint32_t bits = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int j = q * 8 + e;
-      const float kj = (e & 1) ? hi_f(kr[j / 2]) : lo_f(kr[j / 2]);
-      const float rho = __fsub_rn(kj, c[e]);
-      const int code = int2_code(rho, mnv[g], scv[g]);
-      bits |= (uint32_t)code << (2 * e);
-      if (KEY) {
-        // PSAC: e_j = k_j - (c_j + deq_j); coef_i accumulates U_ji e_j in channel order
-        const float deq = __fmaf_rn((float)code, scv[g], mnv[g]);
-        const float ej = __fsub_rn(kj, __fadd_rn(c[e], deq));
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (i < r) cq[i] = __fmaf_rn(U_s[j * r + i], ej, cq[i]);
+            for (int i = 0; i < 16; ++i)
+              if (i < r) cq[i] = __fmaf_rn(Uj[i], ej, cq[i]);
+          }
+        }
       }
+      reinterpret_cast<uint16_t*>(codew)[q] = (uint16_t)bits;
     }
-    if (q & 1) codew[q / 2] |= bits << 16;
-    else codew[q / 2] = bits;
   }
   uint4* cdst = reinterpret_cast<uint4*>(A.codes + slot * (DH / 4));
-  cdst[0] = make_uint4(codew[0], codew[1], codew[2], codew[3]);
-  cdst[1] = make_uint4(codew[4], codew[5], codew[6], codew[7]);
-  uint4* pdst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(A.params) + slot * NG);
-#pragma unroll
-  for (int g = 0; g < NG; g += 4) pdst[g / 4] = make_uint4(parw[g], parw[g + 1], parw[g + 2], parw[g + 3]);
+  cdst[0] = *reinterpret_cast<const uint4*>(codew);
+  cdst[1] = *reinterpret_cast<const uint4*>(codew + 4);
   if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
   else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
   if (KEY) {
