@@ -42,28 +42,32 @@ __device__ int g_append_timeout;
 namespace {
 using namespace tc;
 
-constexpr int TT = 128;        // tokens per CTA
 constexpr int DH = 128;        // head_dim
 constexpr int NCH = 256;       // centroids per MMA chunk (N)
-constexpr int SURV_MAX = 24;   // survivors kept per token before falling back
+constexpr int SURV_MAX = 16;   // survivors kept per token before falling back
+constexpr int KROW = 136;      // bf16 row stride of the token rows (16-byte aligned)
 
-constexpr uint32_t TILE_A = 128 * 128 * 2;           // A hi / lo (SW128 K-major)
-constexpr uint32_t TILE_B = NCH * 128 * 2;           // -2c chunk (SW128 K-major)
-constexpr uint32_t OFF_AHI = 0;
-constexpr uint32_t OFF_ALO = OFF_AHI + TILE_A;
-constexpr uint32_t OFF_B = OFF_ALO + TILE_A;
-constexpr uint32_t OFF_AEXT = OFF_B + TILE_B;                 // [128][16] bf16 no swizzle
-constexpr uint32_t OFF_BEXT = OFF_AEXT + 128 * 16 * 2;        // [256][16]
-constexpr uint32_t OFF_SURV = OFF_BEXT + NCH * 16 * 2;        // [128][SURV_MAX] u16
-constexpr uint32_t OFF_S = OFF_SURV + TT * SURV_MAX * 2;      // [128] s
-constexpr uint32_t OFF_W = OFF_S + 128 * 4;                   // [8] w
-constexpr uint32_t OFF_U = OFF_W + 8 * 4;                     // [128][16] U
-constexpr uint32_t OFF_RED = OFF_U + 128 * 16 * 4;            // [8]
-constexpr int KROW = 136;                                     // bf16 row stride (16-B aligned)
-constexpr uint32_t OFF_KROW = OFF_RED + 8 * 4 + 16;           // [128][KROW] bf16 token rows
-constexpr uint32_t OFF_CODE = OFF_KROW + TT * KROW * 2;       // [128][8] u32 code words
-constexpr uint32_t OFF_BAR = OFF_CODE + TT * 8 * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 16 + 16 + 1024;
+// Shared memory for a CTA of NT threads (NT tokens: 128, or 256 when C <= 256
+// and the tokens go through the MMA in two halves of 128 rows).
+template <int NT>
+struct Lay {
+  static constexpr uint32_t TILE_A = 128 * 128 * 2;                // A hi / lo (SW128 K-major)
+  static constexpr uint32_t TILE_B = NCH * 128 * 2;                // -2c chunk (SW128 K-major)
+  static constexpr uint32_t AHI = 0;
+  static constexpr uint32_t ALO = AHI + TILE_A;
+  static constexpr uint32_t B = ALO + TILE_A;
+  static constexpr uint32_t AEXT = B + TILE_B;                     // [128][16] bf16 no swizzle
+  static constexpr uint32_t BEXT = AEXT + 128 * 16 * 2;            // [256][16]
+  static constexpr uint32_t SURV = BEXT + NCH * 16 * 2;            // [NT][SURV_MAX] u16
+  static constexpr uint32_t S = SURV + NT * SURV_MAX * 2;          // [128] s
+  static constexpr uint32_t W = S + 128 * 4;                       // [8] w
+  static constexpr uint32_t U = W + 8 * 4;                         // [128][16] U
+  static constexpr uint32_t RED = U + 128 * 16 * 4;                // [8]
+  static constexpr uint32_t KR = RED + 8 * 4 + 16;                 // [NT][KROW] bf16 token rows
+  static constexpr uint32_t BAR = KR + NT * KROW * 2;
+  static constexpr uint32_t BYTES = BAR + 16 + 16 + 1024;
+};
+static_assert(Lay<256>::BYTES <= 227 * 1024, "shared memory of the 256-token CTA");
 
 struct ApArgs {
   const uint16_t* X;      // [n][H][d] bf16
@@ -157,24 +161,27 @@ __device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t*
   d1 = a1;
 }
 
-template <bool KEY, int G>
-__global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
+template <bool KEY, int G, int NT>
+__global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
+  using L = Lay<NT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8);
-  uint16_t* surv = reinterpret_cast<uint16_t*>(smem + OFF_SURV);
-  float* s_s = reinterpret_cast<float*>(smem + OFF_S);
-  float* w_s = reinterpret_cast<float*>(smem + OFF_W);
-  float* U_s = reinterpret_cast<float*>(smem + OFF_U);
-  float* red = reinterpret_cast<float*>(smem + OFF_RED);
-  const uint8_t* bt = smem + OFF_B;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR + 8);
+  uint16_t* surv = reinterpret_cast<uint16_t*>(smem + L::SURV);
+  float* s_s = reinterpret_cast<float*>(smem + L::S);
+  float* w_s = reinterpret_cast<float*>(smem + L::W);
+  float* U_s = reinterpret_cast<float*>(smem + L::U);
+  float* red = reinterpret_cast<float*>(smem + L::RED);
+  const uint8_t* bt = smem + L::B;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int half = tid >> 7;     // MMA half of the CTA's tokens (TMEM columns half * NCH)
+  const int row = tid & 127;     // row of the half = TMEM lane
   const int h = blockIdx.y;
   const int C = A.C, r = A.r, ng = DH / G;
-  const int64_t tok = (int64_t)blockIdx.x * TT + tid;
+  const int64_t tok = (int64_t)blockIdx.x * NT + tid;
   const bool valid = tok < A.n;
   const uint16_t* cent = A.cent + (size_t)h * C * DH;
 
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
     tmem_relinquish();
   }
   // the token row, in shared memory for every later pass
-  uint16_t* krow = reinterpret_cast<uint16_t*>(smem + OFF_KROW) + tid * KROW;
+  uint16_t* krow = reinterpret_cast<uint16_t*>(smem + L::KR) + tid * KROW;
   {
     const uint4* src = reinterpret_cast<const uint4*>(A.X + ((size_t)tok * A.H + h) * DH);
 #pragma unroll 4
@@ -197,63 +204,36 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
       *reinterpret_cast<uint4*>(krow + c * 8) = w;
     }
   }
-  // ---- P0: statistics in force
-  for (int j = tid; j < DH; j += TT) s_s[j] = KEY ? A.sens[(size_t)h * DH + j] : 1.0f;
+  // ---- P0: statistics in force; the constant rows of the extra A step
+  for (int j = tid; j < DH; j += NT) s_s[j] = KEY ? A.sens[(size_t)h * DH + j] : 1.0f;
   if (KEY) {
     if (tid < ng) w_s[tid] = A.wgroup[(size_t)h * ng + tid];
-    for (int e = tid; e < DH * r; e += TT) U_s[e] = A.basis[(size_t)h * DH * r + e];
+    for (int e = tid; e < DH * r; e += NT) U_s[e] = A.basis[(size_t)h * DH * r + e];
   }
-  __syncthreads();
-  // ---- P1: A hi/lo (s*k split), A_t
-  float At = 0.0f;
-  {
-    uint8_t* ahi = smem + OFF_AHI;
-    uint8_t* alo = smem + OFF_ALO;
-#pragma unroll 1
-    for (int c = 0; c < 16; ++c) {
-      const uint4 w4 = *reinterpret_cast<const uint4*>(krow + c * 8);
-      const uint32_t wk[4] = {w4.x, w4.y, w4.z, w4.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        const uint32_t wv = wk[e2];
-        uint16_t hb[2], lb[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int j = c * 8 + e2 * 2 + u;
-          const float kj = u ? hi_f(wv) : lo_f(wv);
-          At = __fmaf_rn(s_s[j], __fmul_rn(kj, kj), At);
-          const float sk = KEY ? __fmul_rn(s_s[j], kj) : kj;
-          hb[u] = bf16_rn(sk);
-          lb[u] = bf16_rn(__fsub_rn(sk, bf2f(hb[u])));
-        }
-        hi[e2] = (uint32_t)hb[0] | ((uint32_t)hb[1] << 16);
-        lo[e2] = (uint32_t)lb[0] | ((uint32_t)lb[1] << 16);
-      }
-      *reinterpret_cast<uint4*>(ahi + sw128_off(tid, c, 128)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      if (KEY)
-        *reinterpret_cast<uint4*>(alo + sw128_off(tid, c, 128)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
+  if (tid < 128) {
     // extra K step: A row = [1, 1, 0 ...]
-    uint8_t* aext = smem + OFF_AEXT;
+    uint8_t* aext = smem + L::AEXT;
     const uint32_t one2 = 0x3F803F80u;  // bf16 1.0, 1.0
     *reinterpret_cast<uint4*>(aext + (tid >> 3) * 256 + (tid & 7) * 16) = make_uint4(one2, 0, 0, 0);
     *reinterpret_cast<uint4*>(aext + (tid >> 3) * 256 + 128 + (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
   }
-  tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  float bmax = 0.0f;  // max of B_i over this thread's centroid rows, then over all
 
-  // ---- P2/P3: per chunk of 256 centroids: B operand, MMAs into TMEM columns
-  const int nchunk = (C + NCH - 1) / NCH;
+  // ---- P1-P3: per chunk of 256 centroids the B operand (-2c and B_i), then per
+  // half of the tokens the A operand (s*k as bf16 hi + lo, A_t) and the MMAs into
+  // TMEM columns (chunk + half) * NCH
+  const int nchunk = (C + NCH - 1) / NCH;  // 1 when NT == 256
+  float At = 0.0f;
+  float bmax = 0.0f;  // max of B_i over this thread's centroid rows, then over all
   bool ok = true;
+  int nmma = 0;
   for (int ch = 0; ch < nchunk; ++ch) {
     const int c0 = ch * NCH, nc = min(NCH, C - c0);
-    uint8_t* btw = smem + OFF_B;
-    uint8_t* bext = smem + OFF_BEXT;
-    for (int rr = tid; rr < NCH; rr += TT) {
+    uint8_t* btw = smem + L::B;
+    uint8_t* bext = smem + L::BEXT;
+    for (int rr = tid; rr < NCH; rr += NT) {
       const int i = c0 + rr;
       const uint4* c4 = reinterpret_cast<const uint4*>(cent + (size_t)i * DH);
       float bacc = 0.0f;  // B_i = sum_j s_j c_ij^2, channel order
@@ -287,35 +267,67 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
           make_uint4((uint32_t)bh | ((uint32_t)bl << 16), 0, 0, 0);
       *reinterpret_cast<uint4*>(bext + (rr >> 3) * 256 + 128 + (rr & 7) * 16) = make_uint4(0, 0, 0, 0);
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, NCH, false, false);
-      const uint32_t sa = smem_u32(smem + OFF_AHI), sl = smem_u32(smem + OFF_ALO);
-      const uint32_t sb = smem_u32(smem + OFF_B);
-      const uint32_t d_t = tmem + ch * NCH;
+    for (int hp = 0; hp < NT / 128; ++hp) {
+      if (ch == 0 && half == hp) {
+        uint8_t* ahi = smem + L::AHI;
+        uint8_t* alo = smem + L::ALO;
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(krow + c * 8);
+          const uint32_t wk[4] = {w4.x, w4.y, w4.z, w4.w};
+          uint32_t hi[4], lo[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t ko = (k >> 2) * (128 * 128) + (k & 3) * 32;
-        const uint32_t kb = (k >> 2) * (NCH * 128) + (k & 3) * 32;
-        mma_bf16_ss(d_t, desc_sw128(sa + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, k > 0);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint32_t wv = wk[e2];
+            uint16_t hb[2], lb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int j = c * 8 + e2 * 2 + u;
+              const float kj = u ? hi_f(wv) : lo_f(wv);
+              At = __fmaf_rn(s_s[j], __fmul_rn(kj, kj), At);
+              const float sk = KEY ? __fmul_rn(s_s[j], kj) : kj;
+              hb[u] = bf16_rn(sk);
+              lb[u] = bf16_rn(__fsub_rn(sk, bf2f(hb[u])));
+            }
+            hi[e2] = (uint32_t)hb[0] | ((uint32_t)hb[1] << 16);
+            lo[e2] = (uint32_t)lb[0] | ((uint32_t)lb[1] << 16);
+          }
+          *reinterpret_cast<uint4*>(ahi + sw128_off(row, c, 128)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          if (KEY)
+            *reinterpret_cast<uint4*>(alo + sw128_off(row, c, 128)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
       }
-      if (KEY) {
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16(128, NCH, false, false);
+        const uint32_t sa = smem_u32(smem + L::AHI), sl = smem_u32(smem + L::ALO);
+        const uint32_t sb = smem_u32(smem + L::B);
+        const uint32_t d_t = tmem + (ch + hp) * NCH;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t ko = (k >> 2) * (128 * 128) + (k & 3) * 32;
           const uint32_t kb = (k >> 2) * (NCH * 128) + (k & 3) * 32;
-          mma_bf16_ss(d_t, desc_sw128(sl + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, 1u);
+          mma_bf16_ss(d_t, desc_sw128(sa + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, k > 0);
         }
+        if (KEY) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t ko = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t kb = (k >> 2) * (NCH * 128) + (k & 3) * 32;
+            mma_bf16_ss(d_t, desc_sw128(sl + ko, 16, 1024), desc_sw128(sb + kb, 16, 1024), idesc, 1u);
+          }
+        }
+        mma_bf16_ss(d_t, desc_noswz(smem_u32(smem + L::AEXT), 128, 256),
+                    desc_noswz(smem_u32(smem + L::BEXT), 128, 256), idesc, 1u);
+        mma_commit(bar);
       }
-      mma_bf16_ss(d_t, desc_noswz(smem_u32(smem + OFF_AEXT), 128, 256),
-                  desc_noswz(smem_u32(smem + OFF_BEXT), 128, 256), idesc, 1u);
-      mma_commit(bar);
+      ok = ok && mbar_wait(bar, nmma & 1);
+      ++nmma;
+      tc_fence_after();
+      __syncthreads();
     }
-    ok = ok && mbar_wait(bar, ch & 1);
-    tc_fence_after();
-    __syncthreads();
   }
   if (!__syncthreads_and(ok)) {
     if (tid == 0) atomicExch(&g_append_timeout, 1);
@@ -323,7 +335,8 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
   if (lane == 0) red[warp] = bmax;
   __syncthreads();
-  bmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  bmax = 0.0f;
+  for (int wv = 0; wv < NT / 32; ++wv) bmax = fmaxf(bmax, red[wv]);
 
   // ---- P4: selection from the approximations (thread t, TMEM lane t)
   const int Mc = KEY ? A.M : 1;
@@ -334,7 +347,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   // positive terms is within (n + 3) 2^-24 < 2^-16.9 relative; gamma = 2^-15.
   const float E = 2.4414062e-4f * sqrtf(At * bmax) + 1.2207031e-4f * bmax;  // 2^-12, 2^-13
   const float gam = 3.0517578e-5f;                                           // 2^-15
-  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+  const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + half * NCH;
   // dM >= the M-th smallest d~: the M-th smallest of the minima of groups of 8
   // columns (M groups hold an element no larger than it).  Group minima are
   // four independent chains per 32 columns; only they enter the sorted list.
@@ -472,7 +485,7 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
 
   // ---- P7: INT2 residual and PSAC coefficients, group by group in channel order
   const size_t slot = (size_t)h * A.tcap + (size_t)(A.t0 + tok);
-  uint32_t* codew = reinterpret_cast<uint32_t*>(smem + OFF_CODE) + tid * 8;
+  uint16_t* codew = reinterpret_cast<uint16_t*>(A.codes + slot * (DH / 4));
   uint32_t* pdst = reinterpret_cast<uint32_t*>(A.params) + slot * NG;
   float cq[16];
 #pragma unroll
@@ -533,12 +546,9 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
           }
         }
       }
-      reinterpret_cast<uint16_t*>(codew)[q] = (uint16_t)bits;
+      codew[q] = (uint16_t)bits;  // channels 8q..8q+7
     }
   }
-  uint4* cdst = reinterpret_cast<uint4*>(A.codes + slot * (DH / 4));
-  cdst[0] = *reinterpret_cast<const uint4*>(codew);
-  cdst[1] = *reinterpret_cast<const uint4*>(codew + 4);
   if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
   else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
   if (KEY) {
@@ -564,19 +574,23 @@ __global__ void __launch_bounds__(TT, 1) append_tc_kernel(const ApArgs A) {
   }
 }
 
-template <bool KEY, int G>
+template <bool KEY, int G, int NT>
 cudaError_t run_tc(const ApArgs& a, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY, G>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  const int smem = (int)Lay<NT>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY, G, NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.n + TT - 1) / TT), a.H);
-  append_tc_kernel<KEY, G><<<grid, TT, SMEM_BYTES, s>>>(a);
+  dim3 grid((unsigned)((a.n + NT - 1) / NT), a.H);
+  append_tc_kernel<KEY, G, NT><<<grid, NT, smem, s>>>(a);
   return cudaGetLastError();
 }
 
+// 256 tokens per CTA (two MMA halves sharing one B tile) when the centroid
+// table fits one 256-row tile, else 128.
 template <bool KEY>
 cudaError_t run_tc_g(const ApArgs& a, cudaStream_t s) {
-  return a.G == 32 ? run_tc<KEY, 32>(a, s) : run_tc<KEY, 16>(a, s);
+  if (a.C <= NCH) return a.G == 32 ? run_tc<KEY, 32, 256>(a, s) : run_tc<KEY, 16, 256>(a, s);
+  return a.G == 32 ? run_tc<KEY, 32, 128>(a, s) : run_tc<KEY, 16, 128>(a, s);
 }
 
 }  // namespace
