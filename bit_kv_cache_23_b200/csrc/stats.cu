@@ -7,9 +7,11 @@
 //   - PSAC uses U = the top-r eigenvectors of M (the principal Query
 //     directions; the pages use r = 8, Fig. 4 / Table 9).
 //
-// stats_accumulate: QSTATS[h] += sum_t q_t q_t^T.  Products of bf16 values are
-// exact in fp32; each 64-token chunk is summed in fp32 (tokens in order) and
-// added to the fp64 running sum, so the result does not depend on scheduling.
+// stats_accumulate: QSTATS[h] += sum_t q_t q_t^T in fp64, each entry summed
+// in token order (M_ij <- M_ij + q_ti q_tj, t = 0, 1, ...).  A product of two
+// bf16 values has at most 16 significant bits and is exact in fp64, so the
+// fused multiply-add rounds exactly as the plain add does: the matrix is the
+// sequential fp64 sum, bit for bit, whatever the launch shape.
 //
 // refresh: s_j = M_jj / n, w_g = sum_{j in g} s_j (fp32 fold over the group),
 // U = top-r eigenvectors of A = M / n by block subspace iteration (see
@@ -21,46 +23,89 @@
 namespace qwm {
 namespace {
 
-constexpr int kTile = 32;
-constexpr int kChunk = 64;
+constexpr int kTile = 32;   // output tile side
+constexpr int kChunk = 32;  // tokens staged per pass
 
-// grid (d/32, d/32, H), block 256: each thread owns a 2x2 block of the 32x32
-// output tile.
-__global__ void __launch_bounds__(256) stats_acc(const uint16_t* __restrict__ Q, int64_t n, int H,
-                                                 int d, double* __restrict__ M) {
-  __shared__ float qi[kChunk][kTile + 1];
-  __shared__ float qj[kChunk][kTile + 1];
-  const int h = blockIdx.z;
-  const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  double tot[2][2] = {{0, 0}, {0, 0}};
+// grid (nt (nt + 1) / 2, H) with nt = d / 32: one CTA per tile (bi <= bj) of
+// the upper block triangle, 64 threads, each owning a 4 x 4 block of the
+// 32 x 32 tile.  Both tiles' token columns are staged in shared memory as fp64;
+// M is symmetric (q_i q_j = q_j q_i exactly), so an off-diagonal tile is
+// written to both (bi, bj) and (bj, bi).
+__global__ void __launch_bounds__(64) stats_acc(const uint16_t* __restrict__ Q, int64_t n, int H,
+                                                int d, double* __restrict__ M) {
+  __shared__ __align__(16) double qi[kChunk][kTile];
+  __shared__ __align__(16) double qj[kChunk][kTile];
+  const int h = blockIdx.y;
+  const int nt = d / kTile;
+  int bi = 0, rem = blockIdx.x;
+  while (rem >= nt - bi) {
+    rem -= nt - bi;
+    ++bi;
+  }
+  const int bj = bi + rem;
+  const int i0 = bi * kTile, j0 = bj * kTile;
+  const int tid = threadIdx.x, ty = tid / 8, tx = tid % 8;
+  double* Mh = M + (size_t)h * d * d;
+  double acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = Mh[(size_t)(i0 + ty * 4 + u) * d + j0 + tx * 4 + v];
+
+  // staging: 2 sides x 32 tokens x 4 pieces of 8 channels = 256 pieces, 4 per thread
+  uint4 pre[4];
+  auto fetch = [&](int64_t b) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + 64 * k, side = e >> 7, tt = (e & 127) >> 2, part = e & 3;
+      const int64_t t = b + tt;
+      const int col = (side ? j0 : i0) + part * 8;
+      pre[k] = make_uint4(0, 0, 0, 0);
+      if (t < n) pre[k] = __ldg(reinterpret_cast<const uint4*>(Q + ((size_t)t * H + h) * d + col));
+    }
+  };
+  auto stage = [&]() {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + 64 * k, side = e >> 7, tt = (e & 127) >> 2, part = e & 3;
+      double* dst = (side ? &qj[tt][0] : &qi[tt][0]) + part * 8;
+      const uint32_t w[4] = {pre[k].x, pre[k].y, pre[k].z, pre[k].w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const double lo = (double)__uint_as_float(w[m] << 16);
+        const double hi = (double)__uint_as_float(w[m] & 0xffff0000u);
+        *reinterpret_cast<double2*>(dst + 2 * m) = make_double2(lo, hi);
+      }
+    }
+  };
+  if (n > 0) fetch(0);
   for (int64_t b = 0; b < n; b += kChunk) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * kTile; e += 256) {
-      int tt = e / kTile, c = e % kTile;
-      int64_t t = b + tt;
-      bool ok = t < n;
-      const uint16_t* row = Q + ((size_t)t * H + h) * d;
-      qi[tt][c] = ok ? bf2f(row[i0 + c]) : 0.0f;
-      qj[tt][c] = ok ? bf2f(row[j0 + c]) : 0.0f;
-    }
+    stage();
     __syncthreads();
-    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-    for (int tt = 0; tt < kChunk; ++tt) {
-      float a0 = qi[tt][ty * 2], a1 = qi[tt][ty * 2 + 1];
-      float b0 = qj[tt][tx * 2], b1 = qj[tt][tx * 2 + 1];
-      acc[0][0] = __fmaf_rn(a0, b0, acc[0][0]);
-      acc[0][1] = __fmaf_rn(a0, b1, acc[0][1]);
-      acc[1][0] = __fmaf_rn(a1, b0, acc[1][0]);
-      acc[1][1] = __fmaf_rn(a1, b1, acc[1][1]);
+    if (b + kChunk < n) fetch(b + kChunk);
+    const int cnt = (n - b < kChunk) ? (int)(n - b) : kChunk;
+#pragma unroll 4
+    for (int tt = 0; tt < cnt; ++tt) {
+      const double2 a01 = *reinterpret_cast<const double2*>(&qi[tt][ty * 4]);
+      const double2 a23 = *reinterpret_cast<const double2*>(&qi[tt][ty * 4 + 2]);
+      const double2 b01 = *reinterpret_cast<const double2*>(&qj[tt][tx * 4]);
+      const double2 b23 = *reinterpret_cast<const double2*>(&qj[tt][tx * 4 + 2]);
+      const double a[4] = {a01.x, a01.y, a23.x, a23.y};
+      const double bb[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bb[v], acc[u][v]);
     }
-    for (int u = 0; u < 2; ++u)
-      for (int v = 0; v < 2; ++v) tot[u][v] += (double)acc[u][v];
   }
-  for (int u = 0; u < 2; ++u)
-    for (int v = 0; v < 2; ++v) {
-      size_t o = ((size_t)h * d + i0 + ty * 2 + u) * d + j0 + tx * 2 + v;
-      M[o] += tot[u][v];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int i = i0 + ty * 4 + u, j = j0 + tx * 4 + v;
+      Mh[(size_t)i * d + j] = acc[u][v];
+      if (bi != bj) Mh[(size_t)j * d + i] = acc[u][v];
     }
 }
 
@@ -68,33 +113,53 @@ __global__ void __launch_bounds__(256) stats_acc(const uint16_t* __restrict__ Q,
 // symmetric positive semi-definite A = M / n, fp64, one CTA per head.  The
 // block X (d x p, p = 16 for r <= 8, else 32) starts from the previous
 // refresh's Ritz vectors (warm) or from the columns of A with the largest
-// diagonal (cold).  Each step orthonormalizes X by Cholesky-QR (twice) and
-// multiplies by A; it stops when the trace of Q^T A Q changes by less than
-// 1e-14 relative (or after a cap).  A final Rayleigh-Ritz step diagonalizes
-// H = Q^T A Q (p x p) by one-sided Jacobi; the Ritz vectors Q W, sorted by
-// descending Ritz value, give U (first r columns) and the next warm start.
+// diagonal (cold).  Each step orthonormalizes X by Cholesky-QR and multiplies
+// by A, a fixed number of steps (3 warm, 30 cold).  A final Rayleigh-Ritz step
+// (Cholesky-QR twice, H = Q^T A Q) diagonalizes the p x p matrix H by one-sided
+// Jacobi; the Ritz vectors Q W, sorted by descending Ritz value, give U (first
+// r columns) and the next warm start.
 struct RefreshSmem {
   double* A;   // [d][d+1] row-major, padded
   double* X;   // [p][d+1] column-major (column k at X + k*(d+1))
   double* Y;   // [p][d+1]
   double* G;   // [p][p]  Gram / projected matrix (column-major for Jacobi)
-  double* L;   // [p][p]  Cholesky factor
+  double* L;   // [p][p]  Cholesky factor (column-major: L[k*p + i] = L_ik)
   double* th;  // [p]     Ritz values
   int* ord;    // [p]
   double* red; // [32]    block reduction scratch
 };
 
-// Y = A X  (each warp takes columns, lanes take rows)
-__device__ void gemm_AX(const RefreshSmem& S, const double* X, double* Y, int d, int p) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32, nw = blockDim.x / 32;
-  for (int k = warp; k < p; k += nw) {
-    const double* xk = X + k * (d + 1);
-    for (int i = lane; i < d; i += 32) {
-      const double* ai = S.A + i * (d + 1);
-      double acc = 0.0;
-      for (int j = 0; j < d; ++j) acc = fma(ai[j], xk[j], acc);
-      Y[k * (d + 1) + i] = acc;
+// Y = A X.  32 (P / 4) threads: thread (cg, lane) owns rows lane + 32 m and
+// columns 4 cg .. 4 cg + 3 (4 D / 32 independent accumulators); rows of A are
+// read without bank conflicts (padded stride), entries of X are broadcast.
+template <int D, int P>
+__device__ void gemm_AX(const double* A, const double* X, double* Y) {
+  constexpr int RM = D / 32;
+  const int t = threadIdx.x;
+  if (t < 32 * (P / 4)) {
+    const int lane = t & 31, cg = t >> 5;
+    const double* x0 = X + 4 * cg * (D + 1);
+    double acc[RM][4];
+#pragma unroll
+    for (int m = 0; m < RM; ++m)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[m][c] = 0.0;
+#pragma unroll 4
+    for (int j = 0; j < D; ++j) {
+      double a[RM], x[4];
+#pragma unroll
+      for (int m = 0; m < RM; ++m) a[m] = A[(lane + 32 * m) * (D + 1) + j];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[c] = x0[c * (D + 1) + j];
+#pragma unroll
+      for (int m = 0; m < RM; ++m)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[m][c] = fma(a[m], x[c], acc[m][c]);
     }
+#pragma unroll
+    for (int m = 0; m < RM; ++m)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) Y[(4 * cg + c) * (D + 1) + lane + 32 * m] = acc[m][c];
   }
   __syncthreads();
 }
@@ -114,84 +179,83 @@ __device__ void gram(const double* X, const double* Y, double* G, int d, int p) 
   __syncthreads();
 }
 
-// One Cholesky-QR pass: X <- X R^-1 with R^T R = X^T X (R = L^T).  One warp
-// factors the p x p Gram matrix and inverts L; then every thread applies
-// L^-1 to rows of X.  Columns whose pivot vanishes (dependent columns) become
-// zero.
-__device__ void cholqr(const RefreshSmem& S, double* X, int d, int p) {
-  gram(X, X, S.G, d, p);
+// One Cholesky-QR pass: X <- X R^-1 with R^T R = X^T X (R = L^T).  Warp 0
+// factors the Gram matrix with lane i holding row i in registers (right-looking,
+// the multipliers passed by shuffles); then each thread takes one row x of X and
+// solves L q = x by forward substitution.  A column whose pivot vanishes
+// (dependent columns) becomes zero.
+template <int D, int P>
+__device__ void cholqr(double* X, double* G, double* L) {
+  gram(X, X, G, D, P);
   if (threadIdx.x < 32) {
-    const int i = threadIdx.x;  // row owned by this lane
+    const int i = threadIdx.x;
+    double g[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) g[j] = (i < P) ? G[j * P + i] : 0.0;
     double tr = 0.0;
-    for (int k = 0; k < p; ++k) tr += S.G[k * p + k];
-    for (int k = 0; k < p; ++k) {
-      const double piv = S.G[k * p + k];
+#pragma unroll
+    for (int k = 0; k < P; ++k) tr += G[k * P + k];
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      const double piv = __shfl_sync(0xffffffffu, g[k], k);
       const bool ok = piv > 1e-26 * tr && piv > 0.0;
       const double dkk = ok ? sqrt(piv) : 0.0;
-      if (i >= k && i < p) S.L[k * p + i] = ok ? (i == k ? dkk : S.G[k * p + i] / dkk) : 0.0;
-      __syncwarp();
-      if (i > k && i < p) {
-        const double lik = S.L[k * p + i];
-        for (int j = k + 1; j <= i; ++j) S.G[j * p + i] -= lik * S.L[k * p + j];
-      }
-      __syncwarp();
-    }
-    // Linv (lower triangular) into G: lane c computes column c by forward
-    // substitution down the column, using only L and its own earlier entries
-    __syncwarp();
-    if (i < p) {
-      const int c = i;
-      for (int r2 = 0; r2 < c; ++r2) S.G[c * p + r2] = 0.0;
-      for (int r2 = c; r2 < p; ++r2) {
-        double v = (r2 == c) ? 1.0 : 0.0;
-        for (int m = c; m < r2; ++m) v -= S.L[m * p + r2] * S.G[c * p + m];
-        const double l = S.L[r2 * p + r2];
-        S.G[c * p + r2] = (l != 0.0) ? v / l : 0.0;
+      double lik = 0.0;
+      if (i == k) lik = dkk;
+      else if (i > k && i < P && ok) lik = g[k] / dkk;
+      if (i < P) L[k * P + i] = lik;
+#pragma unroll
+      for (int j = k + 1; j < P; ++j) {
+        const double ljk = __shfl_sync(0xffffffffu, lik, j);
+        g[j] = g[j] - lik * ljk;  // rows below k; the upper triangle is never read
       }
     }
   }
   __syncthreads();
-  // Q = X R^-1 = X Linv^T: Q[:, k] = sum_{m <= k} X[:, m] Linv[k][m]
-  double* Y = S.Y;
-  for (int e = threadIdx.x; e < p * d; e += blockDim.x) {
-    const int k = e / d, i = e % d;
-    double acc = 0.0;
-    for (int m = 0; m <= k; ++m) acc = fma(X[m * (d + 1) + i], S.G[m * p + k], acc);
-    Y[k * (d + 1) + i] = acc;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < p * d; e += blockDim.x) {
-    const int k = e / d, i = e % d;
-    X[k * (d + 1) + i] = Y[k * (d + 1) + i];
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    double q[P];
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      double v = X[k * (D + 1) + i];
+#pragma unroll
+      for (int m = 0; m < k; ++m) v = v - L[m * P + k] * q[m];
+      const double lkk = L[k * P + k];
+      q[k] = (lkk != 0.0) ? v / lkk : 0.0;
+    }
+#pragma unroll
+    for (int k = 0; k < P; ++k) X[k * (D + 1) + i] = q[k];
   }
   __syncthreads();
 }
 
-// One-sided Jacobi on the p x p column-major matrix G (positive semi-definite):
-// rotate column pairs until orthogonal; 8 threads per pair.  Also applies the
+// One-sided Jacobi on the p x p column-major matrix G (positive semi-definite),
+// in warp 0: rotate column pairs until orthogonal, the p / 2 disjoint pairs of
+// a round-robin round at once, 64 / p lanes per pair.  Also applies the
 // rotations to W (p x p, column-major, starts as the identity).
-__device__ void small_jacobi(double* G, double* W, int p, double* red) {
-  const int tid = threadIdx.x;
-  const int grp = tid / 8, sub = tid % 8;
-  const int npairs = p / 2;
-  for (int e = tid; e < p * p; e += blockDim.x) W[e] = ((e / p) == (e % p)) ? 1.0 : 0.0;
+template <int P>
+__device__ void small_jacobi(double* G, double* W) {
+  constexpr int LPP = 64 / P;  // lanes per pair
+  for (int e = threadIdx.x; e < P * P; e += blockDim.x) W[e] = ((e / P) == (e % P)) ? 1.0 : 0.0;
   __syncthreads();
-  for (int sweep = 0; sweep < 30; ++sweep) {
-    float worst = 0.0f;
-    for (int rnd = 0; rnd < p - 1; ++rnd) {
-      if (grp < npairs) {
-        const int a = (grp == 0) ? 0 : 1 + (grp - 1 + rnd) % (p - 1);
-        const int bb = 1 + (p - 1 - grp - 1 + rnd) % (p - 1);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x, grp = lane / LPP, sub = lane % LPP;
+    for (int sweep = 0; sweep < 30; ++sweep) {
+      float worst = 0.0f;
+      for (int rnd = 0; rnd < P - 1; ++rnd) {
+        const int a = (grp == 0) ? 0 : 1 + (grp - 1 + rnd) % (P - 1);
+        const int bb = 1 + (P - 1 - grp - 1 + rnd) % (P - 1);
         const int pp = min(a, bb), qq = max(a, bb);
-        double* gp = G + pp * p;
-        double* gq = G + qq * p;
+        double* gp = G + pp * P;
+        double* gq = G + qq * P;
         double al = 0.0, be = 0.0, ga = 0.0;
-        for (int i = sub; i < p; i += 8) {
+#pragma unroll
+        for (int i = sub; i < P; i += LPP) {
           al += gp[i] * gp[i];
           be += gq[i] * gq[i];
           ga += gp[i] * gq[i];
         }
-        for (int o = 4; o >= 1; o >>= 1) {
+#pragma unroll
+        for (int o = LPP / 2; o >= 1; o >>= 1) {
           al += __shfl_xor_sync(0xffffffffu, al, o);
           be += __shfl_xor_sync(0xffffffffu, be, o);
           ga += __shfl_xor_sync(0xffffffffu, ga, o);
@@ -202,9 +266,10 @@ __device__ void small_jacobi(double* G, double* W, int p, double* red) {
           const double zeta = (be - al) / (2.0 * ga);
           const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
           const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
-          double* wp = W + pp * p;
-          double* wq = W + qq * p;
-          for (int i = sub; i < p; i += 8) {
+          double* wp = W + pp * P;
+          double* wq = W + qq * P;
+#pragma unroll
+          for (int i = sub; i < P; i += LPP) {
             const double u = gp[i], v = gq[i];
             gp[i] = c * u - s * v;
             gq[i] = s * u + c * v;
@@ -213,28 +278,26 @@ __device__ void small_jacobi(double* G, double* W, int p, double* red) {
             wq[i] = s * wu + c * wv;
           }
         }
+        __syncwarp();
       }
-      __syncthreads();
+      for (int o = 16; o >= 1; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+      if (worst <= 1e-13f) break;
     }
-    for (int o = 16; o >= 1; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
-    __syncthreads();
-    if ((tid & 31) == 0) red[tid / 32] = worst;
-    __syncthreads();
-    float m = 0.0f;
-    for (int w = 0; w < (int)(blockDim.x / 32); ++w) m = fmaxf(m, (float)red[w]);
-    __syncthreads();
-    if (m <= 1e-13f) break;
   }
+  __syncthreads();
 }
 
-// One CTA per head, 512 threads.
-__global__ void __launch_bounds__(512) refresh_kernel(const double* __restrict__ Mall, int64_t n,
-                                                      int d, int G, int r, int p,
+// One CTA per head (512 threads, 256 for P = 32 so that the 32-wide register
+// rows fit); head_dim D and block width P fixed at compile time.
+template <int D, int P>
+__global__ void __launch_bounds__(P == 32 ? 256 : 512) refresh_kernel(const double* __restrict__ Mall, int64_t n,
+                                                      int G, int r,
                                                       float* __restrict__ sens,
                                                       float* __restrict__ wgroup,
                                                       float* __restrict__ basis_slot,
                                                       double* __restrict__ eigvec,
                                                       double* __restrict__ flags) {
+  constexpr int d = D, p = P;
   extern __shared__ double sm[];
   const int h = blockIdx.x;
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -299,26 +362,25 @@ __global__ void __launch_bounds__(512) refresh_kernel(const double* __restrict__
   // block may be nearly degenerate, so the block as a whole is not a stopping
   // test).  Warm starts track a basis that moves little between refreshes.
   const int iters = warm ? 3 : 30;
+  double* Xc = S.X;  // the current block; the product goes to the other buffer
+  double* Yc = S.Y;
   for (int it = 0; it < iters; ++it) {
-    cholqr(S, S.X, d, p);
-    gemm_AX(S, S.X, S.Y, d, p);
-    for (int e = tid; e < p * d; e += nt) {
-      const int k = e / d, i = e % d;
-      S.X[k * (d + 1) + i] = S.Y[k * (d + 1) + i];
-    }
-    __syncthreads();
+    cholqr<D, P>(Xc, S.G, S.L);
+    gemm_AX<D, P>(S.A, Xc, Yc);
+    double* t = Xc;
+    Xc = Yc;
+    Yc = t;
   }
   // ---- Rayleigh-Ritz on the final block
-  cholqr(S, S.X, d, p);
-  cholqr(S, S.X, d, p);
-  gemm_AX(S, S.X, S.Y, d, p);
-  gram(S.X, S.Y, S.G, d, p);              // H = Q^T A Q (column-major, symmetric)
-  double* W = S.Y;                         // Y is free again: W [p][p] in its space
-  double* Hc = S.Y + p * p;                // copy of H to rotate
+  cholqr<D, P>(Xc, S.G, S.L);
+  cholqr<D, P>(Xc, S.G, S.L);
+  gemm_AX<D, P>(S.A, Xc, Yc);
+  gram(Xc, Yc, S.G, d, p);                 // H = Q^T A Q (column-major, symmetric)
+  double* W = Yc;                          // Y is free again: W [p][p] in its space
+  double* Hc = Yc + p * p;                 // copy of H to rotate
   for (int e = tid; e < p * p; e += nt) Hc[e] = S.G[e];
   __syncthreads();
-  small_jacobi(Hc, W, p, S.red);
-  __syncthreads();
+  small_jacobi<P>(Hc, W);
   if (tid < p) {
     double acc = 0.0;
     for (int i = 0; i < p; ++i) acc += Hc[tid * p + i] * Hc[tid * p + i];
@@ -339,7 +401,7 @@ __global__ void __launch_bounds__(512) refresh_kernel(const double* __restrict__
     const int c = e / d, i = e % d;
     const int k = S.ord[c];
     double acc = 0.0;
-    for (int m = 0; m < p; ++m) acc = fma(S.X[m * (d + 1) + i], W[k * p + m], acc);
+    for (int m = 0; m < p; ++m) acc = fma(Xc[m * (d + 1) + i], W[k * p + m], acc);
     Vout[(size_t)c * d + i] = acc;
   }
   __syncthreads();
@@ -391,8 +453,9 @@ cudaError_t launch_init_state(const Dims& D, const CacheView& v, cudaStream_t s)
 
 cudaError_t launch_stats_accumulate(const Dims& D, const uint16_t* Q, int64_t n, double* qstats,
                                     cudaStream_t s) {
-  dim3 grid(D.d / kTile, D.d / kTile, D.H);
-  stats_acc<<<grid, 256, 0, s>>>(Q, n, D.H, D.d, qstats);
+  const int nt = D.d / kTile;
+  dim3 grid(nt * (nt + 1) / 2, D.H);
+  stats_acc<<<grid, 64, 0, s>>>(Q, n, D.H, D.d, qstats);
   return cudaGetLastError();
 }
 
@@ -405,11 +468,15 @@ cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, i
   const int p = refresh_block(D.d, D.r);
   size_t smem = ((size_t)D.d * (D.d + 1) + 2 * (size_t)p * (D.d + 1) + 2 * p * p + p + 32) * 8 +
                 (size_t)p * 4 + 64;
-  cudaError_t e =
-      cudaFuncSetAttribute(refresh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = refresh_kernel<128, 16>;
+  if (D.d == 128 && p == 32) kern = refresh_kernel<128, 32>;
+  else if (D.d == 64 && p == 16) kern = refresh_kernel<64, 16>;
+  else if (D.d == 64 && p == 32) kern = refresh_kernel<64, 32>;
+  else if (!(D.d == 128 && p == 16)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  refresh_kernel<<<D.H, 512, smem, s>>>(v.qstats, n_total, D.d, D.G, D.r, p, v.sens, v.wgroup,
-                                        slot, v.eigvec, flags);
+  kern<<<D.H, p == 32 ? 256 : 512, smem, s>>>(v.qstats, n_total, D.G, D.r, v.sens, v.wgroup, slot, v.eigvec,
+                              flags);
   return cudaGetLastError();
 }
 

@@ -153,10 +153,14 @@ QWM_API qwm_status qwm_build_centroids(qwm_cache* c, const void* K, const void* 
 
 /* Historical Query statistics [review, Summary: "historical Query
  * second-moment statistics"; Eq. 7 M = E[q q^T]]: QSTATS[h] += sum_t q_t q_t^T,
- * n_queries += n_q.  With refresh_basis != 0 it then refreshes what QSAC and
- * PSAC read: s_j = M_jj / n, w_g = sum_{j in g} s_j, U = top-r eigenvectors of
- * M / n (Jacobi, warm-started from the last refresh), stored as a new basis
- * version used by later appends.  Q: [n_q][H][d] bf16 device, n_q >= 0.
+ * n_queries += n_q.  Each fp64 entry is summed in token order, so QSTATS is
+ * the sequential fp64 sum bit for bit (the products of bf16 values are exact).
+ * With refresh_basis != 0 it then refreshes what QSAC and PSAC read:
+ * s_j = fp32(M_jj / n), w_g = the fp32 sum of s_j over group g in channel
+ * order, U = top-r eigenvectors of M / n (fp64 block subspace iteration with
+ * a Rayleigh-Ritz step, warm-started from the last refresh; columns signed so
+ * that the largest-magnitude entry is positive), stored as a new basis version
+ * used by later appends.  Q: [n_q][H][d] bf16 device, n_q >= 0.
  * Errors: INVALID_ARG, ALIGNMENT, CAPACITY (no free basis slot), CUDA. */
 QWM_API qwm_status qwm_update_query_stats(qwm_cache* c, const void* Q, int64_t n_q,
                                   int32_t refresh_basis, void* stream);

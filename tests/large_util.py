@@ -8,10 +8,12 @@ seeded generator, so no large array crosses a process boundary.
 
 Token encodings depend only on the frame's inputs and the state in force at
 append time (centroid tables, sensitivities s, group weights w, basis U).  The
-centroids are compared bit for bit first; s, w and U are compared with the
-oracle's own fp64 refresh within tolerance and then the GPU's values are
-installed, as in the small-config parity tests, so that the codes can be
-compared exactly.
+oracle runs on its own state throughout: its own k-means tables, its own fp64
+statistics of the sampled heads (accumulated here frame by frame) and its own
+refresh.  At every refresh the GPU's statistics matrix, s and w must equal the
+oracle's bit for bit, its basis is compared within tolerance, and the oracle's U
+is installed as the GPU's basis of the sampled heads, so that both sides encode
+with the same state and the codes can be compared exactly.
 """
 from __future__ import annotations
 
@@ -70,30 +72,21 @@ def encode_frames(args):
     return {k: getattr(oc, k)[0, :n].copy() for k in fields}
 
 
-def stats_head(args):
-    """Oracle fp64 Query second-moment matrix of head h over frames [0, f1)."""
-    name, seed, h, f1 = args
-    c = syn.get_config(name)
-    src = syn.FrameSource(c, seed)
-    M = np.zeros((c.head_dim, c.head_dim))
-    for f in range(f1):
-        oracle.stats_accumulate(src.queries(f, heads=[h])[:, 0, :], M)
-    return M
-
-
 # ----------------------------------------------------------------- driver
-def run_full(name, heads, attn_frames, attn_rows, seed=None, check_refresh=3):
+def run_full(name, heads, attn_frames, attn_rows, seed=None):
     """Run configuration `name` at full size; returns measured discrepancies."""
     import torch
 
     import bit_kv_cache_23_b200 as q
-    from parity_util import attention_error, make_gpu_cache, to_dev, u16
+    from parity_util import (attention_error, make_gpu_cache, new_state_report,
+                             refresh_from_oracle, to_dev, u16)
 
     c = syn.get_config(name)
     seed = c.seed if seed is None else seed
     F = c.frames
-    out = dict(packed_mismatch={}, cent_equal=True, attn=[], stats_rel=0.0, orth_err=0.0,
-               proj_err=0.0, frames=F)
+    out = dict(packed_mismatch={}, cent_equal=True, attn=[], frames=F, refreshes=0)
+    out.update(new_state_report())
+    Mref = {h: np.zeros((c.head_dim, c.head_dim)) for h in heads}
     rng = np.random.default_rng(2024)
     g = make_gpu_cache(c)
     with pool() as P:
@@ -111,13 +104,11 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None, check_refresh=3):
                 g.build_centroids(Kd, Vd, iters=c.kmeans_iters)
             refresh = (f % c.refresh_every) == 0
             g.update_query_stats(Qd, refresh_basis=refresh)
+            for h in heads:
+                oracle.stats_accumulate(Q[:, h, :], Mref[h])
             nq += Q.shape[0]
             if refresh:
-                torch.cuda.synchronize()
-                s = g.view("sens").cpu().numpy()
-                w = g.view("wgroup").cpu().numpy()
-                U = g.view("basis")[g.version].cpu().numpy()
-                ver_state = {h: (s[h].copy(), w[h].copy(), U[h].copy()) for h in heads}
+                ver_state = refresh_from_oracle(g, Mref, nq, heads, c.rank, c.group, out)
                 refreshes.append((f, nq))
             for h in heads:
                 states[h].append(ver_state[h])
@@ -132,9 +123,11 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None, check_refresh=3):
                 attn_out[f] = (rows, Q[rows][:, heads, :].copy(), Og[rows][:, heads, :].copy(),
                                g.len)
         torch.cuda.synchronize()
+        out["refreshes"] = len(refreshes)
         CKg = g.view("cent_k").cpu().numpy().view(np.uint16)
         CVg = g.view("cent_v").cpu().numpy().view(np.uint16)
-        for h, (ck, cv) in zip(heads, km.get()):
+        cents = dict(zip(heads, km.get()))     # the oracle's own tables
+        for h, (ck, cv) in cents.items():
             out["cent_equal"] &= bool(np.array_equal(ck, CKg[h]) and np.array_equal(cv, CVg[h]))
 
         # every token of the sampled heads, re-encoded by the oracle
@@ -144,7 +137,7 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None, check_refresh=3):
         for h in heads:
             for f0 in range(0, F, chunk):
                 f1 = min(F, f0 + chunk)
-                tasks.append((name, seed, h, f0, f1, CKg[h].copy(), CVg[h].copy(),
+                tasks.append((name, seed, h, f0, f1, cents[h][0], cents[h][1],
                               states[h][f0:f1]))
                 keys.append((h, f0, f1))
         enc = P.map(encode_frames, tasks, chunksize=1)
@@ -167,31 +160,12 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None, check_refresh=3):
                 if ne:
                     out["packed_mismatch"][(h, k)] = ne
 
-        # statistics and basis at a few refreshes, against the oracle's fp64 refresh
-        picks = [refreshes[i] for i in sorted(set(
-            np.linspace(0, len(refreshes) - 1, min(check_refresh, len(refreshes))).astype(int)))]
-        Ms = P.map(stats_head, [(name, seed, h, f + 1) for (f, _) in picks for h in heads])
-        i = 0
-        for (f, nqf) in picks:
-            for h in heads:
-                so, wo, Uo, _ = oracle.refresh(Ms[i], nqf, c.rank, c.group)
-                s, w, U = states[h][f]
-                out["stats_rel"] = max(out["stats_rel"],
-                                       float(np.abs(s - so).max() / np.abs(so).max()))
-                if c.rank:
-                    Ug = U.astype(np.float64)[:, :c.rank]
-                    out["orth_err"] = max(out["orth_err"],
-                                          float(np.abs(Ug.T @ Ug - np.eye(c.rank)).max()))
-                    P1 = Ug @ Ug.T
-                    P2 = Uo.astype(np.float64) @ Uo.T.astype(np.float64)
-                    out["proj_err"] = max(out["proj_err"], float(np.linalg.norm(P1 - P2, 2)))
-                i += 1
 
     # attention on sampled rows, over the oracle's own reconstruction
     for hi, h in enumerate(heads):
         oc = oracle.OracleCache(1, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank,
                                 F * N, max_versions=len(refreshes) + 2)
-        oc.set_state(CK=CKg[h][None], CV=CVg[h][None])
+        oc.set_state(CK=cents[h][0][None], CV=cents[h][1][None])
         for k, v in ofields[h].items():
             getattr(oc, k)[0, :F * N] = v
         # versions: 0 = the zero basis before any refresh, then one per refresh

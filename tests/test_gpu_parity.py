@@ -1,9 +1,10 @@
 """GPU path (C ABI through the binding) against the CPU oracle.
 
-Bit-exact: centroid tables, centroid indices, INT2 codes, fp16 group
-parameters, INT8 coefficients and scales.  Tolerance: attention output within
-max-abs 2e-2 and mean-abs 2e-3 of the oracle's fp64 attention over the same
-reconstructed cache; statistics and basis against the oracle's fp64 versions.
+Bit-exact: centroid tables, the Query statistics matrix, s and w, centroid
+indices, INT2 codes, fp16 group parameters, INT8 coefficients and scales.
+Tolerance: the basis against the oracle's Jacobi basis (which both sides then
+encode with), and attention output within max-abs 2e-2 and mean-abs 2e-3 of the
+oracle's fp64 attention over its own reconstructed cache.
 """
 import numpy as np
 import pytest
@@ -11,7 +12,8 @@ import torch
 
 import oracle
 import qwm_synth as syn
-from parity_util import ATOL_MAX, ATOL_MEAN, run_layer, to_dev, u16
+from parity_util import (ATOL_MAX, ATOL_MEAN, compare_packed, new_state_report,
+                         refresh_from_oracle, run_layer, stack_state, to_dev, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -19,7 +21,8 @@ pytestmark = pytest.mark.gpu
 def _assert_common(out, proj_tol=1e-4):
     assert out["cent_k_equal"] and out["cent_v_equal"], "k-means centroids differ"
     assert out["packed_mismatch"] == {}, out["packed_mismatch"]
-    assert out["stats_rel"] < 1e-5, out["stats_rel"]
+    assert out["stats_mismatch"] == 0, out["stats_mismatch"]
+    assert out["sw_mismatch"] == 0, out["sw_mismatch"]
     assert out["orth_err"] < 1e-5, out["orth_err"]
     assert out["proj_err"] < proj_tol, out["proj_err"]
     for f, mx, mean in out["attn"]:
@@ -33,9 +36,15 @@ def test_tiny_full():
     g, oc = out["gpu"], out["oracle"]
     Kp, Vp = g.reconstruct()
     Ko, Vo = oc.reconstruct(0)
-    kg = syn.bf16_bits_to_f32(u16(Kp[0]))
-    ko = syn.bf16_bits_to_f32(Ko)
-    assert np.all(np.abs(kg - ko) <= np.spacing(np.abs(ko)) * 1.01 + 1e-30)
+    kg = syn.bf16_bits_to_f32(u16(Kp[0])).astype(np.float64)
+    ko = syn.bf16_bits_to_f32(Ko).astype(np.float64)
+    # one bf16 ulp (8 significant bits) of the larger magnitude: the two sums may
+    # straddle a bf16 rounding boundary; that must stay rare
+    big = np.maximum(np.abs(kg), np.abs(ko))
+    ulp = np.where(big > 0, 2.0 ** (np.floor(np.log2(np.where(big > 0, big, 1.0))) - 7), 0.0)
+    diff = np.abs(kg - ko)
+    assert np.all(diff <= ulp), float((diff / np.maximum(ulp, 1e-300)).max())
+    assert np.count_nonzero(diff) <= 1e-3 * diff.size, np.count_nonzero(diff)
     assert np.array_equal(u16(Vp[0]), Vo)
 
 
@@ -81,25 +90,28 @@ def test_degenerate_inputs():
     CK = g.view("cent_k").cpu().numpy().view(np.uint16).copy()
     CV = g.view("cent_v").cpu().numpy().view(np.uint16).copy()
     ck, _ = oracle.kmeans(K[:, 0, :], C, 3)
-    assert np.array_equal(ck, CK[0])
-    oc.set_state(CK=CK, CV=CV)
+    cv, _ = oracle.kmeans(V[:, 0, :], C, 3)
+    assert np.array_equal(ck, CK[0]) and np.array_equal(cv, CV[0])
+    oc.set_state(CK=ck[None], CV=cv[None])
     # appends before any query statistics: s = 1, U = 0
     for n in (1, 7, 32):
         t0 = g.len
         g.append_kv(to_dev(K[:n]), to_dev(V[:n]))
         oc.append_kv(K[:n], V[:n])
-        from parity_util import compare_packed
         assert compare_packed(g, oc, t0, g.len) == {}
     Q = syn.f32_to_bf16_bits(rng.standard_normal((3, H, d)).astype(np.float32))
     g.update_query_stats(to_dev(Q), refresh_basis=True)   # fewer queries than rank
-    s, w, U = (g.view("sens").cpu().numpy(), g.view("wgroup").cpu().numpy(),
-               g.view("basis")[g.version].cpu().numpy())
-    assert np.all(np.isfinite(U))
+    Mref = {0: np.zeros((d, d))}
+    oracle.stats_accumulate(Q[:, 0, :], Mref[0])
+    rep = new_state_report()
+    # rank-deficient statistics: the basis is not unique, so only the oracle's is used
+    st = refresh_from_oracle(g, Mref, 3, [0], 4, 16, rep, check_basis=False)
+    assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
+    s, w, U = stack_state(st, H)
     oc.set_state(s=s, w=w, U=U)
     t0 = g.len
     g.append_kv(to_dev(K), to_dev(V))
     oc.append_kv(K, V)
-    from parity_util import compare_packed
     assert compare_packed(g, oc, t0, g.len) == {}
     O = g.attention(to_dev(Q))
     torch.cuda.synchronize()
@@ -113,8 +125,6 @@ def test_head128_shapes(G, C, M, r):
     """head_dim 128 with groups of 16, C not a power of two, C = 512 (two MMA
     chunks), M up to 8 and ranks other than 8: every packed field bit for bit,
     attention within tolerance; keys with outlier channels and frame drift."""
-    from parity_util import compare_packed
-
     H, d, n = 3, 128, 700
     q = pytest.importorskip("bit_kv_cache_23_b200")
     g = q.QuantKVCache(H, d, C, G, M, r, 3 * n, max_versions=8)
@@ -131,18 +141,28 @@ def test_head128_shapes(G, C, M, r):
     torch.cuda.synchronize()
     CK = g.view("cent_k").cpu().numpy().view(np.uint16).copy()
     CV = g.view("cent_v").cpu().numpy().view(np.uint16).copy()
-    oc.set_state(CK=CK, CV=CV)
+    ck = np.stack([oracle.kmeans(K[0][:, h, :], C, 4)[0] for h in range(H)])
+    cv = np.stack([oracle.kmeans(V[0][:, h, :], C, 4)[0] for h in range(H)])
+    assert np.array_equal(ck, CK) and np.array_equal(cv, CV)
+    oc.set_state(CK=ck, CV=cv)
+    Mref = {h: np.zeros((d, d)) for h in range(H)}
+    rep = new_state_report()
     for f in range(3):
         Q = syn.f32_to_bf16_bits((3.3 * rng.standard_normal((200, H, 8)) @ basis.T
                                   + 0.5 * rng.standard_normal((200, H, d))).astype(np.float32))
         g.update_query_stats(to_dev(Q), refresh_basis=True)
-        torch.cuda.synchronize()
-        oc.set_state(s=g.view("sens").cpu().numpy(), w=g.view("wgroup").cpu().numpy(),
-                     U=g.view("basis")[g.version].cpu().numpy())
+        for h in range(H):
+            oracle.stats_accumulate(Q[:, h, :], Mref[h])
+        st = refresh_from_oracle(g, Mref, 200 * (f + 1), range(H), r, G, rep,
+                                 check_basis=(r <= 8))
+        s, w, U = stack_state(st, H)
+        oc.set_state(s=s, w=w, U=U)
         t0 = g.len
         g.append_kv(to_dev(K[f]), to_dev(V[f]))
         oc.append_kv(K[f], V[f])
         assert compare_packed(g, oc, t0, g.len) == {}, f
+    assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
+    assert rep["orth_err"] < 1e-5 and rep["proj_err"] < 1e-3, rep
     O = g.attention(to_dev(Q))
     torch.cuda.synchronize()
     assert q.qwm_device_status() == 0
