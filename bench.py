@@ -230,6 +230,94 @@ class Workload:
         self.nstep += 1
 
 
+# ----------------------------------------------------------------------------- ablations
+# (name, M, r, Query statistics taken, tensors quantized); None = the layer's own.
+ABLATIONS = [
+    ("quantwm", None, None, True, "kv"),     # QSAC + PSAC, both tensors
+    ("qvg", 1, 0, False, "kv"),              # plain nearest centroid: M = 1, s = 1, r = 0
+    ("qsac_only", None, 0, True, "kv"),      # no compensation (rank 0)
+    ("rank2", None, 2, True, "kv"),
+    ("rank4", None, 4, True, "kv"),
+    ("rank16", None, 16, True, "kv"),
+    ("k_only", None, None, True, "k"),       # Keys quantized, Values exact
+    ("v_only", None, None, True, "v"),       # Values quantized, Keys exact
+]
+
+
+def run_ablation(cfg: syn.LayerConfig, device, frames: int) -> list:
+    """Quality of each quantization setting on a synthetic layer: top-1 key
+    selection shift (fraction of query rows and heads whose highest-scoring key
+    changes), K / V reconstruction error relative to the mean square of the exact
+    tensors, error of the attention output against exact bf16 attention (absolute,
+    and relative to the mean square of the exact output, which is small here: the
+    synthetic keys carry no structure, so attention is spread over many keys),
+    and the compression ratio.
+    Every step runs in the library's kernels (append, reconstruction, top-1, the
+    fused attention, and attention over exact or reconstructed bf16 segments on an
+    empty cache); torch only reduces the differences to means."""
+    import bit_kv_cache_23_b200 as q
+
+    c = dataclasses.replace(cfg, frames=frames)
+    src = syn.FrameSource(c)
+    data = [src.frame(f) for f in range(c.frames)]
+    Kx = torch.cat([dev_bf16(K, device) for _, K, _ in data], 0)
+    Vx = torch.cat([dev_bf16(V, device) for _, _, V in data], 0)
+    Qd = dev_bf16(data[-1][0], device)
+    T = Kx.shape[0]
+    empty = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank, 16,
+                           device=device)
+    Oexact = empty.attention_ext(Qd, Kx, Vx).float()
+    e_o = Oexact.pow(2).mean().item()
+    e_k, e_v = Kx.float().pow(2).mean().item(), Vx.float().pow(2).mean().item()
+    out = []
+    for name, M, r, stats, which in ABLATIONS:
+        M = c.n_cand if M is None else M
+        r = c.rank if r is None else r
+        g = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, M, r, T,
+                           max_versions=c.frames + 2, device=device)
+        for f, (Q, K, V) in enumerate(data):
+            Kd, Vd = dev_bf16(K, device), dev_bf16(V, device)
+            if f == 0:
+                g.build_centroids(Kd, Vd, iters=c.kmeans_iters)
+            if stats:
+                g.update_query_stats(dev_bf16(Q, device),
+                                     refresh_basis=(f % c.refresh_every) == 0)
+            g.append_kv(Kd, Vd)
+        Kp, Vp = g.reconstruct()                       # [H][T][d]
+        Kp = Kp.permute(1, 0, 2).contiguous()
+        Vp = Vp.permute(1, 0, 2).contiguous()
+        k_err = (Kp.float() - Kx.float()).pow(2).mean().item() / e_k
+        v_err = (Vp.float() - Vx.float()).pow(2).mean().item() / e_v
+        if which == "kv":
+            O = g.attention(Qd)
+        elif which == "k":
+            O = empty.attention_ext(Qd, Kp, Vx)
+        else:
+            O = empty.attention_ext(Qd, Kx, Vp)
+        o_mse = (O.float() - Oexact).pow(2).mean().item()
+        shift = 0.0
+        if which != "v":
+            ie, iq = g.top1_shift(Qd, Kx)
+            shift = float((ie != iq).float().mean().item())
+        d, G = c.head_dim, c.group
+        # stored bytes per token-head and tensor (the layout keeps the coefficient
+        # scale even at rank 0)
+        packed = d // 4 + 4 * (d // G) + (1 if c.n_centroids <= 256 else 2)
+        k_bytes = packed + r + 2 if which != "v" else 2 * d
+        v_bytes = packed if which != "k" else 2 * d
+        fixed = (c.heads * c.n_centroids * d * 2 * ((which != "v") + (which != "k"))
+                 + (c.frames // c.refresh_every) * c.heads * d * r * 4 * (which != "v"))
+        ratio = 4.0 * d * T * c.heads / (T * c.heads * (k_bytes + v_bytes) + fixed)
+        out.append({"ablation": name, "M": M, "r": r, "query_stats": stats, "quantized": which,
+                    "top1_shift": shift, "k_rel_mse": k_err, "v_rel_mse": v_err,
+                    "out_mse": o_mse, "out_rel_mse": o_mse / e_o, "compression_ratio": ratio,
+                    "workload": f"{c.name} layer, {c.frames} frames x {c.tokens_per_frame} "
+                                f"tokens, {c.heads} heads, queries of the last frame"})
+        del g, Kp, Vp, O
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------------------- oracle arm
 def oracle_throughput(cfg: syn.LayerConfig, cache=None, budget_s: float = 12.0):
     """The CPU oracle, as it stands, on a bounded sample of one step of the
@@ -307,6 +395,9 @@ def main():
     ap.add_argument("--cache-frames", type=int, default=0,
                     help="cache length in frames (default: the configuration's); smaller "
                          "values give the short runs used for ncu captures")
+    ap.add_argument("--ablation", action="store_true",
+                    help="instead of timing, print one JSON line per quantization setting "
+                         "(QVG, QSAC only, rank sweep, K-only, V-only) with its quality")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -318,6 +409,15 @@ def main():
                      f"{cfg.frames} latent frames x {cfg.tokens_per_frame} tokens, "
                      f"{cfg.q_rows}-query chunk, C={cfg.n_centroids}, G={cfg.group}, "
                      f"M={cfg.n_cand}, r={cfg.rank}")
+
+    if args.ablation:
+        if rank == 0:
+            device = torch.device("cuda", local)
+            torch.cuda.set_device(device)
+            frames = args.cache_frames if args.cache_frames > 0 else cfg.frames
+            for line in run_ablation(syn.get_config(args.config), device, frames):
+                print(json.dumps(line), flush=True)
+        return
 
     if args.impl == "reference":
         if rank != 0:

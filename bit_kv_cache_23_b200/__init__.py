@@ -21,7 +21,7 @@ __all__ = [
     "QwmError", "qwm_config", "qwm_sizes", "qwm_buffers", "qwm_cache", "BUFFER_NAMES",
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
     "qwm_build_centroids", "qwm_build_centroids_noalloc", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
-    "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
+    "qwm_attention_ext", "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +90,7 @@ def lib():
             "qwm_update_query_stats": (I32, [pc, _P, I64, I32, _P]),
             "qwm_append_kv": (I32, [pc, _P, _P, I64, _P]),
             "qwm_attention": (I32, [pc, _P, I64, F32, _P, _P]),
+            "qwm_attention_ext": (I32, [pc, _P, I64, _P, _P, I64, F32, _P, _P, _P]),
             "qwm_reconstruct": (I32, [pc, I64, I64, _P, _P, _P]),
             "qwm_top1_shift": (I32, [pc, _P, I64, _P, _P, _P, _P]),
             "qwm_device_status": (I32, [ctypes.POINTER(ctypes.c_int32)]),
@@ -186,6 +187,27 @@ def qwm_attention(cache: qwm_cache, Q: torch.Tensor, O: torch.Tensor | None = No
     return O
 
 
+def qwm_attention_ext(cache: qwm_cache, Q: torch.Tensor, K_seg: torch.Tensor | None = None,
+                      V_seg: torch.Tensor | None = None, O: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, scale: float = 0.0,
+                      stream=None) -> torch.Tensor:
+    """Attention over the packed cache followed by the bf16 segment (K_seg, V_seg),
+    [n_seg][H][d]; lse, if given, is a [n_q][H] float32 tensor that receives the
+    natural-log softmax denominators."""
+    if O is None:
+        O = torch.empty_like(Q)
+    n_seg = 0 if K_seg is None else K_seg.shape[0]
+    if (K_seg is None) != (V_seg is None) or (V_seg is not None and V_seg.shape != K_seg.shape):
+        raise ValueError("K_seg and V_seg must be given together, with equal shapes")
+    kp = _dev_ptr(K_seg, "K_seg", torch.bfloat16) if n_seg else None
+    vp = _dev_ptr(V_seg, "V_seg", torch.bfloat16) if n_seg else None
+    lp = _dev_ptr(lse, "lse", torch.float32) if lse is not None else None
+    _check("qwm_attention_ext", lib().qwm_attention_ext(
+        ctypes.byref(cache), _dev_ptr(Q, "Q", torch.bfloat16), Q.shape[0], kp, vp, n_seg,
+        float(scale), _dev_ptr(O, "O", torch.bfloat16), lp, _stream(stream, Q.device)))
+    return O
+
+
 def qwm_reconstruct(cache: qwm_cache, t0: int, n: int, device, stream=None):
     H, d = cache.cfg.heads, cache.cfg.head_dim
     Kp = torch.empty((H, n, d), dtype=torch.bfloat16, device=device)
@@ -266,6 +288,10 @@ class QuantKVCache:
 
     def attention(self, Q, O=None, scale=0.0, stream=None):
         return qwm_attention(self.c, Q, O, scale, stream)
+
+    def attention_ext(self, Q, K_seg=None, V_seg=None, O=None, lse=None, scale=0.0,
+                      stream=None):
+        return qwm_attention_ext(self.c, Q, K_seg, V_seg, O, lse, scale, stream)
 
     def reconstruct(self, t0=0, n=None, stream=None):
         n = self.len - t0 if n is None else n

@@ -184,7 +184,30 @@ qwm_status qwm_attention(const qwm_cache* c, const void* Q, int64_t n_q, float s
   if (!(scale > 0.0f)) scale = 1.0f / sqrtf((float)D.d);
   CacheView v = view_of(c);
   return cuda_status(launch_attention(D, v, c->len, (const uint16_t*)Q, n_q, scale, (uint16_t*)O,
-                                      (cudaStream_t)stream));
+                                      Segment{}, (cudaStream_t)stream));
+}
+
+qwm_status qwm_attention_ext(const qwm_cache* c, const void* Q, int64_t n_q, const void* K_seg,
+                             const void* V_seg, int64_t n_seg, float scale, void* O, float* lse,
+                             void* stream) {
+  if (!cache_ok(c) || n_q < 0 || n_seg < 0 || (n_q > 0 && (!Q || !O)) ||
+      (n_seg > 0 && (!K_seg || !V_seg)))
+    return QWM_ERR_INVALID_ARG;
+  if ((Q && !aligned(Q, 16)) || (O && !aligned(O, 16)) || (K_seg && !aligned(K_seg, 16)) ||
+      (V_seg && !aligned(V_seg, 16)) || (lse && !aligned(lse, 4)))
+    return QWM_ERR_ALIGNMENT;
+  if (c->len + n_seg <= 0 || (c->len > 0 && !c->has_centroids)) return QWM_ERR_STATE;
+  if (n_q == 0) return QWM_OK;
+  Dims D = dims_of(&c->cfg);
+  if (!(scale > 0.0f)) scale = 1.0f / sqrtf((float)D.d);
+  CacheView v = view_of(c);
+  Segment sg;
+  sg.K = (const uint16_t*)K_seg;
+  sg.V = (const uint16_t*)V_seg;
+  sg.n = n_seg;
+  sg.lse = lse;
+  return cuda_status(launch_attention(D, v, c->len, (const uint16_t*)Q, n_q, scale, (uint16_t*)O,
+                                      sg, (cudaStream_t)stream));
 }
 
 qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, void* Kp, void* Vp,

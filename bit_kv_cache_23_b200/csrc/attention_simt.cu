@@ -14,10 +14,13 @@ constexpr int KT = 64;   // keys per tile
 
 __device__ __forceinline__ float round_bf16(float x) { return bf2f(f2bf(x)); }
 
+// Keys 0 .. T-1 come from the packed cache, keys T .. T+sg.n-1 from the bf16
+// segment.
 template <int D>
 __global__ void __launch_bounds__(256) attn_simt(const Dims Dm, const CacheView v, int64_t T,
                                                  const uint16_t* __restrict__ Q, int64_t nq,
-                                                 float scale_log2, uint16_t* __restrict__ O) {
+                                                 float scale_log2, uint16_t* __restrict__ O,
+                                                 const Segment sg) {
   extern __shared__ float sm[];
   float* Qs = sm;                   // [QT][D+1]
   float* Ks = Qs + QT * (D + 1);    // [KT][D+1]
@@ -37,7 +40,8 @@ __global__ void __launch_bounds__(256) attn_simt(const Dims Dm, const CacheView 
 #pragma unroll
   for (int u = 0; u < D / 4; ++u) o[u] = 0.0f;
   const PackedHead p = packed_head(v, Dm, h);
-  for (int64_t k0 = 0; k0 < T; k0 += KT) {
+  const int64_t Ttot = T + sg.n;
+  for (int64_t k0 = 0; k0 < Ttot; k0 += KT) {
     __syncthreads();
     for (int e = tid; e < KT * D; e += 256) {
       int kk = e / D, j = e % D;
@@ -47,6 +51,10 @@ __global__ void __launch_bounds__(256) attn_simt(const Dims Dm, const CacheView 
         const float* U_h = basis_of(v, Dm, v.tokver[t], h);
         kv = round_bf16(key_elem(p, Dm, U_h, t, j));
         vv = round_bf16(value_elem(p, Dm, t, j));
+      } else if (t < Ttot) {
+        const size_t o = ((size_t)(t - T) * H + h) * D + j;
+        kv = bf2f(sg.K[o]);
+        vv = bf2f(sg.V[o]);
       }
       Ks[kk * (D + 1) + j] = kv;
       Vs[kk * D + j] = vv;
@@ -64,7 +72,7 @@ __global__ void __launch_bounds__(256) attn_simt(const Dims Dm, const CacheView 
 #pragma unroll
     for (int u = 0; u < KT / 4; ++u) {
       int64_t t = k0 + u * 4 + sub;
-      s[u] = (t < T) ? s[u] * scale_log2 : -INFINITY;
+      s[u] = (t < Ttot) ? s[u] * scale_log2 : -INFINITY;
       mx = fmaxf(mx, s[u]);
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -96,6 +104,7 @@ __global__ void __launch_bounds__(256) attn_simt(const Dims Dm, const CacheView 
     const float inv = 1.0f / l;
 #pragma unroll
     for (int u = 0; u < D / 4; ++u) O[((size_t)q * H + h) * D + u * 4 + sub] = f2bf(o[u] * inv);
+    if (sg.lse && sub == 0) sg.lse[(size_t)q * H + h] = (m + log2f(l)) * 0.6931471805599453f;
   }
 }
 
@@ -183,7 +192,8 @@ __global__ void __launch_bounds__(256) top1_kernel(const Dims Dm, const CacheVie
 }  // namespace
 
 cudaError_t launch_attention_simt(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                                  int64_t nq, float scale, uint16_t* O, cudaStream_t s) {
+                                  int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                                  cudaStream_t s) {
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid((unsigned)((nq + QT - 1) / QT), D.H);
   if (D.d == 128) {
@@ -191,13 +201,13 @@ cudaError_t launch_attention_simt(const Dims& D, const CacheView& v, int64_t T, 
     cudaError_t e = cudaFuncSetAttribute(attn_simt<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    attn_simt<128><<<grid, 256, smem, s>>>(D, v, T, Q, nq, scale_log2, O);
+    attn_simt<128><<<grid, 256, smem, s>>>(D, v, T, Q, nq, scale_log2, O, sg);
   } else {
     size_t smem = (size_t)(QT * 65 + KT * 65 + KT * 64 + QT * (KT + 1)) * 4;
     cudaError_t e = cudaFuncSetAttribute(attn_simt<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    attn_simt<64><<<grid, 256, smem, s>>>(D, v, T, Q, nq, scale_log2, O);
+    attn_simt<64><<<grid, 256, smem, s>>>(D, v, T, Q, nq, scale_log2, O, sg);
   }
   return cudaGetLastError();
 }
@@ -230,9 +240,10 @@ cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint
 
 // head_dim 128 runs on the tensor cores; other shapes use the CUDA-core kernel.
 cudaError_t launch_attention(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                             int64_t nq, float scale, uint16_t* O, cudaStream_t s) {
-  if (attention_tc_supported(D)) return launch_attention_tc(D, v, T, Q, nq, scale, O, s);
-  return launch_attention_simt(D, v, T, Q, nq, scale, O, s);
+                             int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                             cudaStream_t s) {
+  if (attention_tc_supported(D)) return launch_attention_tc(D, v, T, Q, nq, scale, O, sg, s);
+  return launch_attention_simt(D, v, T, Q, nq, scale, O, sg, s);
 }
 
 }  // namespace qwm

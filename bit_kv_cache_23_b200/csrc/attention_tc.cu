@@ -98,13 +98,26 @@ enum {
 struct TcArgs {
   Dims Dm;
   CacheView v;
-  int64_t T;
+  int64_t T;     // packed tokens (key tiles 0 .. ntp - 1)
   const uint16_t* Q;
   int64_t nq;
   float scale_log2;
   uint16_t* O;
-  int kx;  // extra K width for the compensation (0, 16 or 32)
+  int kx;        // extra K width for the compensation (0, 16 or 32)
+  const uint16_t* Ks;  // bf16 segment [nseg][H][d] after the packed tokens (tiles ntp ..)
+  const uint16_t* Vs;
+  int64_t nseg;
+  float* lse;    // [nq][H] natural-log softmax denominators, or null
+  int ntp;       // key tiles of the packed part
 };
+
+// Valid keys of tile j: packed tiles first, then (SEG) the segment's tiles.
+template <bool SEG>
+__device__ __forceinline__ int tile_valid(const TcArgs& A, int j) {
+  const int64_t rem = (!SEG || j < A.ntp) ? A.T - (int64_t)j * KT
+                                          : A.nseg - (int64_t)(j - A.ntp) * KT;
+  return (int)(rem < KT ? rem : KT);
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -182,6 +195,7 @@ __device__ __forceinline__ float row_max(const float (&s)[64], int n) {
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
+template <bool SEG>
 __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              uint32_t tmem, int ntile, int nqt) {
   const int warp = threadIdx.x >> 5;
@@ -261,8 +275,7 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
         tc_fence_after();
       }
     }
-    const int64_t kb = (int64_t)j * KT;
-    const int nvalid = (int)((A.T - kb) < KT ? (A.T - kb) : KT);
+    const int nvalid = tile_valid<SEG>(A, j);
     float m_row;
     {
       float s[64];
@@ -326,6 +339,8 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
   float la, lb;
   f2unpack(l2, la, lb);
   const float inv = 1.0f / (la + lb);
+  // sum_t 2^(s_t scale log2 e) = l 2^m_used
+  if (A.lse && q < A.nq) A.lse[(size_t)q * H + h] = (m_used + log2f(la + lb)) * 0.6931471805599453f;
   uint4* dst = reinterpret_cast<uint4*>(A.O + ((size_t)q * H + h) * DH);
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
@@ -464,6 +479,27 @@ __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, con
   cp_async_commit();
 }
 
+// Segment tile jj (jj >= ntp): this thread's 16-byte chunks of the bf16 K and V
+// rows copied as they are into the same swizzled stage positions.
+__device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem, int jj, int k,
+                                                 int qq) {
+  const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
+  const int64_t t = (int64_t)(jj - A.ntp) * KT + k;
+  if (t < A.nseg) {
+    const size_t row = ((size_t)t * A.Dm.H + blockIdx.y) * DH;
+    const uint16_t* kr = A.Ks + row;
+    const uint16_t* vr = A.Vs + row;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = 4 * qq + ((cc + qq) & 3);
+      cp_async16(st + ST_K + sw128_off(k, c, KT), kr + c * 8);
+      cp_async16(st + ST_V + sw128_off(k, c, KT), vr + c * 8);
+    }
+  }
+  cp_async_commit();
+}
+
+template <bool SEG>
 __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              int ntile) {
   const int dq = threadIdx.x - 256;  // 0..255
@@ -475,18 +511,29 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
   const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
   uint32_t* kvinfo = reinterpret_cast<uint32_t*>(smem + OFF_INFO);
   bool ok = true;
+  const int ntp = SEG ? A.ntp : ntile;
+  // the version pair segment tiles carry: that of the last packed tile, so the
+  // compensation slab stays in place (segment keys have zero BX rows)
+  const uint32_t seg_pair =
+      (SEG && kx && ntp > 0) ? tile_pair_global(A.v.tokver, A.T, ntp - 1) : 0u;
   // prologue: gathers of tiles 0 and 1 (their K-hat / V' stages start free)
   for (int jj = 0; jj < 2 && jj < ntile; ++jj) {
-    if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
-    issue_gather(A, smem, ph, jj, k, qq);
+    if (!SEG || jj < ntp) {
+      if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
+      issue_gather(A, smem, ph, jj, k, qq);
+    } else {
+      issue_seg_gather(A, smem, jj, k, qq);
+    }
   }
   for (int j = 0; ok && j < ntile; ++j) {
     if (j + 2 < ntile) {
       const int j2 = j + 2;
-      if (!warp_wait(&bars[B_LOAD_FULL + j2 % NPK], (j2 / NPK) & 1)) { ok = false; break; }
+      if ((!SEG || j2 < ntp) &&
+          !warp_wait(&bars[B_LOAD_FULL + j2 % NPK], (j2 / NPK) & 1)) { ok = false; break; }
       if (j2 >= NKV &&
           !warp_wait(&bars[B_KV_EMPTY + j2 % NKV], ((j2 / NKV) - 1) & 1)) { ok = false; break; }
-      issue_gather(A, smem, ph, j2, k, qq);
+      if (!SEG || j2 < ntp) issue_gather(A, smem, ph, j2, k, qq);
+      else issue_seg_gather(A, smem, j2, k, qq);
       cp_async_wait<2>();
     } else if (j + 1 < ntile) {
       cp_async_wait<1>();
@@ -498,6 +545,23 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
     uint8_t* kb = st + ST_K;
     uint8_t* vb = st + ST_V;
     uint8_t* xb = st + ST_BX;
+    if (SEG && j >= ntp) {
+      // segment tile: rows already in place; zero rows past the segment's end
+      // and zero compensation rows
+      if ((int64_t)(j - ntp) * KT + k >= A.nseg) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t off = sw128_off(k, 4 * qq + cc, KT);
+          *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (qq < kx / 8) *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(0, 0, 0, 0);
+      if (dq == 0) kvinfo[s] = seg_pair;
+      fence_proxy_async_smem();
+      warp_arrive(&bars[B_KV_FULL + s]);
+      continue;
+    }
     const uint8_t* pk = smem + OFF_PK + sp * PK_BYTES;
     const int64_t t0 = (int64_t)j * KT;
     const int64_t t = t0 + k;
@@ -746,6 +810,7 @@ __device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_
   if (!ok) timeout_flag();
 }
 
+template <bool SEG>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -753,7 +818,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBAR * 8);
   const int warp = threadIdx.x / 32;
-  const int ntile = (int)((A.T + KT - 1) / KT);
+  const int ntile = SEG ? A.ntp + (int)((A.nseg + KT - 1) / KT) : A.ntp;
   const int nqt = ((int64_t)blockIdx.x * BQ + QT < A.nq) ? 2 : 1;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NPK; ++i) {
@@ -788,15 +853,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   if (warp < 8) {
-    softmax_role(A, smem, bars, tmem, ntile, nqt);
+    softmax_role<SEG>(A, smem, bars, tmem, ntile, nqt);
   } else if (warp < 8 + NDQW) {
-    dequant_role(A, smem, bars, ntile);
+    dequant_role<SEG>(A, smem, bars, ntile);
   } else if (warp < W_PROD) {
     const int p = warp - W_MMA;
     if ((threadIdx.x & 31) == 0 && p < nqt) mma_role(A, smem, bars, tmem, ntile, p);
     __syncwarp();
   } else {
-    producer_role(A, smem, bars, ntile);
+    producer_role(A, smem, bars, A.ntp);  // packed tiles only
   }
   tc_fence_before();
   __syncthreads();
@@ -811,7 +876,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
 bool attention_tc_supported(const Dims& D) { return D.d == DH; }
 
 cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                                int64_t nq, float scale, uint16_t* O, cudaStream_t s) {
+                                int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                                cudaStream_t s) {
   TcArgs a;
   a.Dm = D;
   a.v = v;
@@ -820,12 +886,20 @@ cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, co
   a.nq = nq;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
-  a.kx = (D.r == 0) ? 0 : (D.r <= 8 ? 16 : 32);  // two slots of 8 or 16 columns
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  // two slots of 8 or 16 columns; none without packed keys
+  a.kx = (D.r == 0 || T == 0) ? 0 : (D.r <= 8 ? 16 : 32);
+  a.Ks = sg.K;
+  a.Vs = sg.V;
+  a.nseg = sg.n;
+  a.lse = sg.lse;
+  a.ntp = (int)((T + KT - 1) / KT);
+  // the segment variant only when there is one (no extra branches otherwise)
+  auto kern = sg.n > 0 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((nq + BQ - 1) / BQ), D.H);
-  attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(a);
+  kern<<<grid, NTHREADS, SMEM_BYTES, s>>>(a);
   return cudaGetLastError();
 }
 

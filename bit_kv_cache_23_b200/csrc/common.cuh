@@ -92,6 +92,16 @@ __device__ __forceinline__ int int2_code(float rho, float mn, float sc) {
   return c;
 }
 
+// Keys and values attended after the packed cache: a bf16 segment
+// [n][H][d] (token-major, like K and V), and an optional [nq][H] fp32 output of
+// the natural-log softmax denominators.
+struct Segment {
+  const uint16_t* K = nullptr;
+  const uint16_t* V = nullptr;
+  int64_t n = 0;
+  float* lse = nullptr;
+};
+
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_init_state(const Dims& D, const CacheView& v, cudaStream_t s);
 cudaError_t launch_kmeans(const Dims& D, const uint16_t* X, int64_t n, int iters, uint16_t* cent_out,
@@ -103,7 +113,8 @@ cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, i
 cudaError_t launch_append(const Dims& D, const CacheView& v, const uint16_t* K, const uint16_t* V,
                           int64_t n, int64_t t0, int version, cudaStream_t s);
 cudaError_t launch_attention(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                             int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+                             int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                             cudaStream_t s);
 cudaError_t launch_reconstruct(const Dims& D, const CacheView& v, int64_t t0, int64_t n,
                                uint16_t* Kp, uint16_t* Vp, cudaStream_t s);
 cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
@@ -113,9 +124,11 @@ cudaError_t launch_top1(const Dims& D, const CacheView& v, int64_t T, const uint
 size_t kmeans_workspace_bytes(const Dims& D);
 bool attention_tc_supported(const Dims& D);
 cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                                int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+                                int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                                cudaStream_t s);
 cudaError_t launch_attention_simt(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
-                                  int64_t nq, float scale, uint16_t* O, cudaStream_t s);
+                                  int64_t nq, float scale, uint16_t* O, const Segment& sg,
+                                  cudaStream_t s);
 int read_and_clear_tc_timeout();
 int read_and_clear_append_timeout();
 bool append_tc_supported(const Dims& D);

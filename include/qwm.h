@@ -181,6 +181,25 @@ QWM_API qwm_status qwm_append_kv(qwm_cache* c, const void* K, const void* V, int
 QWM_API qwm_status qwm_attention(const qwm_cache* c, const void* Q, int64_t n_q, float scale, void* O,
                          void* stream);
 
+/* Attention over the packed history followed by a bf16 segment: keys
+ * 0 .. len-1 reconstructed from the packed cache as in qwm_attention, then
+ * keys len .. len+n_seg-1 taken exactly from K_seg / V_seg.  In an
+ * autoregressive world model the cache holds the finished frames while the
+ * frame being generated attends to them and to its own, not yet quantized,
+ * keys and values at every denoising step ("Flickering after quantization?",
+ * opening paragraphs: the KV cache stores the historical frames); the pages do
+ * not describe this step, and this is its plainest reading.  With len == 0 it
+ * is plain bf16 attention over the segment.
+ * Q, O: [n_q][H][d] bf16 device; K_seg, V_seg: [n_seg][H][d] bf16 device
+ * (may be null when n_seg == 0); lse: null, or [n_q][H] fp32 device receiving
+ * ln sum_t exp(scale q . k_t) over all len + n_seg keys, for merging with
+ * attention over other keys.  scale <= 0 selects 1/sqrt(d).  Nothing is
+ * stored in the cache.  Errors: INVALID_ARG, ALIGNMENT, STATE (no keys at all,
+ * or a non-empty cache without centroids), CUDA. */
+QWM_API qwm_status qwm_attention_ext(const qwm_cache* c, const void* Q, int64_t n_q,
+                                     const void* K_seg, const void* V_seg, int64_t n_seg,
+                                     float scale, void* O, float* lse, void* stream);
+
 /* Reconstructed cache, for inspection: K', V' of tokens [t0, t0+n) as
  * [H][n][d] bf16 device arrays.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
 QWM_API qwm_status qwm_reconstruct(const qwm_cache* c, int64_t t0, int64_t n, void* Kp, void* Vp,

@@ -76,6 +76,7 @@ def lib():
             "qo_reconstruct_head": (None, [I32, I32, I32, I32, I32, I32, I64, I64, P, P, P, P,
                                            P, P, P, P, P, P, P, P, P, P]),
             "qo_attention_head": (None, [P, I64, I64, P, P, I64, I32, F64, P]),
+            "qo_attention_lse": (None, [P, I64, I64, P, I64, I32, F64, P]),
             "qo_top1": (None, [P, I64, I64, P, I64, I64, I32, P]),
             "qo_bytes_per_token_head": (I64, [I32, I32, I32, I32]),
         }
@@ -238,6 +239,15 @@ def attention_head(Q, Kp, Vp, scale):
     O = np.zeros((nq, d), np.float64)
     lib().qo_attention_head(_p(Q), nq, d, _p(Kp), _p(Vp), T, d, float(scale), _p(O))
     return O
+
+
+def attention_lse(Q, K, scale):
+    """Q [nq][d], K [T][d] (bf16 bits) -> ln sum_t exp(scale q . k_t) per row, fp64."""
+    Q = np.ascontiguousarray(Q, np.uint16); K = np.ascontiguousarray(K, np.uint16)
+    nq, d = Q.shape
+    out = np.zeros(nq, np.float64)
+    lib().qo_attention_lse(_p(Q), nq, d, _p(K), K.shape[0], d, float(scale), _p(out))
+    return out
 
 
 def top1(Q, K):

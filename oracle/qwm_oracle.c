@@ -605,6 +605,29 @@ QO_API void qo_attention_head(const uint16_t* Q, int64_t nq, int64_t qstride, co
   free(l); free(q);
 }
 
+/* Log of the softmax denominator of each query row over keys K [T][d] (fp64):
+ *   lse_i = ln sum_t exp(scale * q_i . k_t),  taken as m + ln sum exp(l_t - m)
+ * with m the row maximum (so that two attentions over disjoint key sets can be
+ * merged with weights exp(lse)).  T == 0 gives -inf. */
+QO_API void qo_attention_lse(const uint16_t* Q, int64_t nq, int64_t qstride, const uint16_t* K,
+                             int64_t T, int d, double scale, double* lse) {
+  double* l = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  for (int64_t i = 0; i < nq; ++i) {
+    double m = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j)
+        acc += (double)bf(Q[i * qstride + j]) * (double)bf(K[(size_t)t * d + j]);
+      l[t] = acc * scale;
+      if (l[t] > m) m = l[t];
+    }
+    double den = 0.0;
+    for (int64_t t = 0; t < T; ++t) den += exp(l[t] - m);
+    lse[i] = (T > 0) ? m + log(den) : -INFINITY;
+  }
+  free(l);
+}
+
 /* Top-1 key of each query row: argmax_t q . k_t (fp64 dot of the bf16 values),
  * ties to the lower t.  K rows with stride `kstride`. */
 QO_API void qo_top1(const uint16_t* Q, int64_t nq, int64_t qstride, const uint16_t* K, int64_t T,

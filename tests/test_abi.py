@@ -107,6 +107,28 @@ def test_call_order_and_capacity_errors():
     assert L.qwm_build_centroids(ctypes.byref(c), p, p, 100, 10, None) == 1  # n < C
 
 
+def test_attention_ext_argument_checks():
+    L = q.lib()
+    p = ctypes.c_void_p(0x200000)
+    c = _fake_cache(has_centroids=1, len=0)
+    # no keys at all: empty cache and empty segment
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, None, None, 0, 0.0, p, None, None) == 4
+    # a segment needs both K and V
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, p, None, 8, 0.0, p, None, None) == 1
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, p, p, -1, 0.0, p, None, None) == 1
+    # 16-byte alignment of the segment, 4-byte alignment of lse
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, ctypes.c_void_p(0x200008), p, 8, 0.0, p,
+                               None, None) == 2
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, p, p, 8, 0.0, p,
+                               ctypes.c_void_p(0x200002), None) == 2
+    # a non-empty cache without centroids
+    c = _fake_cache(has_centroids=0, len=10)
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 4, p, p, 8, 0.0, p, None, None) == 4
+    # nothing to do for zero query rows (no device work)
+    c = _fake_cache(has_centroids=1, len=0)
+    assert L.qwm_attention_ext(ctypes.byref(c), p, 0, p, p, 8, 0.0, p, None, None) == 0
+
+
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(q.qwm_config) == 40
     assert ctypes.sizeof(q.qwm_buffers) == 8 * q.NBUF

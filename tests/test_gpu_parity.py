@@ -71,6 +71,38 @@ def test_top1_shift_tiny():
         assert np.all(best - mine <= 1e-4 * np.abs(best) + 1e-4)
 
 
+def test_qvg_mode_without_statistics():
+    """QVG reading (M = 1, s = 1, r = 0): no Query statistics are ever taken, so
+    every key goes to its plain nearest centroid; head_dim 128 and 64."""
+    q = pytest.importorskip("bit_kv_cache_23_b200")
+    for (H, d, C, G, n) in [(3, 128, 256, 32, 900), (2, 64, 16, 16, 300)]:
+        g = q.QuantKVCache(H, d, C, G, 1, 0, 2 * n, max_versions=2)
+        oc = oracle.OracleCache(H, d, C, G, 1, 0, 2 * n)
+        rng = np.random.default_rng(4000 + d)
+        w = np.ones(d)
+        w[rng.permutation(d)[:4]] = 6.0
+        K = [syn.f32_to_bf16_bits((rng.standard_normal((n, H, d)) * w).astype(np.float32))
+             for _ in range(2)]
+        V = [syn.f32_to_bf16_bits(rng.standard_normal((n, H, d)).astype(np.float32))
+             for _ in range(2)]
+        g.build_centroids(to_dev(K[0]), to_dev(V[0]), iters=3)
+        ck = np.stack([oracle.kmeans(K[0][:, h, :], C, 3)[0] for h in range(H)])
+        cv = np.stack([oracle.kmeans(V[0][:, h, :], C, 3)[0] for h in range(H)])
+        oc.set_state(CK=ck, CV=cv)
+        for f in range(2):
+            t0 = g.len
+            g.append_kv(to_dev(K[f]), to_dev(V[f]))
+            oc.append_kv(K[f], V[f])
+            assert compare_packed(g, oc, t0, g.len) == {}, (d, f)
+        Q = syn.f32_to_bf16_bits(rng.standard_normal((150, H, d)).astype(np.float32))
+        O = g.attention(to_dev(Q))
+        torch.cuda.synchronize()
+        assert q.qwm_device_status() == 0
+        Oref = oc.attention(Q)
+        err = np.abs(syn.bf16_bits_to_f32(u16(O)) - Oref)
+        assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (d, err.max(), err.mean())
+
+
 def test_degenerate_inputs():
     """Constant keys (zero residual groups), repeated tokens, one-token appends,
     a ragged tail and zero-variance channels."""
@@ -120,11 +152,16 @@ def test_degenerate_inputs():
     assert err.max() <= 2e-2 and err.mean() <= 2e-3
 
 
-@pytest.mark.parametrize("G,C,M,r", [(16, 64, 4, 8), (32, 48, 3, 16), (16, 512, 8, 5)])
+@pytest.mark.parametrize("G,C,M,r", [(16, 64, 4, 8), (32, 48, 3, 16), (16, 512, 8, 5),
+                                     (32, 256, 1, 0), (32, 256, 4, 0), (32, 256, 1, 8),
+                                     (32, 256, 4, 2), (16, 128, 4, 4)])
 def test_head128_shapes(G, C, M, r):
     """head_dim 128 with groups of 16, C not a power of two, C = 512 (two MMA
     chunks), M up to 8 and ranks other than 8: every packed field bit for bit,
-    attention within tolerance; keys with outlier channels and frame drift."""
+    attention within tolerance; keys with outlier channels and frame drift.
+    Also the ablation settings: M = 1 and r = 0 (plain nearest centroid with the
+    sensitivity weights, no compensation), QSAC alone (r = 0), PSAC alone
+    (M = 1), and ranks 2 and 4."""
     H, d, n = 3, 128, 700
     q = pytest.importorskip("bit_kv_cache_23_b200")
     g = q.QuantKVCache(H, d, C, G, M, r, 3 * n, max_versions=8)
@@ -156,7 +193,7 @@ def test_head128_shapes(G, C, M, r):
         st = refresh_from_oracle(g, Mref, 200 * (f + 1), range(H), r, G, rep,
                                  check_basis=(r <= 8))
         s, w, U = stack_state(st, H)
-        oc.set_state(s=s, w=w, U=U)
+        oc.set_state(s=s, w=w, U=U if r else None)
         t0 = g.len
         g.append_kv(to_dev(K[f]), to_dev(V[f]))
         oc.append_kv(K[f], V[f])

@@ -342,6 +342,40 @@ def test_attention_unquantized_matches_sdpa_fp64():
         assert np.abs(O - ref.numpy()).max() <= 1e-5
 
 
+def test_attention_lse_brute_force_and_invariants():
+    """ln sum exp against math.fsum over Python floats on small cases; equal keys
+    give s + ln T; a key set split in two merges through the log-sum-exp weights
+    into the attention over the union."""
+    rng = np.random.default_rng(33)
+    for (nq, T, d) in [(3, 1, 64), (4, 37, 64), (2, 130, 128)]:
+        Q = _bf(rng.standard_normal((nq, d)))
+        K = _bf(rng.standard_normal((T, d)) * 3)
+        sc = 1.0 / math.sqrt(d)
+        got = oracle.attention_lse(Q, K, sc)
+        qf = syn.bf16_bits_to_f32(Q).astype(np.float64)
+        kf = syn.bf16_bits_to_f32(K).astype(np.float64)
+        for i in range(nq):
+            s = [sc * math.fsum(float(a) * float(b) for a, b in zip(qf[i], kf[t])) for t in range(T)]
+            m = max(s)
+            ref = m + math.log(math.fsum(math.exp(x - m) for x in s))
+            assert abs(got[i] - ref) <= 1e-12 * max(1.0, abs(ref))
+    Q = _bf(rng.standard_normal((3, 64)))
+    k = _bf(rng.standard_normal((1, 64)))
+    K = np.repeat(k, 50, axis=0)
+    s0 = (syn.bf16_bits_to_f32(Q).astype(np.float64) @ syn.bf16_bits_to_f32(k[0]).astype(np.float64)) * 0.125
+    assert np.allclose(oracle.attention_lse(Q, K, 0.125), s0 + math.log(50), rtol=0, atol=1e-12)
+    K = _bf(rng.standard_normal((90, 64)))
+    V = _bf(rng.standard_normal((90, 64)))
+    Q = _bf(rng.standard_normal((5, 64)))
+    O = oracle.attention_head(Q, K, V, 0.125)
+    O1, O2 = oracle.attention_head(Q, K[:40], V[:40], 0.125), oracle.attention_head(Q, K[40:], V[40:], 0.125)
+    l1, l2 = oracle.attention_lse(Q, K[:40], 0.125), oracle.attention_lse(Q, K[40:], 0.125)
+    l = oracle.attention_lse(Q, K, 0.125)
+    w1, w2 = np.exp(l1 - l)[:, None], np.exp(l2 - l)[:, None]
+    assert np.allclose(w1 + w2, 1.0, atol=1e-12)
+    assert np.allclose(w1 * O1 + w2 * O2, O, atol=1e-12)
+
+
 def test_top1_matches_numpy_argmax():
     rng = np.random.default_rng(32)
     Q = _bf(rng.standard_normal((20, 64)))
