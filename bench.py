@@ -165,22 +165,27 @@ def dev_bf16(a: np.ndarray, device) -> torch.Tensor:
 
 
 class Workload:
-    def __init__(self, cfg: syn.LayerConfig, device, extra_versions: int, pool: int = 4):
+    """The layer (or this rank's block of its heads) filled with all its frames."""
+
+    def __init__(self, cfg: syn.LayerConfig, device, extra_versions: int, pool: int = 4,
+                 heads=None):
         import bit_kv_cache_23_b200 as q
 
         self.cfg = cfg
         self.device = device
         c = cfg
-        self.cache = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand,
-                                    c.rank, c.total_tokens,
+        self.heads = list(range(c.heads)) if heads is None else list(heads)
+        self.cache = q.QuantKVCache(len(self.heads), c.head_dim, c.n_centroids, c.group,
+                                    c.n_cand, c.rank, c.total_tokens,
                                     max_versions=c.frames // c.refresh_every + extra_versions + 4,
                                     device=device)
         src = syn.FrameSource(c)
         self.src = src
         self.pool = []
         self.host_pool = []
+        hs = None if heads is None else self.heads
         for f in range(c.frames):
-            Q, K, V = src.frame(f)
+            Q, K, V = src.frame(f, hs)
             Qd, Kd, Vd = dev_bf16(Q, device), dev_bf16(K, device), dev_bf16(V, device)
             if f == 0:
                 self.cache.build_centroids(Kd, Vd, iters=c.kmeans_iters)
@@ -395,6 +400,10 @@ def main():
     ap.add_argument("--cache-frames", type=int, default=0,
                     help="cache length in frames (default: the configuration's); smaller "
                          "values give the short runs used for ncu captures")
+    ap.add_argument("--shard", default="replica", choices=["replica", "heads"],
+                    help="with several ranks: a whole layer per rank (weak scaling), or the "
+                         "layer's heads split over the ranks (strong scaling); neither "
+                         "exchanges data between ranks")
     ap.add_argument("--ablation", action="store_true",
                     help="instead of timing, print one JSON line per quantization setting "
                          "(QVG, QSAC only, rank sweep, K-only, V-only) with its quality")
@@ -453,18 +462,25 @@ def main():
     torch.cuda.set_device(device)
     peaks = load_peaks()
     W, K = max(3, args.warmup), args.steps
-    wl = Workload(cfg, device, extra_versions=2 * (W + K) + 8)
+    from bit_kv_cache_23_b200 import shard
+
+    if args.shard == "heads":
+        h0, h1 = shard.head_range(rank, world, cfg.heads)
+        heads = list(range(h0, h1))
+    else:
+        heads = None
+    wl = Workload(cfg, device, extra_versions=2 * (W + K) + 8, heads=heads)
+    nh = len(wl.heads)
+    # query tokens of the whole layer this rank serves per step (a fraction of a
+    # layer when the heads are split)
+    units = cfg.q_rows * nh / cfg.heads
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return shard.max_over_ranks(x, device)
 
     for i in range(W):
         wl.step(i)
@@ -489,7 +505,7 @@ def main():
                     for e in evs])
     stats_ms, app_ms, att_ms = (float(x) for x in seg.mean(0))
     ms_step = total_ms / K
-    value = world * cfg.q_rows / (ms_step * 1e-3)
+    value = shard.throughput(units, ms_step * 1e-3, device)
     # our kernels in the timed region: per step statistics, append K and V and
     # attention, plus the refresh kernel on the steps that refresh the basis
     n_launches = 4 * K + sum(1 for n in range(nstep0, nstep0 + K) if n % cfg.refresh_every == 0)
@@ -512,24 +528,26 @@ def main():
         torch.cuda.synchronize(device)
         barrier()
         e2e_ms = max_over_ranks(s2.elapsed_time(e2)) / K
-        e2e = {"value": world * cfg.q_rows / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e = {"value": shard.throughput(units, e2e_ms * 1e-3, device), "unit": UNIT,
                "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),
                "d2h_bytes_per_step": int(Qh.numel() * 2)}
 
     # ---- derived figures
     c = cfg
     T = c.total_tokens
-    att_flop = 4.0 * c.q_rows * T * c.head_dim * c.heads
+    # per launch on this rank (its heads)
+    att_flop = 4.0 * c.q_rows * T * c.head_dim * nh
     att_tflops = att_flop / (att_ms * 1e-3) / 1e12
     per_tok = 2 * (c.head_dim // 4 + 4 * (c.head_dim // c.group) + (1 if c.n_centroids <= 256 else 2)) + c.rank + 2
-    app_bytes = c.tokens_per_frame * c.heads * (4 * c.head_dim + per_tok)
+    app_bytes = c.tokens_per_frame * nh * (4 * c.head_dim + per_tok)
     app_gbs = app_bytes / (app_ms * 1e-3) / 1e9
     fixed = 2 * c.heads * c.n_centroids * c.head_dim * 2 + (c.frames // c.refresh_every) * c.heads * c.head_dim * c.rank * 4
     compression = (4.0 * c.head_dim * T * c.heads) / (T * c.heads * per_tok + fixed)
 
     top1 = None
     if not args.no_top1 and rank == 0:
-        Kall = torch.cat([dev_bf16(wl.src.keys(f), device) for f in range(c.frames - 1)]
+        hs = None if heads is None else wl.heads
+        Kall = torch.cat([dev_bf16(wl.src.keys(f, hs), device) for f in range(c.frames - 1)]
                          + [wl.pool[(wl.nstep - 1) % len(wl.pool)][1]], 0)
         ie, iq = wl.cache.top1_shift(wl.pool[(wl.nstep - 1) % len(wl.pool)][0], Kall)
         top1 = float((ie != iq).float().mean().item())
@@ -537,13 +555,15 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_name,
-                   "l2": (f"packed cache of {T * c.heads * per_tok / 1e6:.0f} MB read per step "
-                          f"({'larger' if T * c.heads * per_tok > 126e6 else 'smaller'} than "
+                   "l2": (f"packed cache of {T * nh * per_tok / 1e6:.0f} MB read per step "
+                          f"({'larger' if T * nh * per_tok > 126e6 else 'smaller'} than "
                           "the 126 MB L2), step inputs rotate over 4 HBM-resident frames"),
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": (f"heads split over {world} ranks ({nh} on rank 0)"
+                                   if args.shard == "heads" else f"replicas x{world}")},
         "gpu_launches": n_launches,
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16"],
                      "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
