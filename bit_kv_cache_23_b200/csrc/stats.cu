@@ -260,12 +260,12 @@ __device__ void small_jacobi(double* G, double* W) {
           be += __shfl_xor_sync(0xffffffffu, be, o);
           ga += __shfl_xor_sync(0xffffffffu, ga, o);
         }
-        const double nrm = sqrt(al * be);
-        if (ga != 0.0 && fabs(ga) > 1e-15 * nrm) {
-          worst = fmaxf(worst, (float)(fabs(ga) / nrm));
+        // rotate unless the pair is orthogonal to 1e-15 (compared squared: no root)
+        if (ga != 0.0 && ga * ga > 1e-30 * (al * be)) {
+          worst = fmaxf(worst, fabsf((float)ga) * rsqrtf((float)al * (float)be));
           const double zeta = (be - al) / (2.0 * ga);
           const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-          const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
+          const double c = rsqrt(1.0 + t * t), s = c * t;
           double* wp = W + pp * P;
           double* wq = W + qq * P;
 #pragma unroll
