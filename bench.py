@@ -273,16 +273,18 @@ class Workload:
 
 
 # ----------------------------------------------------------------------------- ablations
-# (name, M, r, Query statistics taken, tensors quantized); None = the layer's own.
+# (name, M, r, Query statistics taken, tensors quantized, full-quadratic QSAC);
+# None = the layer's own.
 ABLATIONS = [
-    ("quantwm", None, None, True, "kv"),     # QSAC + PSAC, both tensors
-    ("qvg", 1, 0, False, "kv"),              # plain nearest centroid: M = 1, s = 1, r = 0
-    ("qsac_only", None, 0, True, "kv"),      # no compensation (rank 0)
-    ("rank2", None, 2, True, "kv"),
-    ("rank4", None, 4, True, "kv"),
-    ("rank16", None, 16, True, "kv"),
-    ("k_only", None, None, True, "k"),       # Keys quantized, Values exact
-    ("v_only", None, None, True, "v"),       # Values quantized, Keys exact
+    ("quantwm", None, None, True, "kv", False),     # QSAC + PSAC, both tensors
+    ("qvg", 1, 0, False, "kv", False),              # nearest centroid: M = 1, s = 1, r = 0
+    ("qsac_only", None, 0, True, "kv", False),      # no compensation (rank 0)
+    ("rank2", None, 2, True, "kv", False),
+    ("rank4", None, 4, True, "kv", False),
+    ("rank16", None, 16, True, "kv", False),
+    ("qsac_full_quadratic", None, None, True, "kv", True),  # stage 2 by e^T A e
+    ("k_only", None, None, True, "k", False),       # Keys quantized, Values exact
+    ("v_only", None, None, True, "v", False),       # Values quantized, Keys exact
 ]
 
 
@@ -312,11 +314,11 @@ def run_ablation(cfg: syn.LayerConfig, device, frames: int) -> list:
     e_o = Oexact.pow(2).mean().item()
     e_k, e_v = Kx.float().pow(2).mean().item(), Vx.float().pow(2).mean().item()
     out = []
-    for name, M, r, stats, which in ABLATIONS:
+    for name, M, r, stats, which, full in ABLATIONS:
         M = c.n_cand if M is None else M
         r = c.rank if r is None else r
         g = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, M, r, T,
-                           max_versions=c.frames + 2, device=device)
+                           max_versions=c.frames + 2, device=device, qsac_full=full)
         for f, (Q, K, V) in enumerate(data):
             Kd, Vd = dev_bf16(K, device), dev_bf16(V, device)
             if f == 0:
@@ -351,6 +353,7 @@ def run_ablation(cfg: syn.LayerConfig, device, frames: int) -> list:
                  + (c.frames // c.refresh_every) * c.heads * d * r * 4 * (which != "v"))
         ratio = 4.0 * d * T * c.heads / (T * c.heads * (k_bytes + v_bytes) + fixed)
         out.append({"ablation": name, "M": M, "r": r, "query_stats": stats, "quantized": which,
+                    "qsac_full_quadratic": full,
                     "top1_shift": shift, "k_rel_mse": k_err, "v_rel_mse": v_err,
                     "out_mse": o_mse, "out_rel_mse": o_mse / e_o, "compression_ratio": ratio,
                     "workload": f"{c.name} layer, {c.frames} frames x {c.tokens_per_frame} "

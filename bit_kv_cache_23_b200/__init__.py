@@ -22,10 +22,13 @@ __all__ = [
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
     "qwm_build_centroids", "qwm_build_centroids_noalloc", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
     "qwm_attention_ext", "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
+    "QWM_FLAG_QSAC_FULL",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqwm.so")
+
+QWM_FLAG_QSAC_FULL = 1   # QSAC stage 2 by the full quadratic form e^T A e
 
 BUFFER_NAMES = ["k_codes", "k_params", "k_idx", "k_coef", "k_cscale", "v_codes", "v_params",
                 "v_idx", "cent_k", "cent_v", "qstats", "sens", "wgroup", "basis", "tokver",
@@ -40,7 +43,7 @@ class qwm_config(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("n_centroids", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("n_cand", ctypes.c_int32), ("rank", ctypes.c_int32),
-                ("max_versions", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("max_versions", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int64)]
 
 
@@ -246,12 +249,13 @@ class QuantKVCache:
 
     def __init__(self, heads: int, head_dim: int, n_centroids: int, group: int, n_cand: int,
                  rank: int, max_tokens: int, max_versions: int = 1024, device="cuda",
-                 stream=None):
+                 stream=None, qsac_full: bool = False):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("QuantKVCache lives on a CUDA device")
-        self.cfg = qwm_config(heads, head_dim, n_centroids, group, n_cand, rank, max_versions, 0,
-                              max_tokens)
+        flags = QWM_FLAG_QSAC_FULL if qsac_full else 0
+        self.cfg = qwm_config(heads, head_dim, n_centroids, group, n_cand, rank, max_versions,
+                              flags, max_tokens)
         self.sizes = qwm_cache_sizes(self.cfg)
         self.buffers = {}
         bufs = qwm_buffers()

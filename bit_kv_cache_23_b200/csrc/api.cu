@@ -20,7 +20,7 @@ bool config_ok(const qwm_config* c) {
   if (c->n_cand < 1 || c->n_cand > 8 || c->n_cand > c->n_centroids) return false;
   if (c->rank < 0 || c->rank > 16) return false;
   if (c->max_versions < 1 || c->max_versions > 65535) return false;
-  if (c->reserved != 0) return false;
+  if ((c->flags & ~QWM_FLAG_QSAC_FULL) != 0) return false;
   if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 40)) return false;
   return true;
 }
@@ -36,6 +36,7 @@ Dims dims_of(const qwm_config* c) {
   D.ng = c->head_dim / c->group;
   D.tcap = (c->max_tokens + 127) / 128 * 128;
   D.idx_bytes = c->n_centroids <= 256 ? 1 : 2;
+  D.qsac_full = (c->flags & QWM_FLAG_QSAC_FULL) ? 1 : 0;
   return D;
 }
 

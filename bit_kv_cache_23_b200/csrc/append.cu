@@ -9,7 +9,10 @@
 //      perturbation of its INT2 residual, sum_g w_g R_g^2 (R_g the residual's
 //      range in group g, w_g = sum of s over the group; the constant 1/108 of
 //      step^2/12 with step = R/3 is dropped), folded over groups in order;
-//      ties keep the earlier shortlist position;
+//      ties keep the earlier shortlist position.  With the full-quadratic
+//      option the score is e^T A e instead (e the Key error the candidate
+//      leaves after INT2, A = fp32(M / n) in force; y_i = fold_j fma(A_ij, e_j),
+//      then fold_i fma(e_i, y_i));
 //   3. INT2 residual: per group mn = fp16 round-down(min), sc = fp16
 //      round-up((max - mn)/3), code = #{k : rho >= mn + (k + 0.5) sc};
 //   4. PSAC: e = k - (c + mn + code sc); coef_q = fold_j fma(U_jq, e_j, acc);
@@ -49,12 +52,55 @@ struct AppendArgs {
   int8_t* coef;           // [H][tcap][r]  (keys)
   uint16_t* cscale;       // [H][tcap]     (keys)
   uint16_t* tokver;       // [tcap]        (keys)
+  double* eigvec;         // refresh state holding A = fp32(M / n) per head (full-quadratic)
   int64_t n, t0, tcap;
-  int H, C, G, M, r, idx_bytes, version;
+  int H, C, G, M, r, idx_bytes, version, qfull;
 };
 
 __device__ __forceinline__ bool lex_less(float a, int ia, float b, int ib) {
   return a < b || (a == b && ia < ib);
+}
+
+// Full-quadratic QSAC score of one candidate, taken by one warp: lane owns
+// channels lane*CPL.. and the group range (lo, hi) of its group.  The Key error
+// e of the candidate goes to the warp's row `ew`; y_i = sum_j A_ij e_j is
+// folded over j in order by the lane owning row i (A symmetric: row i is read
+// as column i, coalesced), then lane 0 folds sum_i e_i y_i over i in order.
+template <int D>
+__device__ float full_score(const AppendArgs& A, int h, int lane, const float* kv,
+                            const uint16_t* crow, float lo, float hi, float* ew) {
+  constexpr int CPL = D / 32;
+  uint16_t mnh, sch;
+  float mn, sc;
+  int2_params(lo, hi, mnh, sch, mn, sc);
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) {
+    const float cv = bf2f(crow[u]);
+    const float rho = __fsub_rn(kv[u], cv);
+    const float deq = __fmaf_rn((float)int2_code(rho, mn, sc), sc, mn);
+    ew[lane * CPL + u] = __fsub_rn(kv[u], __fadd_rn(cv, deq));
+  }
+  __syncwarp();
+  const float* Ah = qsnap_of(A.eigvec, D, h);
+  float y[CPL];
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) {
+    const int i = u * 32 + lane;
+    float acc = 0.0f;
+    for (int j = 0; j < D; ++j) acc = __fmaf_rn(Ah[(size_t)j * D + i], ew[j], acc);
+    y[u] = acc;
+  }
+  float score = 0.0f;  // i = 32 u + l in increasing order
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) {
+    for (int l = 0; l < 32; ++l) {
+      const float yi = __shfl_sync(0xffffffffu, y[u], l);
+      score = __fmaf_rn(ew[32 * u + l], yi, score);
+    }
+  }
+  __syncwarp();  // every lane has read `ew` before the caller reuses it
+  return score;  // the same value on every lane
 }
 
 template <int D, bool KEY>
@@ -165,11 +211,15 @@ __global__ void __launch_bounds__(NT) append_kernel(AppendArgs A) {
             lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
             hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
           }
-          const float R = __fsub_rn(hi, lo);
           float score = 0.0f;
-          for (int g = 0; g < ng; ++g) {
-            float Rg = __shfl_sync(0xffffffffu, R, g * lpg);
-            score = __fmaf_rn(w_s[g], __fmul_rn(Rg, Rg), score);
+          if (A.qfull) {
+            score = full_score<D>(A, h, lane, kv, crow, lo, hi, es + warp * D);
+          } else {
+            const float R = __fsub_rn(hi, lo);
+            for (int g = 0; g < ng; ++g) {
+              float Rg = __shfl_sync(0xffffffffu, R, g * lpg);
+              score = __fmaf_rn(w_s[g], __fmul_rn(Rg, Rg), score);
+            }
           }
           if (bm < 0 || score < best) { best = score; bm = m; }
         }
@@ -301,6 +351,8 @@ cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_
   a.coef = v.k_coef;
   a.cscale = v.k_cscale;
   a.tokver = v.tokver;
+  a.eigvec = v.eigvec;
+  a.qfull = Dm.qsac_full;
   cudaError_t e = (Dm.d == 128) ? run<128, true>(a, s) : run<64, true>(a, s);
   if (e != cudaSuccess) return e;
   // values

@@ -604,7 +604,7 @@ int read_and_clear_append_timeout() {
 
 bool append_tc_supported(const Dims& D) {
   return D.d == DH && (D.G == 16 || D.G == 32) && D.C % 16 == 0 && D.C <= 512 && D.M <= 8 &&
-         D.r <= 16;
+         D.r <= 16 && !D.qsac_full;
 }
 
 cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t* K,

@@ -16,7 +16,14 @@ struct Dims {
   int H, d, C, G, M, r, ng;
   int64_t tcap;
   int idx_bytes;  // 1 if C <= 256 else 2
+  int qsac_full;  // QSAC stage 2 by the full quadratic form e^T A e
 };
+
+// fp32 snapshot A = M / n of head h kept with the refresh state (after the
+// first 32 Ritz-vector columns of the head's d x d fp64 block).
+__host__ __device__ inline float* qsnap_of(double* eigvec, int d, int h) {
+  return reinterpret_cast<float*>(eigvec + (size_t)h * d * d + 32 * (size_t)d);
+}
 
 // Views of the cache buffers (device pointers).
 struct CacheView {

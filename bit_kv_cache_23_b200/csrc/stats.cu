@@ -291,7 +291,7 @@ __device__ void small_jacobi(double* G, double* W) {
 // rows fit); head_dim D and block width P fixed at compile time.
 template <int D, int P>
 __global__ void __launch_bounds__(P == 32 ? 256 : 512) refresh_kernel(const double* __restrict__ Mall, int64_t n,
-                                                      int G, int r,
+                                                      int G, int r, int qfull,
                                                       float* __restrict__ sens,
                                                       float* __restrict__ wgroup,
                                                       float* __restrict__ basis_slot,
@@ -304,9 +304,12 @@ __global__ void __launch_bounds__(P == 32 ? 256 : 512) refresh_kernel(const doub
   float* s_out = sens + (size_t)h * d;
   float* w_out = wgroup + (size_t)h * (d / G);
   float* U = basis_slot + (size_t)h * d * (r > 0 ? r : 1);
+  float* snap = qsnap_of(eigvec, d, h);  // A = fp32(M / n) for the full-quadratic score
   if (n <= 0) {
     for (int j = tid; j < d; j += nt) s_out[j] = 1.0f;
     for (int e = tid; e < d * r; e += nt) U[e] = 0.0f;
+    if (qfull)
+      for (int e = tid; e < d * d; e += nt) snap[e] = 0.0f;
     __syncthreads();
     if (tid < d / G) {
       float acc = 0.0f;
@@ -328,6 +331,8 @@ __global__ void __launch_bounds__(P == 32 ? 256 : 512) refresh_kernel(const doub
   const double inv = 1.0 / (double)n;
   for (int e = tid; e < d * d; e += nt) S.A[(e / d) * (d + 1) + (e % d)] = M[e] * inv;
   for (int j = tid; j < d; j += nt) s_out[j] = __double2float_rn(M[(size_t)j * d + j] / (double)n);
+  if (qfull)
+    for (int e = tid; e < d * d; e += nt) snap[e] = __double2float_rn(M[e] / (double)n);
   __syncthreads();
   if (tid < d / G) {
     float acc = 0.0f;
@@ -475,8 +480,8 @@ cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, i
   else if (!(D.d == 128 && p == 16)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<D.H, p == 32 ? 256 : 512, smem, s>>>(v.qstats, n_total, D.G, D.r, v.sens, v.wgroup, slot, v.eigvec,
-                              flags);
+  kern<<<D.H, p == 32 ? 256 : 512, smem, s>>>(v.qstats, n_total, D.G, D.r, D.qsac_full, v.sens,
+                                               v.wgroup, slot, v.eigvec, flags);
   return cudaGetLastError();
 }
 

@@ -64,7 +64,19 @@ typedef enum qwm_status {
 
 /* Quantizer and capacity.  Supported: head_dim 64 or 128; group 16 or 32 and
  * dividing head_dim; 1 <= n_centroids <= 512; 1 <= n_cand <= min(8, C);
- * 0 <= rank <= 16; 1 <= max_versions <= 65535; max_tokens >= 1. */
+ * 0 <= rank <= 16; 1 <= max_versions <= 65535; max_tokens >= 1; flags a
+ * combination of the QWM_FLAG_* bits. */
+
+/* QSAC stage 2 with the full quadratic form: each shortlisted centroid c is
+ * scored by e^T A e, where e = k - (c + deq(INT2(k - c))) is the Key error
+ * that c would leave and A = fp32(M / n) is the Query second moment in force
+ * (Eq. 7 E[(q^T e)^2] = e^T M e with all of M; evolve.pub review, Strengths:
+ * "full quadratic form gives no consistent gain at higher latency", Table 10).
+ * Folds: y_i = sum_j A_ij e_j over j in order, then sum_i e_i y_i over i in
+ * order, fp32 fused multiply-adds.  Without the flag the diagonal score
+ * sum_g w_g R_g^2 is used.  Appends with the flag run on the CUDA cores. */
+#define QWM_FLAG_QSAC_FULL 1
+
 typedef struct qwm_config {
   int32_t heads;        /* H                                             */
   int32_t head_dim;     /* d                                             */
@@ -73,7 +85,7 @@ typedef struct qwm_config {
   int32_t n_cand;       /* M: QSAC shortlist size                        */
   int32_t rank;         /* r: PSAC rank                                  */
   int32_t max_versions; /* slots for successive bases U (one per refresh) */
-  int32_t reserved;     /* must be 0                                     */
+  int32_t flags;        /* QWM_FLAG_* bits (0: the method as described)   */
   int64_t max_tokens;   /* cache capacity per head                       */
 } qwm_config;
 
@@ -91,8 +103,12 @@ typedef struct qwm_config {
  *   WGROUP    [H][ng]          fp32    w_g = sum of s_j over group g
  *   BASIS     [max_versions][H][d][r] fp32  PSAC bases, slot = version
  *   TOKVER    [Tcap]           uint16  basis version of each cached token
- *   EIGVEC    [H][d][d] + [H]  fp64    eigenvectors of the last refresh, then one
- *                                      warm-start flag per head
+ *   EIGVEC    [H][d][d] + [H]  fp64    refresh state: per head the Ritz vectors
+ *                                      of the last refresh (first 32 columns of d),
+ *                                      then, with QWM_FLAG_QSAC_FULL, A = fp32(M/n)
+ *                                      in force ([d][d] fp32 from double offset
+ *                                      32 d); after all heads one warm-start flag
+ *                                      per head
  *   WORKSPACE                  bytes   scratch for centroid building and basis refresh */
 typedef enum qwm_buffer_id {
   QWM_BUF_K_CODES = 0, QWM_BUF_K_PARAMS, QWM_BUF_K_IDX, QWM_BUF_K_COEF, QWM_BUF_K_CSCALE,

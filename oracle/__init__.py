@@ -67,10 +67,12 @@ def lib():
             "qo_int2_decode": (None, [P, P, I32, I32, P]),
             "qo_qsac_shortlist": (None, [P, P, I32, I32, P, I32, P, P]),
             "qo_qsac_score": (F32, [P, P, P, I32, I32]),
-            "qo_encode_key": (None, [P, P, I32, I32, I32, I32, P, P, P, I32, P, P, P, P, P, P]),
+            "qo_qsac_score_full": (F32, [P, P, P, I32, I32]),
+            "qo_encode_key": (None, [P, P, I32, I32, I32, I32, P, P, P, I32, P, P, P, P, P, P,
+                                     P]),
             "qo_encode_value": (None, [P, P, I32, I32, I32, P, P, P]),
             "qo_append_frame": (None, [I32, I32, I32, I32, I32, I32, I64, I64, P, P, I64, P, P,
-                                       P, P, P, P, P, P, P, P, P, P, P]),
+                                       P, P, P, P, P, P, P, P, P, P, P, P]),
             "qo_reconstruct_key": (None, [P, P, P, P, U16, P, I32, I32, I32, P, P]),
             "qo_reconstruct_value": (None, [P, P, P, I32, I32, P]),
             "qo_reconstruct_head": (None, [I32, I32, I32, I32, I32, I32, I64, I64, P, P, P, P,
@@ -190,8 +192,9 @@ def qsac_score(k, c, w, G) -> float:
     return float(lib().qo_qsac_score(_p(k), _p(c), _p(w), k.shape[0], G))
 
 
-def encode_key(k, CK, G, M, s, w, U):
-    """One key row -> dict(idx, codes, params, coef, cscale, shortlist)."""
+def encode_key(k, CK, G, M, s, w, U, Afull=None):
+    """One key row -> dict(idx, codes, params, coef, cscale, shortlist).  With
+    Afull ([d][d] fp32) QSAC stage 2 scores by the full quadratic form."""
     k = np.ascontiguousarray(k, np.uint16); CK = np.ascontiguousarray(CK, np.uint16)
     s = np.ascontiguousarray(s, np.float32); w = np.ascontiguousarray(w, np.float32)
     U = np.ascontiguousarray(U, np.float32)
@@ -202,10 +205,26 @@ def encode_key(k, CK, G, M, s, w, U):
     idx = np.zeros(1, np.int32); codes = np.zeros(d // 4, np.uint8)
     params = np.zeros(2 * (d // G), np.uint16); coef = np.zeros(max(r, 1), np.int8)
     cs = np.zeros(1, np.uint16); sl = np.zeros(M, np.int32)
+    Af = None if Afull is None else np.ascontiguousarray(Afull, np.float32)
     lib().qo_encode_key(_p(k), _p(CK), C, d, G, M, _p(s), _p(w), _p(U), r, _p(idx), _p(codes),
-                        _p(params), _p(coef), _p(cs), _p(sl))
+                        _p(params), _p(coef), _p(cs), _p(sl), None if Af is None else _p(Af))
     return dict(idx=int(idx[0]), codes=codes, params=params, coef=coef[:r], cscale=int(cs[0]),
                 shortlist=sl)
+
+
+def qsac_score_full(k, c, A, G):
+    """e^T A e for the Key error e that centroid c leaves after INT2 (fp32 folds)."""
+    k = np.ascontiguousarray(k, np.uint16); c = np.ascontiguousarray(c, np.uint16)
+    A = np.ascontiguousarray(A, np.float32)
+    return float(lib().qo_qsac_score_full(_p(k), _p(c), _p(A), k.shape[0], G))
+
+
+def full_quadratic_matrix(M: np.ndarray, n: int) -> np.ndarray:
+    """A = fp32(M / n) (fp64 division, rounded once), the matrix the full-quadratic
+    QSAC score reads; zero before any query."""
+    if n <= 0:
+        return np.zeros(M.shape, np.float32)
+    return (np.asarray(M, np.float64) / float(n)).astype(np.float32)
 
 
 def encode_value(v, CV, G):
@@ -271,8 +290,10 @@ class OracleCache:
     reconstructs a token forever after.
     """
 
-    def __init__(self, H, d, C, G, M, r, Tcap, max_versions=256):
+    def __init__(self, H, d, C, G, M, r, Tcap, max_versions=256, qsac_full=False):
         self.H, self.d, self.C, self.G, self.n_cand, self.r = H, d, C, G, M, r
+        # full-quadratic QSAC: A = fp32(M / n) in force, per head
+        self.A = np.zeros((H, d, d), np.float32) if qsac_full else None
         self.Tcap = int(Tcap)
         ng = d // G
         idt = np.uint8 if C <= 256 else np.uint16
@@ -316,13 +337,17 @@ class OracleCache:
             for h in range(self.H):
                 s, w, Uh, _ = refresh(self.M[h], self.nq, self.r, self.G)
                 self.s[h], self.w[h] = s, w
+                if self.A is not None:
+                    self.A[h] = full_quadratic_matrix(self.M[h], self.nq)
                 if self.r:
                     U[h] = Uh
             self.U.append(U)
 
-    def set_state(self, s=None, w=None, U=None, CK=None, CV=None):
-        """Install state produced elsewhere (e.g. by the GPU) so that encodings can
-        be compared bit for bit with the same inputs."""
+    def set_state(self, s=None, w=None, U=None, CK=None, CV=None, A=None):
+        """Install a state: the tests install the oracle's own refresh and k-means
+        results computed outside this object."""
+        if A is not None:
+            self.A = np.ascontiguousarray(A, np.float32)
         if s is not None:
             self.s = np.ascontiguousarray(s, np.float32)
         if w is not None:
@@ -345,7 +370,8 @@ class OracleCache:
                               self.len, _p(K), _p(V), n, _p(self.CK), _p(self.CV), _p(self.s),
                               _p(self.w), _p(U), _p(self.k_codes), _p(self.k_params),
                               _p(self.k_idx), _p(self.k_coef), _p(self.k_cscale),
-                              _p(self.v_codes), _p(self.v_params), _p(self.v_idx))
+                              _p(self.v_codes), _p(self.v_params), _p(self.v_idx),
+                              None if self.A is None else _p(self.A))
         self.tok_ver[self.len:self.len + n] = self.version
         self.len += n
 

@@ -422,6 +422,28 @@ QO_API float qo_qsac_score(const uint16_t* k, const uint16_t* c, const float* w,
   return acc;
 }
 
+/* QSAC stage 2 with the full quadratic form (Eq. 7 with all of M; evolve.pub
+ * review, Strengths, Table 10): the Key error the candidate c leaves after
+ * INT2, e = k - (c + deq(INT2(k - c))), scored as e^T A e with A = fp32(M / n)
+ * [d][d] in force; y_i = fold_j fmaf(A_ij, e_j), then fold_i fmaf(e_i, y_i). */
+QO_API float qo_qsac_score_full(const uint16_t* k, const uint16_t* c, const float* A, int d,
+                                int G) {
+  float rho[512] = {0.0f}, deq[512], e[512];
+  uint8_t codes[128];
+  uint16_t params[64];
+  for (int j = 0; j < d; ++j) rho[j] = bf(k[j]) - bf(c[j]);
+  qo_int2_encode(rho, d, G, codes, params);
+  qo_int2_decode(codes, params, d, G, deq);
+  for (int j = 0; j < d; ++j) e[j] = bf(k[j]) - (bf(c[j]) + deq[j]);
+  float score = 0.0f;
+  for (int i = 0; i < d; ++i) {
+    float y = 0.0f;
+    for (int j = 0; j < d; ++j) y = fmaf(A[(size_t)i * d + j], e[j], y);
+    score = fmaf(e[i], y, score);
+  }
+  return score;
+}
+
 /* full key encoding for one token-head.
  * PSAC [SP-en, PSAC; REV, Summary]: e = k - K_hat with K_hat = C[a] + deq(rho);
  * c_r = fold_j fmaf(U_jr, e_j, acc); cs = fp16_RU(max_r |c_r| / 127);
@@ -429,14 +451,19 @@ QO_API float qo_qsac_score(const uint16_t* k, const uint16_t* c, const float* w,
 QO_API void qo_encode_key(const uint16_t* k, const uint16_t* CK, int C, int d, int G, int M,
                           const float* s, const float* w, const float* U, int r,
                           int32_t* idx, uint8_t* codes, uint16_t* params, int8_t* coef,
-                          uint16_t* cscale, int32_t* shortlist_out) {
+                          uint16_t* cscale, int32_t* shortlist_out, const float* Afull) {
   int32_t cand[64];
   qo_qsac_shortlist(k, CK, C, d, s, M, cand, NULL);
   int best = 0;
-  float bscore = qo_qsac_score(k, CK + (size_t)cand[0] * d, w, d, G);
-  for (int m = 1; m < M; ++m) {
-    float sc = qo_qsac_score(k, CK + (size_t)cand[m] * d, w, d, G);
-    if (sc < bscore) { bscore = sc; best = m; }
+  /* stage 2 only ranks a shortlist of two or more */
+  if (M > 1) {
+    float bscore = Afull ? qo_qsac_score_full(k, CK + (size_t)cand[0] * d, Afull, d, G)
+                         : qo_qsac_score(k, CK + (size_t)cand[0] * d, w, d, G);
+    for (int m = 1; m < M; ++m) {
+      float sc = Afull ? qo_qsac_score_full(k, CK + (size_t)cand[m] * d, Afull, d, G)
+                       : qo_qsac_score(k, CK + (size_t)cand[m] * d, w, d, G);
+      if (sc < bscore) { bscore = sc; best = m; }
+    }
   }
   int a = cand[best];
   *idx = a;
@@ -502,7 +529,7 @@ QO_API void qo_append_frame(int H, int d, int C, int G, int M, int r, int64_t Tc
                             const float* w, const float* U,
                             uint8_t* k_codes, uint16_t* k_params, void* k_idx, int8_t* k_coef,
                             uint16_t* k_cscale, uint8_t* v_codes, uint16_t* v_params,
-                            void* v_idx) {
+                            void* v_idx, const float* Afull) {
   int ng = d / G;
   for (int h = 0; h < H; ++h) {
     const uint16_t* ck = CK + (size_t)h * C * d;
@@ -513,7 +540,7 @@ QO_API void qo_append_frame(int H, int d, int C, int G, int M, int r, int64_t Tc
       qo_encode_key(K + ((size_t)t * H + h) * d, ck, C, d, G, M, s + (size_t)h * d,
                     w + (size_t)h * ng, U + (size_t)h * d * r, r, &ia,
                     k_codes + slot * (d / 4), k_params + slot * ng * 2, k_coef + slot * r,
-                    k_cscale + slot, NULL);
+                    k_cscale + slot, NULL, Afull ? Afull + (size_t)h * d * d : NULL);
       qo_encode_value(V + ((size_t)t * H + h) * d, cv, C, d, G, &ib,
                       v_codes + slot * (d / 4), v_params + slot * ng * 2);
       if (C <= 256) {

@@ -31,9 +31,18 @@ def test_library_exports_every_declared_symbol():
 
 def _cfg(**kw):
     base = dict(heads=40, head_dim=128, n_centroids=256, group=32, n_cand=4, rank=8,
-                max_versions=64, reserved=0, max_tokens=37440)
+                max_versions=64, flags=0, max_tokens=37440)
     base.update(kw)
     return q.qwm_config(**base)
+
+
+def test_full_quadratic_flag_accepted():
+    out = q.qwm_sizes()
+    assert q.lib().qwm_cache_sizes(ctypes.byref(_cfg(flags=q.QWM_FLAG_QSAC_FULL)),
+                                   ctypes.byref(out)) == 0
+    # the fp32 snapshot of M / n fits after 32 Ritz columns in each head's fp64 block
+    for d in (64, 128):
+        assert 32 * d * 8 + d * d * 4 <= d * d * 8
 
 
 def test_sizes_follow_layout():
@@ -52,7 +61,7 @@ def test_sizes_follow_layout():
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(group=8), dict(n_centroids=0),
                                  dict(n_centroids=513), dict(n_cand=9), dict(n_cand=300),
-                                 dict(rank=17), dict(max_versions=0), dict(reserved=1),
+                                 dict(rank=17), dict(max_versions=0), dict(flags=2), dict(flags=-1),
                                  dict(max_tokens=0), dict(heads=0)])
 def test_invalid_configs_rejected(bad):
     out = q.qwm_sizes()

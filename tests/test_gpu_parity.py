@@ -103,6 +103,55 @@ def test_qvg_mode_without_statistics():
         assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (d, err.max(), err.mean())
 
 
+@pytest.mark.parametrize("d,C,G,M,r", [(128, 64, 32, 4, 8), (64, 16, 16, 4, 4)])
+def test_full_quadratic_qsac(d, C, G, M, r):
+    """QSAC stage 2 by e^T A e (the full-quadratic option, CUDA-core append): the
+    GPU's snapshot A = fp32(M / n) equals the oracle's bit for bit, and every
+    packed field matches the oracle's encoding with the same option."""
+    q = pytest.importorskip("bit_kv_cache_23_b200")
+    H, n, F = 2, 300, 3
+    g = q.QuantKVCache(H, d, C, G, M, r, F * n, max_versions=F + 2, qsac_full=True)
+    oc = oracle.OracleCache(H, d, C, G, M, r, F * n, qsac_full=True)
+    rng = np.random.default_rng(5000 + d)
+    w = np.ones(d)
+    w[rng.permutation(d)[:4]] = 6.0
+    basis = np.linalg.qr(rng.standard_normal((d, 8)))[0]
+    Mref = {h: np.zeros((d, d)) for h in range(H)}
+    rep = new_state_report()
+    for f in range(F):
+        K = syn.f32_to_bf16_bits(((rng.standard_normal((n, H, d)) + 0.3 * rng.standard_normal(d))
+                                  * w).astype(np.float32))
+        V = syn.f32_to_bf16_bits(rng.standard_normal((n, H, d)).astype(np.float32))
+        Q = syn.f32_to_bf16_bits((3.0 * rng.standard_normal((n, H, 8)) @ basis.T
+                                  + 0.5 * rng.standard_normal((n, H, d))).astype(np.float32))
+        if f == 0:
+            g.build_centroids(to_dev(K), to_dev(V), iters=3)
+            oc.set_state(CK=np.stack([oracle.kmeans(K[:, h, :], C, 3)[0] for h in range(H)]),
+                         CV=np.stack([oracle.kmeans(V[:, h, :], C, 3)[0] for h in range(H)]))
+        g.update_query_stats(to_dev(Q), refresh_basis=True)
+        for h in range(H):
+            oracle.stats_accumulate(Q[:, h, :], Mref[h])
+        st = refresh_from_oracle(g, Mref, n * (f + 1), range(H), r, G, rep, check_basis=False)
+        s, wg, U = stack_state(st, H)
+        A = np.stack([oracle.full_quadratic_matrix(Mref[h], n * (f + 1)) for h in range(H)])
+        eig = g.view("eigvec").cpu().numpy()
+        for h in range(H):
+            blk = eig[h * d * d:(h + 1) * d * d].view(np.float32)[64 * d:64 * d + d * d]
+            assert np.array_equal(blk.view(np.uint32), A[h].reshape(-1).view(np.uint32)), (f, h)
+        oc.set_state(s=s, w=wg, U=U, A=A)
+        t0 = g.len
+        g.append_kv(to_dev(K), to_dev(V))
+        oc.append_kv(K, V)
+        assert compare_packed(g, oc, t0, g.len) == {}, f
+    assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
+    O = g.attention(to_dev(Q))
+    torch.cuda.synchronize()
+    assert q.qwm_device_status() == 0
+    Oref = oc.attention(Q)
+    err = np.abs(syn.bf16_bits_to_f32(u16(O)) - Oref)
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
+
+
 def test_degenerate_inputs():
     """Constant keys (zero residual groups), repeated tokens, one-token appends,
     a ragged tail and zero-variance channels."""

@@ -240,6 +240,66 @@ def test_stats_and_basis_match_planted_query_subspace():
         assert abs(np.mean((qf @ e) ** 2) - e @ Mf @ e) < 1e-9 * (e @ Mf @ e)
 
 
+def _int2_error(k, c, G):
+    """Key error e = k - (c + deq(INT2(k - c))) in fp64, from the pinned INT2 codec."""
+    kf = syn.bf16_bits_to_f32(k).astype(np.float64)
+    cf = syn.bf16_bits_to_f32(c).astype(np.float64)
+    rho = (syn.bf16_bits_to_f32(k) - syn.bf16_bits_to_f32(c)).astype(np.float32)
+    codes, params = oracle.int2_encode(rho, G)
+    deq = oracle.int2_decode(codes, params, k.shape[0], G).astype(np.float64)
+    return kf - (cf + deq)
+
+
+def test_full_quadratic_score_is_mean_squared_logit_error():
+    """Eq. 7 with all of M: for A = (sum_t q_t q_t^T) / n the score equals the mean
+    of (q_t . e)^2 over the same queries (exact identity; fp32 rounding only).
+    With A = I it is |e|^2, with a rank-one A = q q^T it is (q . e)^2."""
+    rng = np.random.default_rng(21)
+    d, G, n = 64, 16, 300
+    basis = np.linalg.qr(rng.standard_normal((d, 4)))[0]
+    Q = _bf(3.0 * rng.standard_normal((n, 4)) @ basis.T + 0.3 * rng.standard_normal((n, d)))
+    M = np.zeros((d, d))
+    oracle.stats_accumulate(Q, M)
+    A = oracle.full_quadratic_matrix(M, n)
+    qf = syn.bf16_bits_to_f32(Q).astype(np.float64)
+    for _ in range(20):
+        k = _bf(rng.standard_normal(d) * 1.5)
+        c = _bf(rng.standard_normal(d))
+        e = _int2_error(k, c, G)
+        ref = np.mean((qf @ e) ** 2)
+        assert abs(oracle.qsac_score_full(k, c, A, G) - ref) <= 1e-4 * ref
+        assert abs(oracle.qsac_score_full(k, c, np.eye(d, dtype=np.float32), G) - e @ e) \
+            <= 1e-5 * (e @ e)
+        q1 = qf[0].astype(np.float32)
+        A1 = np.outer(q1, q1).astype(np.float32)
+        assert abs(oracle.qsac_score_full(k, c, A1, G) - (q1.astype(np.float64) @ e) ** 2) \
+            <= 1e-4 * (np.abs(q1) @ np.abs(e)) ** 2
+    assert np.array_equal(oracle.full_quadratic_matrix(M, 0), np.zeros((d, d), np.float32))
+
+
+def test_full_quadratic_choice_minimizes_its_score():
+    """With the full-quadratic option the chosen centroid is the shortlist member
+    with the smallest e^T A e (ties to the earlier position), and the shortlist
+    itself (stage 1) is unchanged."""
+    rng = np.random.default_rng(22)
+    d, G, C, Mc = 64, 16, 32, 4
+    CK = _bf(rng.standard_normal((C, d)))
+    s = rng.uniform(0.2, 2.0, d).astype(np.float32)
+    X = rng.standard_normal((d, d))
+    A = (X @ X.T / d).astype(np.float32)
+    U = np.zeros((d, 0), np.float32)
+    changed = 0
+    for _ in range(100):
+        k = _bf(rng.standard_normal(d) * 1.5)
+        diag = oracle.encode_key(k, CK, G, Mc, s, _group_sums(s, G), U)
+        full = oracle.encode_key(k, CK, G, Mc, s, _group_sums(s, G), U, Afull=A)
+        assert np.array_equal(diag["shortlist"], full["shortlist"])
+        scores = [oracle.qsac_score_full(k, CK[i], A, G) for i in full["shortlist"]]
+        assert full["idx"] == full["shortlist"][int(np.argmin(scores))]
+        changed += full["idx"] != diag["idx"]
+    assert changed > 0     # the two scores do disagree on some keys
+
+
 def test_refresh_without_history_is_identity():
     s, w, U, _ = oracle.refresh(np.zeros((64, 64)), 0, 4, 16)
     assert np.all(s == 1.0) and np.all(U == 0.0) and np.all(w == 16.0)
