@@ -109,7 +109,7 @@ def test_full_quadratic_qsac(d, C, G, M, r):
     GPU's snapshot A = fp32(M / n) equals the oracle's bit for bit, and every
     packed field matches the oracle's encoding with the same option."""
     q = pytest.importorskip("bit_kv_cache_23_b200")
-    H, n, F = 2, 300, 3
+    H, n, F = 2, 700, 3
     g = q.QuantKVCache(H, d, C, G, M, r, F * n, max_versions=F + 2, qsac_full=True)
     oc = oracle.OracleCache(H, d, C, G, M, r, F * n, qsac_full=True)
     rng = np.random.default_rng(5000 + d)
@@ -144,10 +144,11 @@ def test_full_quadratic_qsac(d, C, G, M, r):
         oc.append_kv(K, V)
         assert compare_packed(g, oc, t0, g.len) == {}, f
     assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
-    O = g.attention(to_dev(Q))
+    Qa = Q[:200]
+    O = g.attention(to_dev(Qa))
     torch.cuda.synchronize()
     assert q.qwm_device_status() == 0
-    Oref = oc.attention(Q)
+    Oref = oc.attention(Qa)
     err = np.abs(syn.bf16_bits_to_f32(u16(O)) - Oref)
     assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
 
