@@ -363,6 +363,54 @@ def run_ablation(cfg: syn.LayerConfig, device, frames: int) -> list:
     return out
 
 
+# ----------------------------------------------------------------------------- segment
+def run_segment(cfg: syn.LayerConfig, device, reps: int = 10) -> list:
+    """Times attention of the newest frame's queries over (a) the packed history,
+    (b) the packed history followed by the frame's own keys and values as an exact
+    bf16 segment, and (c) the same kernel over all keys as bf16 (an empty cache),
+    which isolates what decoding the packed cache costs.  CUDA events on the
+    launching stream, median of `reps` after 3 warm-ups; every input set is
+    larger than the L2."""
+    import bit_kv_cache_23_b200 as q
+
+    c = cfg
+    wl = Workload(c, device, extra_versions=4)
+    src = wl.src
+    # the frame being generated: the next one, not yet in the cache
+    Qd, Kd, Vd = (dev_bf16(a, device) for a in src.frame(c.frames))
+    Kall = torch.cat([dev_bf16(src.keys(f), device) for f in range(c.frames)] + [Kd], 0)
+    Vall = torch.cat([dev_bf16(src.values(f), device) for f in range(c.frames)] + [Vd], 0)
+    empty = q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank, 16,
+                           device=device)
+    O = torch.empty_like(Qd)
+    T, nseg = wl.cache.len, Kd.shape[0]
+    cases = [
+        ("packed history", T, lambda: wl.cache.attention(Qd, O)),
+        ("packed history + bf16 segment", T + nseg,
+         lambda: wl.cache.attention_ext(Qd, Kd, Vd, O=O)),
+        ("all keys bf16 (no decode)", Kall.shape[0],
+         lambda: empty.attention_ext(Qd, Kall, Vall, O=O)),
+    ]
+    out = []
+    for name, keys, fn in cases:
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(device)
+            ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        flop = 4.0 * c.q_rows * keys * c.head_dim * c.heads
+        out.append({"attention": name, "keys": int(keys), "ms": ms,
+                    "TFLOP_per_s": flop / (ms * 1e-3) / 1e12,
+                    "workload": f"{c.name} layer, {c.q_rows} queries x {c.heads} heads"})
+    return out
+
+
 # ----------------------------------------------------------------------------- oracle arm
 def oracle_throughput(cfg: syn.LayerConfig, cache=None, budget_s: float = 12.0):
     """The CPU oracle, as it stands, on a bounded sample of one step of the
@@ -447,6 +495,9 @@ def main():
     ap.add_argument("--ablation", action="store_true",
                     help="instead of timing, print one JSON line per quantization setting "
                          "(QVG, QSAC only, rank sweep, K-only, V-only) with its quality")
+    ap.add_argument("--segment", action="store_true",
+                    help="instead of the step, time attention over the packed history, over "
+                         "history + the frame's bf16 segment, and over all keys in bf16")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -458,6 +509,14 @@ def main():
                      f"{cfg.frames} latent frames x {cfg.tokens_per_frame} tokens, "
                      f"{cfg.q_rows}-query chunk, C={cfg.n_centroids}, G={cfg.group}, "
                      f"M={cfg.n_cand}, r={cfg.rank}")
+
+    if args.segment:
+        if rank == 0:
+            device = torch.device("cuda", local)
+            torch.cuda.set_device(device)
+            for line in run_segment(cfg, device):
+                print(json.dumps(line), flush=True)
+        return
 
     if args.ablation:
         if rank == 0:
