@@ -140,7 +140,7 @@ class ClockSampler:
 # frames): ncu dram__bytes_read.sum + dram__bytes_write.sum captured at 6 cached
 # frames and scaled to 24 by the packed-cache bytes (see the attention profile
 # summary).  Valid only for the kernel source it was taken on (hash below).
-ATTN_TRAFFIC = {"sha256_16": "eb5354167438f6e5", "config": "480p", "frames": 24,
+ATTN_TRAFFIC = {"sha256_16": "152b87895d45369e", "config": "480p", "frames": 24,
                 "bytes_per_launch": 63.00e6 + 1.66e6 + (161.7e6 - 40.4e6)}
 
 

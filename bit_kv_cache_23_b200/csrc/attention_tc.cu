@@ -17,7 +17,7 @@
 // a key whose version is neither (a tile spanning three versions) is
 // compensated element-wise by its dequant thread instead.
 //
-// One CTA per (head, 256 query rows = two 128-row Q tiles); 576 threads:
+// One CTA per (head, 256 query rows = two 128-row Q tiles); 608 threads:
 //   warps 0-7   softmax: warp w serves Q tile w/4, TMEM lanes 32(w%4)..+31 =
 //               query rows; online softmax in the log2 domain with a lazy
 //               rescale of O, P written back into TMEM over S (bf16 pairs).
@@ -25,18 +25,28 @@
 //               their centroid chunks with 16-byte async copies two tiles
 //               ahead, then rewrite them in place as K-hat / V' (bf16, the
 //               128B-swizzled layouts the UMMA descriptors read).
-//   warp 16     MMA: one thread issues, per key tile and Q tile, S = Q K^T
-//               (+ AX BX^T) and O += P V', alternating the two Q tiles so the
-//               tensor pipe works on one while the softmax works on the other.
-//   warp 17     producer: bulk-copies (TMA engine) the tile's packed codes,
+//   warps 16-17 MMA: one issuing thread per Q tile, S = Q K^T (+ AX BX^T)
+//               then, once the softmax has written P, O += P V'; the two
+//               threads interleave on the tensor pipe, which works on one Q
+//               tile while the softmax works on the other.
+//   warp 18     producer: bulk-copies (TMA engine) the tile's packed codes,
 //               group parameters, coefficients, versions and centroid indices
-//               into the stage, and builds [U_va | U_vb] in bf16 on changes.
+//               into the packed-field ring, and builds [U_va | U_vb] in bf16
+//               on changes.
 // TMEM (512 columns): per Q tile p, Q at 256p (64 columns of bf16 pairs), S/P
-// at 256p+64, O at 256p+128.  Shared memory: a ring of 4 stages of K-hat, V',
-// packed fields and the compensation slab.  Every mbarrier wait is bounded
-// (about 1 s); a timeout sets a device flag that qwm_device_status() reports,
-// every role then leaves its loop, and in-flight copies and MMAs are drained
-// (bounded) before the TMEM is freed.
+// at 256p+64, O at 256p+128.  Shared memory: a ring of 4 K-hat / V' /
+// compensation-slab stages (released by the MMA) and a ring of 5 packed-field
+// stages (released by the dequant).
+//
+// The SEG instance also attends over a bf16 segment after the packed tokens
+// (the frame being generated): its tiles follow the packed ones, and the
+// dequant warps copy their rows into the same swizzled stages instead of
+// decoding; they carry the last packed tile's version pair and zero
+// compensation rows.  An optional output receives ln sum exp of the scores.
+//
+// Every mbarrier wait is bounded (about 1 s); a timeout sets a device flag
+// that qwm_device_status() reports, every role then leaves its loop, and
+// in-flight copies and MMAs are drained (bounded) before the TMEM is freed.
 #include <math.h>
 
 #include "dequant.cuh"
