@@ -18,9 +18,12 @@
 // fold and ranked by (D, i).  A token with more than SURV_MAX survivors is
 // rescored over all C centroids.
 //
-// One CTA per (head, 128 tokens), 128 threads: thread t owns token t and TMEM
-// lane t; the token rows sit in shared memory (16-byte aligned, conflict-free
-// rows).  Thread 0 issues the MMAs.
+// One CTA per (head, NT tokens), NT threads: thread t owns token t and a TMEM
+// lane; the token rows sit in shared memory (16-byte aligned, conflict-free
+// rows).  NT = 256 when C <= 256 (two 128-row MMA halves share one centroid
+// tile, TMEM lanes split by half), else 128.  Thread 0 issues the MMAs.  The
+// candidate threshold comes from the M-th smallest minimum over groups of 8
+// centroids, and survivors are rescored in pairs.
 // After the MMAs the -2c tile stays in shared memory and serves as the
 // centroid table for the exact passes (c = -0.5 * (-2c) is exact), so that the
 // rescoring, the QSAC score, the INT2 codes and the PSAC coefficients read
