@@ -21,7 +21,8 @@
 // One CTA per (head, NT tokens), NT threads: thread t owns token t and a TMEM
 // lane; the token rows sit in shared memory (16-byte aligned, conflict-free
 // rows).  NT = 256 when C <= 256 (two 128-row MMA halves share one centroid
-// tile, TMEM lanes split by half), else 128.  Thread 0 issues the MMAs.  The
+// tile; each half writes its own TMEM column range, token t in lane t % 128),
+// else 128.  Thread 0 issues the MMAs.  The
 // candidate threshold comes from the M-th smallest minimum over groups of 8
 // centroids, and survivors are rescored in pairs.
 // After the MMAs the -2c tile stays in shared memory and serves as the
