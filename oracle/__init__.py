@@ -77,6 +77,8 @@ def lib():
             "qo_reconstruct_value": (None, [P, P, P, I32, I32, P]),
             "qo_reconstruct_head": (None, [I32, I32, I32, I32, I32, I32, I64, I64, P, P, P, P,
                                            P, P, P, P, P, P, P, P, P, P]),
+            "qo_reconstruct_range": (None, [I32, I32, I32, I32, I32, I32, I64, I64, I64, P, P, P,
+                                            P, P, P, P, P, P, P, P, P, P, P]),
             "qo_attention_head": (None, [P, I64, I64, P, P, I64, I32, F64, P]),
             "qo_attention_lse": (None, [P, I64, I64, P, I64, I32, F64, P]),
             "qo_top1": (None, [P, I64, I64, P, I64, I64, I32, P]),
@@ -306,8 +308,10 @@ class OracleCache:
         self.v_params = np.zeros((H, self.Tcap, ng, 2), np.uint16)
         self.v_idx = np.zeros((H, self.Tcap), idt)
         self.tok_ver = np.zeros(self.Tcap, np.uint16)
-        self.CK = None
-        self.CV = None
+        # centroid tables: one (CK, CV) pair per build; each token keeps the
+        # version in force at its append (tok_cver), like the basis versions
+        self.cent_versions = []
+        self.tok_cver = np.zeros(self.Tcap, np.uint16)
         self.M = np.zeros((H, d, d), np.float64)
         self.nq = 0
         self.s = np.ones((H, d), np.float32)
@@ -319,14 +323,51 @@ class OracleCache:
     def version(self):
         return len(self.U) - 1
 
-    def build_centroids(self, K, V, iters=10):
-        """K, V [n][H][d] bf16 bits (frame 0)."""
+    # the tables in force (the latest version)
+    @property
+    def CK(self):
+        return self.cent_versions[-1][0] if self.cent_versions else None
+
+    @CK.setter
+    def CK(self, v):
+        self._set_current(0, v)
+
+    @property
+    def CV(self):
+        return self.cent_versions[-1][1] if self.cent_versions else None
+
+    @CV.setter
+    def CV(self, v):
+        self._set_current(1, v)
+
+    def _set_current(self, i, v):
+        v = np.ascontiguousarray(v, np.uint16)
+        if not self.cent_versions:
+            self.cent_versions.append([None, None])
+        self.cent_versions[-1][i] = v
+
+    @property
+    def cent_version(self):
+        return len(self.cent_versions) - 1
+
+    def _kmeans_tables(self, K, V, iters):
         H, d, C = self.H, self.d, self.C
-        self.CK = np.zeros((H, C, d), np.uint16)
-        self.CV = np.zeros((H, C, d), np.uint16)
+        CK = np.zeros((H, C, d), np.uint16)
+        CV = np.zeros((H, C, d), np.uint16)
         for h in range(H):
-            self.CK[h], _ = kmeans(K[:, h, :], C, iters)
-            self.CV[h], _ = kmeans(V[:, h, :], C, iters)
+            CK[h], _ = kmeans(K[:, h, :], C, iters)
+            CV[h], _ = kmeans(V[:, h, :], C, iters)
+        return CK, CV
+
+    def build_centroids(self, K, V, iters=10):
+        """K, V [n][H][d] bf16 bits (frame 0): the first centroid tables."""
+        self.cent_versions = [list(self._kmeans_tables(K, V, iters))]
+
+    def rebuild_centroids(self, K, V, iters=10):
+        """Centroid refresh under drift: k-means on a recent frame K, V gives a new
+        version of the tables; later appends encode against it, while tokens
+        already cached keep the tables they were encoded with."""
+        self.cent_versions.append(list(self._kmeans_tables(K, V, iters)))
 
     def update_query_stats(self, Q, refresh_basis=True):
         for h in range(self.H):
@@ -355,9 +396,9 @@ class OracleCache:
         if U is not None:
             self.U.append(np.ascontiguousarray(U, np.float32).reshape(self.H, self.d, -1))
         if CK is not None:
-            self.CK = np.ascontiguousarray(CK, np.uint16)
+            self.CK = CK
         if CV is not None:
-            self.CV = np.ascontiguousarray(CV, np.uint16)
+            self.CV = CV
 
     def append_kv(self, K, V):
         n = K.shape[0]
@@ -373,6 +414,7 @@ class OracleCache:
                               _p(self.v_codes), _p(self.v_params), _p(self.v_idx),
                               None if self.A is None else _p(self.A))
         self.tok_ver[self.len:self.len + n] = self.version
+        self.tok_cver[self.len:self.len + n] = self.cent_version
         self.len += n
 
     def reconstruct(self, h):
@@ -383,11 +425,21 @@ class OracleCache:
         r = self.r
         if r == 0:
             Uall = np.zeros((len(self.U), self.H, self.d, 1), np.float32)
-        lib().qo_reconstruct_head(h, self.H, self.d, self.C, self.G, r, self.Tcap, T,
-                                  _p(self.CK), _p(self.CV), _p(Uall), _p(self.tok_ver),
-                                  _p(self.k_codes), _p(self.k_params), _p(self.k_idx),
-                                  _p(self.k_coef), _p(self.k_cscale), _p(self.v_codes),
-                                  _p(self.v_params), _p(self.v_idx), _p(Kp), _p(Vp))
+        # runs of tokens sharing one centroid-table version (versions only grow)
+        t0 = 0
+        while t0 < T:
+            cv = int(self.tok_cver[t0])
+            t1 = t0
+            while t1 < T and self.tok_cver[t1] == cv:
+                t1 += 1
+            CK, CV = self.cent_versions[cv]
+            lib().qo_reconstruct_range(h, self.H, self.d, self.C, self.G, r, self.Tcap, t0, t1,
+                                       _p(CK), _p(CV), _p(Uall), _p(self.tok_ver),
+                                       _p(self.k_codes), _p(self.k_params), _p(self.k_idx),
+                                       _p(self.k_coef), _p(self.k_cscale), _p(self.v_codes),
+                                       _p(self.v_params), _p(self.v_idx), _p(Kp[t0:]),
+                                       _p(Vp[t0:]))
+            t0 = t1
         return Kp, Vp
 
     def attention(self, Q, rows=None, heads=None, scale=None):

@@ -582,6 +582,31 @@ QO_API void qo_reconstruct_value(const uint16_t* c, const uint8_t* codes, const 
 
 /* Reconstruct the whole cache of one head: K', V' [T][d] bf16.
  * U_all [n_versions][H][d][r], tok_ver [Tcap] (version of each token). */
+/* Tokens [t0, t1) of head h (Kp, Vp indexed by t - t0), reconstructed with the
+ * centroid tables CK, CV given (the tables in force when those tokens were
+ * appended). */
+QO_API void qo_reconstruct_range(int h, int H, int d, int C, int G, int r, int64_t Tcap,
+                                 int64_t t0, int64_t t1, const uint16_t* CK, const uint16_t* CV,
+                                 const float* U_all, const uint16_t* tok_ver,
+                                 const uint8_t* k_codes, const uint16_t* k_params,
+                                 const void* k_idx, const int8_t* k_coef,
+                                 const uint16_t* k_cscale, const uint8_t* v_codes,
+                                 const uint16_t* v_params, const void* v_idx, uint16_t* Kp,
+                                 uint16_t* Vp) {
+  int ng = d / G;
+  for (int64_t t = t0; t < t1; ++t) {
+    int64_t slot = (int64_t)h * Tcap + t;
+    int a = (C <= 256) ? ((const uint8_t*)k_idx)[slot] : ((const uint16_t*)k_idx)[slot];
+    int b = (C <= 256) ? ((const uint8_t*)v_idx)[slot] : ((const uint16_t*)v_idx)[slot];
+    const float* U = U_all + ((size_t)tok_ver[t] * H + h) * d * r;
+    qo_reconstruct_key(CK + ((size_t)h * C + a) * d, k_codes + slot * (d / 4),
+                       k_params + slot * ng * 2, k_coef + slot * r, k_cscale[slot], U, d, G, r,
+                       Kp + (size_t)(t - t0) * d, NULL);
+    qo_reconstruct_value(CV + ((size_t)h * C + b) * d, v_codes + slot * (d / 4),
+                         v_params + slot * ng * 2, d, G, Vp + (size_t)(t - t0) * d);
+  }
+}
+
 QO_API void qo_reconstruct_head(int h, int H, int d, int C, int G, int r, int64_t Tcap, int64_t T,
                                 const uint16_t* CK, const uint16_t* CV, const float* U_all,
                                 const uint16_t* tok_ver, const uint8_t* k_codes,

@@ -459,3 +459,84 @@ def test_packed_bytes_follow_compression_formula():
     assert oc.packed_bytes() == per * c.heads * oc.len
     for (d, C, G, r, want) in [(128, 256, 32, 8, 108), (128, 512, 32, 8, 110)]:
         assert oracle.bytes_per_token_head(d, C, G, r) == want
+
+
+# ----------------------------------------------------------------------------- centroid refresh
+def _drift_cache(rebuild_every, frames=12, n=192, sigma=0.4, seed=31):
+    import dataclasses
+    c = dataclasses.replace(syn.get_config("1min"), heads=1, tokens_per_frame=n, q_rows=n,
+                            frames=frames, n_centroids=32, drift_sigma=sigma)
+    src = syn.FrameSource(c, seed)
+    oc = oracle.OracleCache(1, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank,
+                            frames * n)
+    Ks = []
+    for f in range(frames):
+        Q, K, V = src.frame(f)
+        if f == 0:
+            oc.build_centroids(K, V, iters=5)
+        elif rebuild_every and f % rebuild_every == 0:
+            oc.rebuild_centroids(K, V, iters=5)
+        oc.update_query_stats(Q, refresh_basis=True)
+        oc.append_kv(K, V)
+        Ks.append(K[:, 0, :])
+    return oc, np.concatenate(Ks), n
+
+
+def test_ranged_reconstruction_equals_whole_head():
+    """One table version: the per-run reconstruction equals the whole-head routine."""
+    oc, _, _ = _drift_cache(0, frames=3)
+    Kp, Vp = oc.reconstruct(0)
+    T = oc.len
+    Kh = np.zeros((T, oc.d), np.uint16); Vh = np.zeros((T, oc.d), np.uint16)
+    Uall = np.ascontiguousarray(np.stack(oc.U), np.float32)
+    P = oracle._p
+    oracle.lib().qo_reconstruct_head(0, 1, oc.d, oc.C, oc.G, oc.r, oc.Tcap, T, P(oc.CK), P(oc.CV),
+                                     P(Uall), P(oc.tok_ver), P(oc.k_codes), P(oc.k_params),
+                                     P(oc.k_idx), P(oc.k_coef), P(oc.k_cscale), P(oc.v_codes),
+                                     P(oc.v_params), P(oc.v_idx), P(Kh), P(Vh))
+    assert np.array_equal(Kp, Kh) and np.array_equal(Vp, Vh)
+
+
+def test_centroid_rebuild_keeps_old_tokens():
+    """Tokens appended before a centroid rebuild reconstruct bit for bit as before."""
+    import dataclasses
+    c = dataclasses.replace(syn.get_config("1min"), heads=1, tokens_per_frame=160, q_rows=160,
+                            frames=4, n_centroids=32, drift_sigma=0.4)
+    src = syn.FrameSource(c, 5)
+    oc = oracle.OracleCache(1, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank, 4 * 160)
+    for f in range(2):
+        Q, K, V = src.frame(f)
+        if f == 0:
+            oc.build_centroids(K, V, iters=4)
+        oc.update_query_stats(Q, True)
+        oc.append_kv(K, V)
+    before = oc.reconstruct(0)
+    Q, K, V = src.frame(2)
+    oc.rebuild_centroids(K, V, iters=4)
+    assert oc.cent_version == 1 and not np.array_equal(oc.cent_versions[0][0], oc.CK)
+    oc.update_query_stats(Q, True)
+    oc.append_kv(K, V)
+    after = oc.reconstruct(0)
+    assert np.array_equal(after[0][:320], before[0]) and np.array_equal(after[1][:320], before[1])
+    assert np.all(oc.tok_cver[:320] == 0) and np.all(oc.tok_cver[320:480] == 1)
+    # rebuilding from the first frame's data gives the first tables again (determinism)
+    _, K0, V0 = src.frame(0)
+    oc.rebuild_centroids(K0, V0, iters=4)
+    assert np.array_equal(oc.CK, oc.cent_versions[0][0])
+    assert np.array_equal(oc.CV, oc.cent_versions[0][1])
+
+
+def test_centroid_rebuild_tracks_key_drift():
+    """Under a drifting Key mean, tables rebuilt every 4 frames from the newest
+    frame leave a smaller reconstruction error on the late frames than the
+    frame-0 tables do."""
+    stale, K, n = _drift_cache(0)
+    fresh, _, _ = _drift_cache(4)
+    kf = syn.bf16_bits_to_f32(K).astype(np.float64)
+    late = slice(len(kf) - 4 * n, len(kf))
+    err = {}
+    for name, oc in (("stale", stale), ("fresh", fresh)):
+        Kp, _ = oc.reconstruct(0)
+        err[name] = float(np.mean((syn.bf16_bits_to_f32(Kp).astype(np.float64)[late] - kf[late]) ** 2))
+    assert err["fresh"] < 0.9 * err["stale"], err
+
