@@ -22,17 +22,18 @@ __all__ = [
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
     "qwm_build_centroids", "qwm_build_centroids_noalloc", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
     "qwm_attention_ext", "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
-    "QWM_FLAG_QSAC_FULL",
+    "QWM_FLAG_QSAC_FULL", "QWM_NOALLOC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqwm.so")
 
 QWM_FLAG_QSAC_FULL = 1   # QSAC stage 2 by the full quadratic form e^T A e
+QWM_NOALLOC_SCRATCH_BYTES = 16 << 20   # fixed scratch of qwm_build_centroids_noalloc
 
 BUFFER_NAMES = ["k_codes", "k_params", "k_idx", "k_coef", "k_cscale", "v_codes", "v_params",
                 "v_idx", "cent_k", "cent_v", "qstats", "sens", "wgroup", "basis", "tokver",
-                "eigvec", "workspace"]
+                "centver", "eigvec", "workspace"]
 NBUF = len(BUFFER_NAMES)
 
 STATUS = {0: "QWM_OK", 1: "QWM_ERR_INVALID_ARG", 2: "QWM_ERR_ALIGNMENT", 3: "QWM_ERR_CAPACITY",
@@ -44,7 +45,7 @@ class qwm_config(ctypes.Structure):
                 ("n_centroids", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("n_cand", ctypes.c_int32), ("rank", ctypes.c_int32),
                 ("max_versions", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("max_tokens", ctypes.c_int64)]
+                ("max_cent_versions", ctypes.c_int32), ("max_tokens", ctypes.c_int64)]
 
 
 class qwm_sizes(ctypes.Structure):
@@ -61,7 +62,8 @@ class qwm_cache(ctypes.Structure):
                 ("len", ctypes.c_int64), ("n_queries", ctypes.c_int64),
                 ("frames", ctypes.c_int32), ("n_versions", ctypes.c_int32),
                 ("cur_version", ctypes.c_int32), ("has_centroids", ctypes.c_int32),
-                ("has_eigvec", ctypes.c_int32), ("magic", ctypes.c_int32)]
+                ("has_eigvec", ctypes.c_int32), ("magic", ctypes.c_int32),
+                ("n_cent_versions", ctypes.c_int32), ("cur_cent_version", ctypes.c_int32)]
 
 
 class QwmError(RuntimeError):
@@ -249,13 +251,13 @@ class QuantKVCache:
 
     def __init__(self, heads: int, head_dim: int, n_centroids: int, group: int, n_cand: int,
                  rank: int, max_tokens: int, max_versions: int = 1024, device="cuda",
-                 stream=None, qsac_full: bool = False):
+                 stream=None, qsac_full: bool = False, max_cent_versions: int = 1):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("QuantKVCache lives on a CUDA device")
         flags = QWM_FLAG_QSAC_FULL if qsac_full else 0
         self.cfg = qwm_config(heads, head_dim, n_centroids, group, n_cand, rank, max_versions,
-                              flags, max_tokens)
+                              flags, max_cent_versions, max_tokens)
         self.sizes = qwm_cache_sizes(self.cfg)
         self.buffers = {}
         bufs = qwm_buffers()
@@ -281,6 +283,10 @@ class QuantKVCache:
     def version(self) -> int:
         return int(self.c.cur_version)
 
+    @property
+    def cent_version(self) -> int:
+        return int(self.c.cur_cent_version)
+
     def build_centroids(self, K, V, iters=10, stream=None):
         qwm_build_centroids(self.c, K, V, iters, stream)
 
@@ -304,10 +310,17 @@ class QuantKVCache:
     def top1_shift(self, Q, K_exact, stream=None):
         return qwm_top1_shift(self.c, Q, K_exact, stream)
 
-    # typed views of the packed buffers (for inspection and tests)
-    def view(self, name: str) -> torch.Tensor:
+    # typed views of the packed buffers (for inspection and tests); the centroid
+    # tables are those of `cent_version` (default: the version in force)
+    def view(self, name: str, cent_version: int | None = None) -> torch.Tensor:
         H, d, C, G, r = (self.cfg.heads, self.cfg.head_dim, self.cfg.n_centroids,
                          self.cfg.group, self.cfg.rank)
+        if name in ("cent_k", "cent_v"):
+            cv = self.cent_version if cent_version is None else int(cent_version)
+            if not 0 <= cv < self.cfg.max_cent_versions:
+                raise IndexError(f"centroid-table version {cv} out of range")
+            n = H * C * d
+            return self.buffers[name][2 * n * cv:2 * n * (cv + 1)].view(torch.int16).view(H, C, d)
         T, ng = self.tcap, d // G
         b = self.buffers[name]
         idt = torch.uint8 if C <= 256 else torch.int16
@@ -316,9 +329,9 @@ class QuantKVCache:
             "k_params": (torch.int16, (H, T, ng, 2)), "v_params": (torch.int16, (H, T, ng, 2)),
             "k_idx": (idt, (H, T)), "v_idx": (idt, (H, T)),
             "k_coef": (torch.int8, (H, T, r)), "k_cscale": (torch.int16, (H, T)),
-            "cent_k": (torch.int16, (H, C, d)), "cent_v": (torch.int16, (H, C, d)),
             "qstats": (torch.float64, (H, d, d)), "sens": (torch.float32, (H, d)),
             "wgroup": (torch.float32, (H, ng)), "tokver": (torch.int16, (T,)),
+            "centver": (torch.int16, (T,)),
             "basis": (torch.float32, (self.cfg.max_versions, H, d, max(r, 1))),
             "eigvec": (torch.float64, (H * d * d + H,)),
         }

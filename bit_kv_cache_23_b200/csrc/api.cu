@@ -8,41 +8,7 @@ using namespace qwm;
 
 namespace {
 
-constexpr int32_t kMagic = 0x51574d31;  // "QWM1"
-
-bool config_ok(const qwm_config* c) {
-  if (!c) return false;
-  if (c->heads < 1 || c->heads > 4096) return false;
-  if (c->head_dim != 64 && c->head_dim != 128) return false;
-  if (c->group != 16 && c->group != 32) return false;
-  if (c->head_dim % c->group) return false;
-  if (c->n_centroids < 1 || c->n_centroids > 512) return false;
-  if (c->n_cand < 1 || c->n_cand > 8 || c->n_cand > c->n_centroids) return false;
-  if (c->rank < 0 || c->rank > 16) return false;
-  if (c->max_versions < 1 || c->max_versions > 65535) return false;
-  if ((c->flags & ~QWM_FLAG_QSAC_FULL) != 0) return false;
-  if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 40)) return false;
-  return true;
-}
-
-Dims dims_of(const qwm_config* c) {
-  Dims D;
-  D.H = c->heads;
-  D.d = c->head_dim;
-  D.C = c->n_centroids;
-  D.G = c->group;
-  D.M = c->n_cand;
-  D.r = c->rank;
-  D.ng = c->head_dim / c->group;
-  D.tcap = (c->max_tokens + 127) / 128 * 128;
-  D.idx_bytes = c->n_centroids <= 256 ? 1 : 2;
-  D.qsac_full = (c->flags & QWM_FLAG_QSAC_FULL) ? 1 : 0;
-  return D;
-}
-
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
-
-bool cache_ok(const qwm_cache* c) { return c && c->magic == kMagic && config_ok(&c->cfg); }
 
 qwm_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return QWM_OK;
@@ -83,13 +49,14 @@ qwm_status qwm_cache_sizes(const qwm_config* cfg, qwm_sizes* out) {
   out->bytes[QWM_BUF_V_CODES] = HT * (D.d / 4);
   out->bytes[QWM_BUF_V_PARAMS] = HT * D.ng * 4;
   out->bytes[QWM_BUF_V_IDX] = HT * D.idx_bytes;
-  out->bytes[QWM_BUF_CENT_K] = (uint64_t)D.H * D.C * D.d * 2;
-  out->bytes[QWM_BUF_CENT_V] = (uint64_t)D.H * D.C * D.d * 2;
+  out->bytes[QWM_BUF_CENT_K] = (uint64_t)cfg->max_cent_versions * cent_slot_elems(D) * 2;
+  out->bytes[QWM_BUF_CENT_V] = (uint64_t)cfg->max_cent_versions * cent_slot_elems(D) * 2;
   out->bytes[QWM_BUF_QSTATS] = (uint64_t)D.H * D.d * D.d * 8;
   out->bytes[QWM_BUF_SENS] = (uint64_t)D.H * D.d * 4;
   out->bytes[QWM_BUF_WGROUP] = (uint64_t)D.H * D.ng * 4;
   out->bytes[QWM_BUF_BASIS] = (uint64_t)cfg->max_versions * D.H * D.d * (D.r > 0 ? D.r : 1) * 4;
   out->bytes[QWM_BUF_TOKVER] = (uint64_t)D.tcap * 2;
+  out->bytes[QWM_BUF_CENTVER] = (uint64_t)D.tcap * 2;
   out->bytes[QWM_BUF_EIGVEC] = (uint64_t)D.H * D.d * D.d * 8 + (uint64_t)D.H * 8;
   out->bytes[QWM_BUF_WORKSPACE] = kmeans_workspace_bytes(D);
   out->bytes_per_token_head = 2 * (D.d / 4 + 4 * D.ng + D.idx_bytes) + D.r + 2;
@@ -113,7 +80,9 @@ qwm_status qwm_cache_init(qwm_cache* c, const qwm_config* cfg, const qwm_buffers
   tmp.tcap = D.tcap;
   tmp.n_versions = 1;
   tmp.cur_version = 0;
-  tmp.magic = kMagic;
+  tmp.n_cent_versions = 0;
+  tmp.cur_cent_version = 0;
+  tmp.magic = kCacheMagic;
   CacheView v = view_of(&tmp);
   cudaError_t e = launch_init_state(D, v, (cudaStream_t)stream);
   if (e != cudaSuccess) return QWM_ERR_CUDA;
@@ -123,16 +92,18 @@ qwm_status qwm_cache_init(qwm_cache* c, const qwm_config* cfg, const qwm_buffers
 
 qwm_status qwm_build_centroids(qwm_cache* c, const void* K, const void* V, int64_t n,
                                int32_t iters, void* stream) {
-  if (!cache_ok(c) || !K || !V) return QWM_ERR_INVALID_ARG;
-  if (!aligned(K, 16) || !aligned(V, 16)) return QWM_ERR_ALIGNMENT;
+  int slot = 0;
+  const qwm_status st = centroid_build_slot(c, K, V, n, iters, &slot);
+  if (st != QWM_OK) return st;
   Dims D = dims_of(&c->cfg);
-  if (n < D.C || n > D.tcap || iters < 1 || iters > 1000) return QWM_ERR_INVALID_ARG;
   CacheView v = view_of(c);
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_kmeans(D, (const uint16_t*)K, n, iters, v.cent_k, v.workspace, s);
-  if (e == cudaSuccess) e = launch_kmeans(D, (const uint16_t*)V, n, iters, v.cent_v, v.workspace, s);
+  const size_t off = (size_t)slot * cent_slot_elems(D);
+  cudaError_t e = launch_kmeans(D, (const uint16_t*)K, n, iters, v.cent_k + off, v.workspace, s);
+  if (e == cudaSuccess)
+    e = launch_kmeans(D, (const uint16_t*)V, n, iters, v.cent_v + off, v.workspace, s);
   if (e != cudaSuccess) return QWM_ERR_CUDA;
-  c->has_centroids = 1;
+  centroid_build_commit(c, slot);
   return QWM_OK;
 }
 
@@ -168,7 +139,7 @@ qwm_status qwm_append_kv(qwm_cache* c, const void* K, const void* V, int64_t n, 
   Dims D = dims_of(&c->cfg);
   CacheView v = view_of(c);
   cudaError_t e = launch_append(D, v, (const uint16_t*)K, (const uint16_t*)V, n, c->len,
-                                c->cur_version, (cudaStream_t)stream);
+                                c->cur_version, c->cur_cent_version, (cudaStream_t)stream);
   if (e != cudaSuccess) return QWM_ERR_CUDA;
   c->len += n;
   c->frames += 1;

@@ -52,9 +52,10 @@ struct AppendArgs {
   int8_t* coef;           // [H][tcap][r]  (keys)
   uint16_t* cscale;       // [H][tcap]     (keys)
   uint16_t* tokver;       // [tcap]        (keys)
+  uint16_t* centver;      // [tcap]        (keys)
   double* eigvec;         // refresh state holding A = fp32(M / n) per head (full-quadratic)
   int64_t n, t0, tcap;
-  int H, C, G, M, r, idx_bytes, version, qfull;
+  int H, C, G, M, r, idx_bytes, version, cver, qfull;
 };
 
 __device__ __forceinline__ bool lex_less(float a, int ia, float b, int ib) {
@@ -264,7 +265,10 @@ __global__ void __launch_bounds__(NT) append_kernel(AppendArgs A) {
       if (lane == 0) {
         if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
         else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
-        if (KEY && h == 0) A.tokver[A.t0 + t] = (uint16_t)A.version;
+        if (KEY && h == 0) {
+          A.tokver[A.t0 + t] = (uint16_t)A.version;
+          A.centver[A.t0 + t] = (uint16_t)A.cver;
+        }
       }
       if (KEY) {
         float* ew = es + warp * D;
@@ -317,17 +321,19 @@ cudaError_t run(const AppendArgs& a, cudaStream_t s) {
 
 cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_t* K,
                                const uint16_t* V, int64_t n, int64_t t0, int version,
-                               cudaStream_t s);
+                               int cent_version, cudaStream_t s);
 
 cudaError_t launch_append(const Dims& Dm, const CacheView& v, const uint16_t* K, const uint16_t* V,
-                          int64_t n, int64_t t0, int version, cudaStream_t s) {
-  if (append_tc_supported(Dm)) return launch_append_tc(Dm, v, K, V, n, t0, version, s);
-  return launch_append_simt(Dm, v, K, V, n, t0, version, s);
+                          int64_t n, int64_t t0, int version, int cent_version, cudaStream_t s) {
+  if (append_tc_supported(Dm))
+    return launch_append_tc(Dm, v, K, V, n, t0, version, cent_version, s);
+  return launch_append_simt(Dm, v, K, V, n, t0, version, cent_version, s);
 }
 
 cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_t* K,
                                const uint16_t* V, int64_t n, int64_t t0, int version,
-                               cudaStream_t s) {
+                               int cent_version, cudaStream_t s) {
+  const size_t coff = (size_t)cent_version * cent_slot_elems(Dm);
   AppendArgs a{};
   a.n = n;
   a.t0 = t0;
@@ -339,9 +345,10 @@ cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_
   a.r = Dm.r;
   a.idx_bytes = Dm.idx_bytes;
   a.version = version;
+  a.cver = cent_version;
   // keys
   a.X = K;
-  a.cent = v.cent_k;
+  a.cent = v.cent_k + coff;
   a.sens = v.sens;
   a.wgroup = v.wgroup;
   a.basis = v.basis + (size_t)version * Dm.H * Dm.d * (Dm.r > 0 ? Dm.r : 1);
@@ -351,13 +358,14 @@ cudaError_t launch_append_simt(const Dims& Dm, const CacheView& v, const uint16_
   a.coef = v.k_coef;
   a.cscale = v.k_cscale;
   a.tokver = v.tokver;
+  a.centver = v.centver;
   a.eigvec = v.eigvec;
   a.qfull = Dm.qsac_full;
   cudaError_t e = (Dm.d == 128) ? run<128, true>(a, s) : run<64, true>(a, s);
   if (e != cudaSuccess) return e;
   // values
   a.X = V;
-  a.cent = v.cent_v;
+  a.cent = v.cent_v + coff;
   a.codes = v.v_codes;
   a.params = v.v_params;
   a.idx = v.v_idx;

@@ -85,8 +85,9 @@ struct ApArgs {
   int8_t* coef;
   uint16_t* cscale;
   uint16_t* tokver;
+  uint16_t* centver;
   int64_t n, t0, tcap;
-  int H, C, G, M, r, idx_bytes, version;
+  int H, C, G, M, r, idx_bytes, version, cver;
 };
 
 __device__ __forceinline__ bool lex_less(float a, int ia, float b, int ib) {
@@ -556,7 +557,10 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
   if (A.idx_bytes == 1) ((uint8_t*)A.idx)[slot] = (uint8_t)a;
   else ((uint16_t*)A.idx)[slot] = (uint16_t)a;
   if (KEY) {
-    if (h == 0) A.tokver[A.t0 + tok] = (uint16_t)A.version;
+    if (h == 0) {
+      A.tokver[A.t0 + tok] = (uint16_t)A.version;
+      A.centver[A.t0 + tok] = (uint16_t)A.cver;
+    }
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i)
@@ -613,7 +617,8 @@ bool append_tc_supported(const Dims& D) {
 
 cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t* K,
                              const uint16_t* V, int64_t n, int64_t t0, int version,
-                             cudaStream_t s) {
+                             int cent_version, cudaStream_t s) {
+  const size_t coff = (size_t)cent_version * cent_slot_elems(Dm);
   ApArgs a{};
   a.n = n;
   a.t0 = t0;
@@ -625,8 +630,9 @@ cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t*
   a.r = Dm.r;
   a.idx_bytes = Dm.idx_bytes;
   a.version = version;
+  a.cver = cent_version;
   a.X = K;
-  a.cent = v.cent_k;
+  a.cent = v.cent_k + coff;
   a.sens = v.sens;
   a.wgroup = v.wgroup;
   a.basis = v.basis + (size_t)version * Dm.H * Dm.d * (Dm.r > 0 ? Dm.r : 1);
@@ -636,10 +642,11 @@ cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t*
   a.coef = v.k_coef;
   a.cscale = v.k_cscale;
   a.tokver = v.tokver;
+  a.centver = v.centver;
   cudaError_t e = run_tc_g<true>(a, s);
   if (e != cudaSuccess) return e;
   a.X = V;
-  a.cent = v.cent_v;
+  a.cent = v.cent_v + coff;
   a.codes = v.v_codes;
   a.params = v.v_params;
   a.idx = v.v_idx;

@@ -4,45 +4,37 @@
 // O = softmax(scale Q K'^T) V' with K' = C_K[a] + deq(R) + U_v (c8 cs) and
 // V' = C_V[b] + deq(R_V) reconstructed on the fly (QuantWM, "Flickering after
 // quantization?" (SynthePulse), PSAC paragraph: the Key error is compensated
-// when the cache is reconstructed; U_v is the basis in force when the key was
-// appended).
-//
-// The compensation term runs on the tensor cores instead of per element:
-//   q . (U_v c_t) = (U_v^T q) . c_t,
-// so each Q K^T gains one extra K16 step (two for r > 8) whose A operand holds
-// AX = [Q U_va | Q U_vb] for the (at most two) basis versions va, vb of the key
-// tile and whose B operand holds each key's c8 cs in the slot of its version.
-// AX itself is a tensor-core product (Q from TMEM times [U_va | U_vb] in bf16),
-// recomputed only when the version pair changes from one key tile to the next;
-// a key whose version is neither (a tile spanning three versions) is
-// compensated element-wise by its dequant thread instead.
+// when the cache is reconstructed; U_v is the basis and C the centroid table in
+// force when the key was appended).  Each element of K' and V' is summed in
+// fp32 and rounded once to bf16, so the tensor cores read the same bf16 cache
+// that the reconstruction returns.
 //
 // One CTA per (head, 256 query rows = two 128-row Q tiles); 608 threads:
 //   warps 0-7   softmax: warp w serves Q tile w/4, TMEM lanes 32(w%4)..+31 =
 //               query rows; online softmax in the log2 domain with a lazy
 //               rescale of O, P written back into TMEM over S (bf16 pairs).
-//   warps 8-15  dequant: four threads per key row of each 64-key tile gather
-//               their centroid chunks with 16-byte async copies two tiles
-//               ahead, then rewrite them in place as K-hat / V' (bf16, the
-//               128B-swizzled layouts the UMMA descriptors read).
-//   warps 16-17 MMA: one issuing thread per Q tile, S = Q K^T (+ AX BX^T)
-//               then, once the softmax has written P, O += P V'; the two
-//               threads interleave on the tensor pipe, which works on one Q
-//               tile while the softmax works on the other.
+//   warps 8-15  dequant: warp 8+s owns channels [16s, 16s+16) of every key of
+//               a 64-key tile (lane l: keys l and l+32); it gathers those
+//               centroid chunks with 16-byte async copies two tiles ahead, then
+//               rewrites them in place as K' / V' (bf16, the 128B-swizzled
+//               layouts the UMMA descriptors read).  All lanes of a warp read the
+//               same basis rows, so the compensation's loads are broadcasts.
+//   warps 16-17 MMA: one issuing thread per Q tile, S = Q K'^T then, once the
+//               softmax has written P, O += P V'; the two threads interleave on
+//               the tensor pipe, which works on one Q tile while the softmax
+//               works on the other.
 //   warp 18     producer: bulk-copies (TMA engine) the tile's packed codes,
-//               group parameters, coefficients, versions and centroid indices
-//               into the packed-field ring, and builds [U_va | U_vb] in bf16
-//               on changes.
+//               group parameters, coefficients, basis and table versions and
+//               centroid indices into the packed-field ring.
 // TMEM (512 columns): per Q tile p, Q at 256p (64 columns of bf16 pairs), S/P
-// at 256p+64, O at 256p+128.  Shared memory: a ring of 4 K-hat / V' /
-// compensation-slab stages (released by the MMA) and a ring of 5 packed-field
-// stages (released by the dequant).
+// at 256p+64, O at 256p+128.  Shared memory: a ring of 5 K' / V' stages
+// (released by the MMA) and a ring of 5 packed-field stages (released by the
+// dequant).
 //
 // The SEG instance also attends over a bf16 segment after the packed tokens
 // (the frame being generated): its tiles follow the packed ones, and the
 // dequant warps copy their rows into the same swizzled stages instead of
-// decoding; they carry the last packed tile's version pair and zero
-// compensation rows.  An optional output receives ln sum exp of the scores.
+// decoding.  An optional output receives ln sum exp of the scores.
 //
 // Every mbarrier wait is bounded (about 1 s); a timeout sets a device flag
 // that qwm_device_status() reports, every role then leaves its loop, and
@@ -63,46 +55,37 @@ constexpr int DH = 128;        // head_dim handled here
 constexpr int KT = 64;         // keys per tile
 constexpr int QT = 128;        // query rows per Q tile (TMEM lanes)
 constexpr int BQ = 2 * QT;     // query rows per CTA
-constexpr int NKV = 4;         // K-hat / V' stages (released by the MMA)
+constexpr int NKV = 5;         // K' / V' stages (released by the MMA)
 constexpr int NPK = 5;         // packed-field stages (released by the dequant)
 constexpr int NTHREADS = 608;  // 8 softmax + 8 dequant + 2 MMA + producer warps
 constexpr int W_MMA = 16;      // warps 16, 17 issue the MMAs of Q tiles 0, 1
 constexpr int W_PROD = 18;
 constexpr int NDQW = 8;        // dequant warps
 
-// ---- shared memory (bytes); K-hat and V' tiles 1024-aligned for the swizzle
+// ---- shared memory (bytes); K' and V' tiles 1024-aligned for the swizzle
 constexpr uint32_t KV_TILE = KT * DH * 2;  // [2 column halves][64 rows][128 B]
-constexpr uint32_t ST_K = 0, ST_V = KV_TILE, ST_BX = 2 * KV_TILE;
-constexpr uint32_t BX_BYTES = KT * 32 * 2;  // [64 keys][<= 32] bf16
-constexpr uint32_t KVST = ST_BX + BX_BYTES;  // 36 KB
+constexpr uint32_t ST_K = 0, ST_V = KV_TILE;
+constexpr uint32_t KVST = 2 * KV_TILE;     // 32 KB
 constexpr uint32_t PK_KCODE = 0, PK_VCODE = 2048, PK_KPAR = 4096, PK_VPAR = 6144,
                    PK_KCOEF = 8192, PK_KCS = 9216, PK_TV = 9344, PK_KIDX = 9472,
-                   PK_VIDX = 9600, PK_BYTES = 9728;
-constexpr uint32_t AX_BYTES = QT * 32 * 2;  // [128 rows][<= 32] bf16 per Q tile
-constexpr uint32_t UB_BYTES = 32 * DH * 2;  // [<= 32 rows][128] bf16 per buffer
+                   PK_VIDX = 9600, PK_CV = 9728, PK_BYTES = 9856;
 constexpr uint32_t OFF_KV = 0;
 constexpr uint32_t OFF_PK = OFF_KV + NKV * KVST;
-constexpr uint32_t OFF_AX = (OFF_PK + NPK * PK_BYTES + 1023) / 1024 * 1024;
-constexpr uint32_t OFF_UB = OFF_AX + 2 * AX_BYTES;
-constexpr uint32_t OFF_INFO = OFF_UB + 2 * UB_BYTES;  // [NKV] version pair of the tile in stage
-constexpr uint32_t OFF_BAR = OFF_INFO + 128;
-constexpr int NBAR = 35;
+constexpr uint32_t OFF_BAR = (OFF_PK + NPK * PK_BYTES + 127) / 128 * 128;
+constexpr int NBAR = 32;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the attention CTA");
 
 enum {
   B_LOAD_FULL = 0,   // [NPK] producer bulk copies (tx bytes) -> dequant
   B_PK_EMPTY = 5,    // [NPK] dequant (one arrival per warp) -> producer
   B_KV_FULL = 10,    // [NKV] dequant (one arrival per warp) -> MMA
-  B_KV_EMPTY = 14,   // [NKV] MMA commit after each Q tile's P V' -> dequant
-  B_S_FULL = 18,     // [2] MMA commit after Q K^T, or after AX on a version change
-  B_P_FULL = 20,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
-  // 22, 23 unused
-  B_AX_FULL = 24,    // [2] softmax (per warp) -> MMA: AX slab in shared memory
-  B_UB_FULL = 26,    // [2] producer -> MMA: [U_va | U_vb] in buffer
-  B_UB_EMPTY = 28,   // [2] MMA commit after the AX products -> producer
-  B_Q_READY = 30,    // softmax (per warp) -> MMA: Q in TMEM
-  B_O_LAST = 31,     // [2] MMA commit after the last P V' of that Q tile
-  B_DONE = 33        // [2] MMA commit -> MMA (drain before exit)
+  B_KV_EMPTY = 15,   // [NKV] MMA commit after each Q tile's P V' -> dequant
+  B_S_FULL = 20,     // [2] MMA commit after Q K'^T
+  B_P_FULL = 22,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
+  B_Q_READY = 24,    // softmax (per warp) -> MMA: Q in TMEM
+  B_O_LAST = 25,     // [2] MMA commit after the last P V' of that Q tile
+  B_DONE = 27        // [2] MMA commit -> MMA (drain before exit)
 };
 
 struct TcArgs {
@@ -113,7 +96,6 @@ struct TcArgs {
   int64_t nq;
   float scale_log2;
   uint16_t* O;
-  int kx;        // extra K width for the compensation (0, 16 or 32)
   const uint16_t* Ks;  // bf16 segment [nseg][H][d] after the packed tokens (tiles ntp ..)
   const uint16_t* Vs;
   int64_t nseg;
@@ -158,28 +140,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, w);
 }
 
-// Versions in force for the first and the last key of tile j, packed as
-// first | last << 16 (read from global memory).
-__device__ __forceinline__ uint32_t tile_pair_global(const uint16_t* tokver, int64_t T, int j) {
-  const int64_t t0 = (int64_t)j * KT;
-  const int64_t t1 = ((t0 + KT) < T ? (t0 + KT) : T) - 1;
-  return (uint32_t)tokver[t0] | ((uint32_t)tokver[t1] << 16);
-}
-
-// Slab layouts (no swizzle, K-major core matrices of 8 rows x 16 B):
-//   AX  [128 rows][kx]: core (row group g, K column kc) at kc*2048 + g*128
-//   BX  [64 keys][kx] : core (g, kc) at kc*1024 + g*128
-//   UB  [kx rows][128]: core (g, kc) at g*2048 + kc*128
-__device__ __forceinline__ uint32_t ax_off(int m, int kc) {
-  return (uint32_t)(kc * 2048 + (m >> 3) * 128 + (m & 7) * 16);
-}
-__device__ __forceinline__ uint32_t bx_off(int n, int kc) {
-  return (uint32_t)(kc * 1024 + (n >> 3) * 128 + (n & 7) * 16);
-}
-__device__ __forceinline__ uint32_t ub_off(int n, int kc) {
-  return (uint32_t)((n >> 3) * 2048 + kc * 128 + (n & 7) * 16);
-}
-
 // ------------------------------------------------------------------ softmax role
 // The exponent reference m_used of a row moves only when the row maximum has
 // grown by more than TAU (log2 units); P then stays below 2^TAU and O, which
@@ -206,14 +166,13 @@ __device__ __forceinline__ float row_max(const float (&s)[64], int n) {
 }
 
 template <bool SEG>
-__device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
-                                             uint32_t tmem, int ntile, int nqt) {
+__device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, uint32_t tmem,
+                                             int ntile, int nqt) {
   const int warp = threadIdx.x >> 5;
   const int p = warp >> 2;          // Q tile
   const int m = threadIdx.x & 127;  // row in the Q tile = TMEM lane
   const int h = blockIdx.y;
   const int H = A.Dm.H;
-  const int kx = A.kx;
   const int64_t q = (int64_t)blockIdx.x * BQ + p * QT + m;
   const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   const uint32_t tq = trow + 256 * p, ts = tq + 64, to = tq + 128;
@@ -239,52 +198,14 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
   warp_arrive(&bars[B_Q_READY]);
   if (p >= nqt) return;
 
-  uint8_t* ax = smem + OFF_AX + p * AX_BYTES;
-  const uint32_t* kvinfo = reinterpret_cast<const uint32_t*>(smem + OFF_INFO);
-  uint32_t prev = 0xffffffffu;
-  int sph = 0;  // phases of S_FULL seen: one per tile, two when the tile brings AX
   float m_used = -INFINITY;
   uint64_t l2 = 0;  // running row sum, as a pair of partial sums
   const float sl2 = A.scale_log2;
   const uint64_t sc2 = f2pack(sl2, sl2);
   bool ok = true;
   for (int j = 0; j < ntile; ++j) {
-    if (!warp_wait(&bars[B_S_FULL + p], sph & 1)) { ok = false; break; }
-    ++sph;
+    if (!warp_wait(&bars[B_S_FULL + p], j & 1)) { ok = false; break; }
     tc_fence_after();
-    if (kx) {
-      // the version pair of the tile (written by the dequant before the stage
-      // was handed to the MMA); on a change the S columns hold AX = Q [U_va | U_vb]
-      const uint32_t pr = kvinfo[j % NKV];
-      if (pr != prev) {
-        prev = pr;
-        uint32_t w[16];
-        if (kx == 16) {
-          float a[16];
-          tmem_ld16(ts, a);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[e] = pack_bf16(a[2 * e], a[2 * e + 1]);
-#pragma unroll
-          for (int e = 8; e < 16; ++e) w[e] = 0u;
-        } else {
-          float a[32];
-          tmem_ld32(ts, a);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = pack_bf16(a[2 * e], a[2 * e + 1]);
-        }
-#pragma unroll
-        for (int kc = 0; kc < 4; ++kc)
-          if (kc < kx / 8)
-            *reinterpret_cast<uint4*>(ax + ax_off(m, kc)) =
-                make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        warp_arrive(&bars[B_AX_FULL + p]);
-        if (!warp_wait(&bars[B_S_FULL + p], sph & 1)) { ok = false; break; }
-        ++sph;
-        tc_fence_after();
-      }
-    }
     const int nvalid = tile_valid<SEG>(A, j);
     float m_row;
     {
@@ -298,7 +219,7 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint8_t* smem, uin
       const bool need = m_row > m_used + TAU;
       if (__any_sync(0xffffffffu, need)) {
         // O holds P V' of tiles < j, all complete: the commit behind S_FULL(j)
-        // tracks every MMA issued before Q K^T of tile j.
+        // tracks every MMA issued before Q K'^T of tile j.
         const float f = need ? ex2(m_used - m_row) : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -425,65 +346,66 @@ __device__ __forceinline__ int staged_idx(const uint8_t* pk, uint32_t off, int k
   return ib == 1 ? (int)pk[off + k] : (int)reinterpret_cast<const uint16_t*>(pk + off)[k];
 }
 
-// Element-wise compensation U (c8 cs) of channels j0..j0+7 (rare path).
-__device__ __forceinline__ void compensate_chunk(uint64_t (&v2)[4], const float* U, const uint8_t* pk,
-                                              int k, int r, int j0) {
-  const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
-  const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
-  for (int pi = 0; pi < 4; ++pi) {
-    float a, b, ca = 0.0f, cb = 0.0f;
-    f2unpack(v2[pi], a, b);
-    for (int i = 0; i < r; ++i) {
-      const float ch = (float)cf[i] * cs;
-      ca = fmaf(__ldg(U + (size_t)(j0 + 2 * pi) * r + i), ch, ca);
-      cb = fmaf(__ldg(U + (size_t)(j0 + 2 * pi + 1) * r + i), ch, cb);
-    }
-    v2[pi] = f2pack(a + ca, b + cb);
+// Rank-8 compensation of one channel for two keys: sum_i U_ji cc_i with the
+// coefficients as pairs {cc_2m, cc_2m+1}; row j of each key's basis holds 8
+// fp32 values (two 16-byte loads; all lanes of the warp read the same row when
+// the keys share a basis version).
+__device__ __forceinline__ void corr8_pair(const float* U0, const float* U1, bool same,
+                                           const uint64_t (&c0)[4], const uint64_t (&c1)[4],
+                                           float& o0, float& o1) {
+  const float4 a0 = __ldg(reinterpret_cast<const float4*>(U0));
+  const float4 b0 = __ldg(reinterpret_cast<const float4*>(U0) + 1);
+  float4 a1 = a0, b1 = b0;
+  if (!same) {
+    a1 = __ldg(reinterpret_cast<const float4*>(U1));
+    b1 = __ldg(reinterpret_cast<const float4*>(U1) + 1);
   }
+  uint64_t s0 = ffma2(f2pack(a0.x, a0.y), c0[0], 0ull);
+  uint64_t s1 = ffma2(f2pack(a1.x, a1.y), c1[0], 0ull);
+  s0 = ffma2(f2pack(a0.z, a0.w), c0[1], s0);
+  s1 = ffma2(f2pack(a1.z, a1.w), c1[1], s1);
+  s0 = ffma2(f2pack(b0.x, b0.y), c0[2], s0);
+  s1 = ffma2(f2pack(b1.x, b1.y), c1[2], s1);
+  s0 = ffma2(f2pack(b0.z, b0.w), c0[3], s0);
+  s1 = ffma2(f2pack(b1.z, b1.w), c1[3], s1);
+  float x, y;
+  f2unpack(s0, x, y);
+  o0 = x + y;
+  f2unpack(s1, x, y);
+  o1 = x + y;
 }
 
-// One tensor (K or V) of this thread's quarter row: centroid chunks read from
-// the stage, residual added, bf16 written back in place.  U != nullptr adds the
-// element-wise compensation U (c8 cs) (a key whose basis version is not one of
-// the tile's two slots).
-__device__ __forceinline__ void deq_quarter(uint8_t* base, const uint32_t (&offs)[4], uint2 w,
-                                            const uint32_t* par, int G, int qq, const float* U,
-                                            const uint8_t* pk, int k, int r) {
-  uint4 cv[4];
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc) cv[cc] = *reinterpret_cast<const uint4*>(base + offs[cc]);
-  GroupConst g;
-  if (G == 32) g = group_const(par[qq]);
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    const int lc = (cc + qq) & 3;  // chunk within the quarter
-    if (G != 32) g = group_const(par[(4 * qq + lc) * 8 / G]);
-    const uint32_t bits = (lc < 2 ? w.x : w.y) >> (16 * (lc & 1));
-    uint64_t v2[4];
-    deq_chunk_f32(cv[cc], bits, g, v2);
-    if (U) compensate_chunk(v2, U, pk, k, r, (4 * qq + lc) * 8);
-    *reinterpret_cast<uint4*>(base + offs[cc]) = pack_chunk(v2);
-  }
+// Compensation of one channel for any rank: sequential fold of U_ji c8_i cs
+// (the coefficients read from the staged packed fields).
+__device__ __forceinline__ float corr_any(const float* Uj, const int8_t* cf, float cs, int r) {
+  float acc = 0.0f;
+  for (int i = 0; i < r; ++i) acc = fmaf(__ldg(Uj + i), (float)cf[i] * cs, acc);
+  return acc;
 }
 
-// Issue this thread's 16-byte centroid-chunk copies for tile jj (key row k,
-// channel chunks 4qq..4qq+3 of K and V); one commit group per tile.
+// Issue this thread's 16-byte centroid-chunk copies for tile jj: keys l and
+// l + 32, channel chunks 2s and 2s + 1 of K and V (s = dequant warp), each from
+// the table version the key was encoded with; one commit group per tile.
 __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, const PackedHead& ph,
-                                             int jj, int k, int qq) {
+                                             int jj, int lane, int sw) {
   const uint8_t* pk = smem + OFF_PK + (jj % NPK) * PK_BYTES;
   const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
-  const int64_t t = (int64_t)jj * KT + k;
-  if (t < A.T) {
-    const int ib = A.Dm.idx_bytes;
-    const int a = staged_idx(pk, PK_KIDX, k, ib);
-    const int b = staged_idx(pk, PK_VIDX, k, ib);
-    const uint16_t* ck = ph.cent_k + (size_t)a * DH;
-    const uint16_t* cv = ph.cent_v + (size_t)b * DH;
+  const int ib = A.Dm.idx_bytes;
+  const uint16_t* cvs = reinterpret_cast<const uint16_t*>(pk + PK_CV);
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int c = 4 * qq + ((cc + qq) & 3);  // same bank-group rotation as the rewrite
-      cp_async16(st + ST_K + sw128_off(k, c, KT), ck + c * 8);
-      cp_async16(st + ST_V + sw128_off(k, c, KT), cv + c * 8);
+  for (int kk = 0; kk < 2; ++kk) {
+    const int k = lane + 32 * kk;
+    const int64_t t = (int64_t)jj * KT + k;
+    if (t < A.T) {
+      const size_t vo = (size_t)cvs[k] * ph.cstride;
+      const uint16_t* ck = ph.cent_k + vo + (size_t)staged_idx(pk, PK_KIDX, k, ib) * DH;
+      const uint16_t* cv = ph.cent_v + vo + (size_t)staged_idx(pk, PK_VIDX, k, ib) * DH;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * sw + cc;
+        cp_async16(st + ST_K + sw128_off(k, c, KT), ck + c * 8);
+        cp_async16(st + ST_V + sw128_off(k, c, KT), cv + c * 8);
+      }
     }
   }
   cp_async_commit();
@@ -491,48 +413,73 @@ __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, con
 
 // Segment tile jj (jj >= ntp): this thread's 16-byte chunks of the bf16 K and V
 // rows copied as they are into the same swizzled stage positions.
-__device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem, int jj, int k,
-                                                 int qq) {
+__device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem, int jj, int lane,
+                                                 int sw) {
   const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
-  const int64_t t = (int64_t)(jj - A.ntp) * KT + k;
-  if (t < A.nseg) {
-    const size_t row = ((size_t)t * A.Dm.H + blockIdx.y) * DH;
-    const uint16_t* kr = A.Ks + row;
-    const uint16_t* vr = A.Vs + row;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int c = 4 * qq + ((cc + qq) & 3);
-      cp_async16(st + ST_K + sw128_off(k, c, KT), kr + c * 8);
-      cp_async16(st + ST_V + sw128_off(k, c, KT), vr + c * 8);
+  for (int kk = 0; kk < 2; ++kk) {
+    const int k = lane + 32 * kk;
+    const int64_t t = (int64_t)(jj - A.ntp) * KT + k;
+    if (t < A.nseg) {
+      const size_t row = ((size_t)t * A.Dm.H + blockIdx.y) * DH;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * sw + cc;
+        cp_async16(st + ST_K + sw128_off(k, c, KT), A.Ks + row + c * 8);
+        cp_async16(st + ST_V + sw128_off(k, c, KT), A.Vs + row + c * 8);
+      }
     }
   }
   cp_async_commit();
+}
+
+// Rewrite chunk c (8 channels) of key row k in place: centroid chunk from the
+// stage, residual (and compensation) added in fp32, one bf16 rounding.
+__device__ __forceinline__ void deq_chunk(uint8_t* base, int k, int c, uint32_t bits16,
+                                          uint32_t par, const float* corr) {
+  const GroupConst g = group_const(par);
+  const uint32_t off = sw128_off(k, c, KT);
+  const uint4 cw = *reinterpret_cast<const uint4*>(base + off);
+  uint64_t v2[4];
+  deq_chunk_f32(cw, bits16, g, v2);
+  if (corr) {
+#pragma unroll
+    for (int pi = 0; pi < 4; ++pi) v2[pi] = fadd2(v2[pi], f2pack(corr[2 * pi], corr[2 * pi + 1]));
+  }
+  *reinterpret_cast<uint4*>(base + off) = pack_chunk(v2);
+}
+
+__device__ __forceinline__ void zero_chunks(uint8_t* kb, uint8_t* vb, int k, int sw) {
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const uint32_t off = sw128_off(k, 2 * sw + cc, KT);
+    *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
+  }
 }
 
 template <bool SEG>
 __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                              int ntile) {
   const int dq = threadIdx.x - 256;  // 0..255
-  const int k = dq >> 2;             // key row in the tile
-  const int qq = dq & 3;             // channel quarter [32 qq, 32 qq + 32)
+  const int sw = dq >> 5;            // channel slice [16 sw, 16 sw + 16)
+  const int lane = dq & 31;          // keys lane, lane + 32
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
-  const int G = Dm.G, ng = Dm.ng, r = Dm.r, kx = A.kx;
-  uint32_t* kvinfo = reinterpret_cast<uint32_t*>(smem + OFF_INFO);
+  const int G = Dm.G, ng = Dm.ng, r = Dm.r;
+  const int gi = (16 * sw) / G;      // the slice's INT2 group (one group: G = 16 or 32)
+  const size_t ustride = (size_t)Dm.H * DH * (r > 0 ? r : 1);  // floats per basis version
+  const float* ubase = A.v.basis + (size_t)h * DH * (r > 0 ? r : 1) + (size_t)16 * sw * r;
   bool ok = true;
   const int ntp = SEG ? A.ntp : ntile;
-  // the version pair segment tiles carry: that of the last packed tile, so the
-  // compensation slab stays in place (segment keys have zero BX rows)
-  const uint32_t seg_pair =
-      (SEG && kx && ntp > 0) ? tile_pair_global(A.v.tokver, A.T, ntp - 1) : 0u;
-  // prologue: gathers of tiles 0 and 1 (their K-hat / V' stages start free)
+  // prologue: gathers of tiles 0 and 1 (their K' / V' stages start free)
   for (int jj = 0; jj < 2 && jj < ntile; ++jj) {
     if (!SEG || jj < ntp) {
       if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
-      issue_gather(A, smem, ph, jj, k, qq);
+      issue_gather(A, smem, ph, jj, lane, sw);
     } else {
-      issue_seg_gather(A, smem, jj, k, qq);
+      issue_seg_gather(A, smem, jj, lane, sw);
     }
   }
   for (int j = 0; ok && j < ntile; ++j) {
@@ -542,8 +489,8 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
           !warp_wait(&bars[B_LOAD_FULL + j2 % NPK], (j2 / NPK) & 1)) { ok = false; break; }
       if (j2 >= NKV &&
           !warp_wait(&bars[B_KV_EMPTY + j2 % NKV], ((j2 / NKV) - 1) & 1)) { ok = false; break; }
-      if (!SEG || j2 < ntp) issue_gather(A, smem, ph, j2, k, qq);
-      else issue_seg_gather(A, smem, j2, k, qq);
+      if (!SEG || j2 < ntp) issue_gather(A, smem, ph, j2, lane, sw);
+      else issue_seg_gather(A, smem, j2, lane, sw);
       cp_async_wait<2>();
     } else if (j + 1 < ntile) {
       cp_async_wait<1>();
@@ -554,80 +501,88 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
     uint8_t* st = smem + OFF_KV + s * KVST;
     uint8_t* kb = st + ST_K;
     uint8_t* vb = st + ST_V;
-    uint8_t* xb = st + ST_BX;
     if (SEG && j >= ntp) {
       // segment tile: rows already in place; zero rows past the segment's end
-      // and zero compensation rows
-      if ((int64_t)(j - ntp) * KT + k >= A.nseg) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t off = sw128_off(k, 4 * qq + cc, KT);
-          *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
+      for (int kk = 0; kk < 2; ++kk) {
+        const int k = lane + 32 * kk;
+        if ((int64_t)(j - ntp) * KT + k >= A.nseg) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t off = sw128_off(k, 2 * sw + cc, KT);
+            *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
+          }
         }
       }
-      if (qq < kx / 8) *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(0, 0, 0, 0);
-      if (dq == 0) kvinfo[s] = seg_pair;
       fence_proxy_async_smem();
       warp_arrive(&bars[B_KV_FULL + s]);
       continue;
     }
     const uint8_t* pk = smem + OFF_PK + sp * PK_BYTES;
     const int64_t t0 = (int64_t)j * KT;
-    const int64_t t = t0 + k;
-    const int nvalid = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
     const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
-    const int va = tv[0], vbv = tv[nvalid - 1];
-    if (t < A.T) {
-      const uint2 kw = *reinterpret_cast<const uint2*>(pk + PK_KCODE + k * 32 + qq * 8);
-      const uint2 vw = *reinterpret_cast<const uint2*>(pk + PK_VCODE + k * 32 + qq * 8);
-      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(pk + PK_KPAR) + k * ng;
-      const uint32_t* vpar = reinterpret_cast<const uint32_t*>(pk + PK_VPAR) + k * ng;
-      bool fallback = false;
-      int ver = 0;
-      if (r > 0) {
-        ver = tv[k];
-        fallback = (ver != va) && (ver != vbv);
-        if (qq < kx / 8) {
-          // compensation slab row: c8 cs in the slot of the key's version
-          // (slot = K columns [0, kx/2) for va, [kx/2, kx) for vb); thread qq
-          // writes core column qq (8 columns)
-          const int per = kx / 16;  // core columns per slot: 1 or 2
-          const int slot = qq / per, i0 = (qq % per) * 8;
-          const int sl = (ver == va) ? 0 : ((ver == vbv) ? 1 : -1);
-          uint32_t w[4] = {0u, 0u, 0u, 0u};
-          if (slot == sl) {
-            const float cs = h2f(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[k]);
-            const int8_t* cf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + k * r;
+    const uint16_t* kcs = reinterpret_cast<const uint16_t*>(pk + PK_KCS);
+    const int8_t* kcf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF);
+    const int k0 = lane, k1 = lane + 32;
+    const bool in0 = t0 + k0 < A.T, in1 = t0 + k1 < A.T;
+    const uint32_t* kpar = reinterpret_cast<const uint32_t*>(pk + PK_KPAR);
+    const uint32_t* vpar = reinterpret_cast<const uint32_t*>(pk + PK_VPAR);
+    // ---- K' rows: residual plus the compensation of this slice's channels
+    {
+      const uint32_t kw0 = *reinterpret_cast<const uint32_t*>(pk + PK_KCODE + k0 * 32 + 4 * sw);
+      const uint32_t kw1 = *reinterpret_cast<const uint32_t*>(pk + PK_KCODE + k1 * 32 + 4 * sw);
+      const uint32_t p0 = kpar[k0 * ng + gi], p1 = kpar[k1 * ng + gi];
+      const int v0 = in0 ? tv[k0] : 0, v1 = in1 ? tv[k1] : v0;
+      const float* U0 = ubase + (size_t)v0 * ustride;
+      const float* U1 = ubase + (size_t)v1 * ustride;
+      const float cs0 = in0 ? h2f(kcs[k0]) : 0.0f, cs1 = in1 ? h2f(kcs[k1]) : 0.0f;
+      uint64_t c0[4], c1[4];
+      if (r == 8) {
+        const int2 w0 = *reinterpret_cast<const int2*>(kcf + 8 * k0);
+        const int2 w1 = *reinterpret_cast<const int2*>(kcf + 8 * k1);
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const float x0 = (i0 + e < r) ? (float)cf[i0 + e] * cs : 0.0f;
-              const float x1 = (i0 + e + 1 < r) ? (float)cf[i0 + e + 1] * cs : 0.0f;
-              w[e / 2] = pack_bf16(x0, x1);
-            }
-          }
-          *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t x0 = m < 2 ? (uint32_t)w0.x : (uint32_t)w0.y;
+          const uint32_t x1 = m < 2 ? (uint32_t)w1.x : (uint32_t)w1.y;
+          const int sh = 16 * (m & 1);
+          // c8 * cs is exact in fp32 (8-bit times 11-bit significands)
+          c0[m] = f2pack((float)(int8_t)(x0 >> sh) * cs0, (float)(int8_t)(x0 >> (sh + 8)) * cs0);
+          c1[m] = f2pack((float)(int8_t)(x1 >> sh) * cs1, (float)(int8_t)(x1 >> (sh + 8)) * cs1);
         }
       }
-      // rotating the chunk order by the quarter keeps the 8 threads of a
-      // shared-memory phase on distinct 16-byte bank groups
-      uint32_t offs[4];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) offs[cc] = sw128_off(k, 4 * qq + ((cc + qq) & 3), KT);
-      const float* U = fallback ? basis_of(A.v, Dm, ver, h) : nullptr;
-      deq_quarter(kb, offs, kw, kpar, G, qq, U, pk, k, r);
-      deq_quarter(vb, offs, vw, vpar, G, qq, nullptr, pk, k, r);
-    } else {
-      // past the end of the cache: zero rows (finite V' under P = 0)
+      for (int cc = 0; cc < 2; ++cc) {
+        float q0[8], q1[8];
+        if (r == 8) {
+          const bool same = (v0 == v1);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const uint32_t off = sw128_off(k, 4 * qq + cc, KT);
-        *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < 8; ++e)
+            corr8_pair(U0 + 8 * (8 * cc + e), U1 + 8 * (8 * cc + e), same, c0, c1, q0[e], q1[e]);
+        } else if (r > 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            q0[e] = corr_any(U0 + (size_t)(8 * cc + e) * r, kcf + k0 * r, cs0, r);
+            q1[e] = corr_any(U1 + (size_t)(8 * cc + e) * r, kcf + k1 * r, cs1, r);
+          }
+        }
+        if (in0) deq_chunk(kb, k0, 2 * sw + cc, (kw0 >> (16 * cc)) & 0xffffu, p0, r > 0 ? q0 : nullptr);
+        if (in1) deq_chunk(kb, k1, 2 * sw + cc, (kw1 >> (16 * cc)) & 0xffffu, p1, r > 0 ? q1 : nullptr);
       }
-      if (qq < kx / 8) *reinterpret_cast<uint4*>(xb + bx_off(k, qq)) = make_uint4(0, 0, 0, 0);
     }
-    if (dq == 0) kvinfo[s] = (uint32_t)va | ((uint32_t)vbv << 16);
+    // ---- V' rows
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int k = lane + 32 * kk;
+      if (kk == 0 ? in0 : in1) {
+        const uint32_t vw = *reinterpret_cast<const uint32_t*>(pk + PK_VCODE + k * 32 + 4 * sw);
+        const uint32_t vp = vpar[k * ng + gi];
+        deq_chunk(vb, k, 2 * sw, vw & 0xffffu, vp, nullptr);
+        deq_chunk(vb, k, 2 * sw + 1, vw >> 16, vp, nullptr);
+      } else {
+        zero_chunks(kb, vb, k, sw);
+      }
+    }
     fence_proxy_async_smem();
     warp_arrive(&bars[B_KV_FULL + s]);
     warp_arrive(&bars[B_PK_EMPTY + sp]);
@@ -643,13 +598,10 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
-  const int ng = Dm.ng, r = Dm.r, kx = A.kx, ib = Dm.idx_bytes;
+  const int ng = Dm.ng, r = Dm.r, ib = Dm.idx_bytes;
   const uint32_t par_bytes = KT * ng * 4, coef_bytes = KT * r, idx_bytes = KT * ib;
   const uint32_t tx = 2 * (KT * DH / 4) + 2 * par_bytes + (r > 0 ? coef_bytes + KT * 2 : 0) +
-                      KT * 2 + 2 * idx_bytes;
-  const uint16_t* tokver = A.v.tokver;
-  uint32_t prev = 0xffffffffu;
-  int nchg = 0;
+                      2 * KT * 2 + 2 * idx_bytes;
   bool ok = true;
   int issued = 0;
   for (int j = 0; j < ntile; ++j) {
@@ -670,48 +622,13 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
         bulk_g2s(smem_u32(pk + PK_KCOEF), ph.k_coef + t0 * r, coef_bytes, bar);
         bulk_g2s(smem_u32(pk + PK_KCS), ph.k_cscale + t0, KT * 2, bar);
       }
-      bulk_g2s(smem_u32(pk + PK_TV), tokver + t0, KT * 2, bar);
+      bulk_g2s(smem_u32(pk + PK_TV), A.v.tokver + t0, KT * 2, bar);
+      bulk_g2s(smem_u32(pk + PK_CV), A.v.centver + t0, KT * 2, bar);
       bulk_g2s(smem_u32(pk + PK_KIDX), (const uint8_t*)ph.k_idx + t0 * ib, idx_bytes, bar);
       bulk_g2s(smem_u32(pk + PK_VIDX), (const uint8_t*)ph.v_idx + t0 * ib, idx_bytes, bar);
     }
     __syncwarp();
     ++issued;
-    if (kx) {
-      const uint32_t pr = tile_pair_global(tokver, A.T, j);
-      if (pr != prev) {
-        // two buffers: the wait is for the change before last, whose tile
-        // precedes this one by at least two, so the MMA can always reach it
-        const int b = nchg & 1;
-        if (nchg >= 2) {
-          if (!warp_wait(&bars[B_UB_EMPTY + b], ((nchg >> 1) - 1) & 1)) { ok = false; break; }
-        }
-        // [U_va | U_vb]^T in bf16: row n = slot * sw + i holds column i of the
-        // slot's basis (zeros past r, and slot 1 is zero when va == vb)
-        const int va = (int)(pr & 0xffff), vbv = (int)(pr >> 16);
-        const int sw = kx / 2;
-        uint8_t* ub = smem + OFF_UB + b * UB_BYTES;
-        const int kc = lane & 15;
-        for (int n = lane >> 4; n < kx; n += 2) {
-          const int sl = n / sw, i = n % sw;
-          const int ver = sl == 0 ? va : (vbv != va ? vbv : -1);
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = 0.0f;
-          if (ver >= 0 && i < r) {
-            const float* U = basis_of(A.v, Dm, ver, h);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = __ldg(U + (size_t)(kc * 8 + e) * r + i);
-          }
-          *reinterpret_cast<uint4*>(ub + ub_off(n, kc)) =
-              make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                         pack_bf16(x[6], x[7]));
-        }
-        fence_proxy_async_smem();
-        warp_arrive(&bars[B_UB_FULL + b]);
-        prev = pr;
-        ++nchg;
-      }
-    }
   }
   // drain: every bulk copy issued has landed before the CTA may exit
   for (int jj = (issued > NPK ? issued - NPK : 0); jj < issued; ++jj)
@@ -723,11 +640,11 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
 // Descriptors are built once; a stage or K-step offset is added to the start
 // address field (bytes / 16; no carry out of the 14-bit field in 227 KB).
 struct MmaDesc {
-  uint64_t k, v, bx, ax, ub;
+  uint64_t k, v;
 };
 
-// S_p = Q_p K-hat^T (8 K16 steps, A from TMEM) + AX_p BX^T for the tile in stage s.
-__device__ __forceinline__ void issue_qk(const MmaDesc& D, uint32_t tmem, int p, int s, int kx) {
+// S_p = Q_p K'^T (8 K16 steps, A from TMEM) for the tile in stage s.
+__device__ __forceinline__ void issue_qk(const MmaDesc& D, uint32_t tmem, int p, int s) {
   constexpr uint32_t IDQ = idesc_bf16(128, KT, false, false);
   const uint32_t tq = tmem + 256 * p, ts = tq + 64;
   const uint64_t kd = D.k + (uint64_t)((s * KVST) >> 4);
@@ -735,12 +652,6 @@ __device__ __forceinline__ void issue_qk(const MmaDesc& D, uint32_t tmem, int p,
   for (int k = 0; k < 8; ++k) {
     const uint32_t koff = ((k >> 2) * (KT * 128) + (k & 3) * 32) >> 4;
     mma_bf16_ts(ts, tq + 8 * k, kd + koff, IDQ, k > 0);
-  }
-  if (kx) {
-    const uint64_t ad = D.ax + (uint64_t)((p * AX_BYTES) >> 4);
-    const uint64_t bd = D.bx + (uint64_t)((s * KVST) >> 4);
-    mma_bf16_ss(ts, ad, bd, IDQ, 1u);
-    if (kx == 32) mma_bf16_ss(ts, ad + (4096 >> 4), bd + (2048 >> 4), IDQ, 1u);
   }
 }
 
@@ -756,58 +667,26 @@ __device__ __forceinline__ void issue_pv(const MmaDesc& D, uint32_t tmem, int p,
                 (!first || k > 0) ? 1u : 0u);
 }
 
-// AX_p = Q_p [U_va | U_vb] into the S columns of Q tile p.
-__device__ __forceinline__ void issue_ax(const MmaDesc& D, uint32_t tmem, int p, int b, int kx) {
-  const uint32_t idx = idesc_bf16(128, kx, false, false);
-  const uint32_t tq = tmem + 256 * p, ts = tq + 64;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    mma_bf16_ts(ts, tq + 8 * k, D.ub + (uint64_t)((b * UB_BYTES + 2 * k * 128) >> 4), idx, k > 0);
-}
-
 // One issuing thread per Q tile p (warps 16 and 17), each running
-//   Q K^T(p, t) [after AX(p) when the version pair changes at t]
-//     -> wait for the softmax -> P V'(p, t) -> Q K^T(p, t + 1) -> ...
+//   Q K'^T(p, t) -> wait for the softmax -> P V'(p, t) -> Q K'^T(p, t + 1) -> ...
 // with blocking waits; the two threads interleave on the tensor pipe, which
-// works on one Q tile while the softmax works on the other.  Q K^T(p, t + 1) and
-// AX(p) come after P V'(p, t) in the thread's issue order, so an MMA that
+// works on one Q tile while the softmax works on the other.  Q K'^T(p, t + 1)
+// comes after P V'(p, t) in the thread's issue order, so an MMA that
 // overwrites the S/P columns never overtakes the P V' that reads them.  A stage
 // is released after both threads' P V' (one commit each).
 __device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                          uint32_t tmem, int ntile, int p) {
   const uint32_t sbase = smem_u32(smem);
-  const int kx = A.kx;
   MmaDesc D;
   D.k = desc_sw128(sbase + OFF_KV + ST_K, 16, 1024);
   D.v = desc_sw128(sbase + OFF_KV + ST_V, KT * 128, 1024);
-  D.bx = desc_noswz(sbase + OFF_KV + ST_BX, 1024, 128);
-  D.ax = desc_noswz(sbase + OFF_AX, 2048, 128);
-  D.ub = desc_noswz(sbase + OFF_UB, 128, 2048);
-  const uint32_t* kvinfo = reinterpret_cast<const uint32_t*>(smem + OFF_INFO);
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
   tc_fence_after();
-  uint32_t prev = 0xffffffffu;
-  int nchg = 0;
   for (int t = 0; ok && t < ntile; ++t) {
     const int s = t % NKV;
     if (!mbar_wait(&bars[B_KV_FULL + s], (t / NKV) & 1)) { ok = false; break; }
     tc_fence_after();
-    if (kx) {
-      const uint32_t pr = kvinfo[s];
-      if (pr != prev) {
-        const int b = nchg & 1;
-        if (!mbar_wait(&bars[B_UB_FULL + b], (nchg >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_ax(D, tmem, p, b, kx);
-        mma_commit(&bars[B_S_FULL + p]);
-        mma_commit(&bars[B_UB_EMPTY + b]);
-        if (!mbar_wait(&bars[B_AX_FULL + p], nchg & 1)) { ok = false; break; }
-        tc_fence_after();
-        ++nchg;
-        prev = pr;
-      }
-    }
-    issue_qk(D, tmem, p, s, kx);
+    issue_qk(D, tmem, p, s);
     mma_commit(&bars[B_S_FULL + p]);
     if (!mbar_wait(&bars[B_P_FULL + p], t & 1)) { ok = false; break; }
     tc_fence_after();
@@ -842,16 +721,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[B_S_FULL + i], 1);
       mbar_init(&bars[B_P_FULL + i], 4);
-      mbar_init(&bars[B_AX_FULL + i], 4);
       mbar_init(&bars[B_O_LAST + i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[B_UB_FULL + i], 1);
-      mbar_init(&bars[B_UB_EMPTY + i], nqt);  // one commit per Q tile
+      mbar_init(&bars[B_DONE + i], 1);
     }
     mbar_init(&bars[B_Q_READY], 8);
-    mbar_init(&bars[B_DONE], 1);
-    mbar_init(&bars[B_DONE + 1], 1);
     fence_mbar_init();
   }
   if (warp == W_MMA) {
@@ -863,7 +736,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   if (warp < 8) {
-    softmax_role<SEG>(A, smem, bars, tmem, ntile, nqt);
+    softmax_role<SEG>(A, bars, tmem, ntile, nqt);
   } else if (warp < 8 + NDQW) {
     dequant_role<SEG>(A, smem, bars, ntile);
   } else if (warp < W_PROD) {
@@ -896,8 +769,6 @@ cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, co
   a.nq = nq;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
-  // two slots of 8 or 16 columns; none without packed keys
-  a.kx = (D.r == 0 || T == 0) ? 0 : (D.r <= 8 ? 16 : 32);
   a.Ks = sg.K;
   a.Vs = sg.V;
   a.nseg = sg.n;

@@ -19,6 +19,72 @@ struct Dims {
   int qsac_full;  // QSAC stage 2 by the full quadratic form e^T A e
 };
 
+// ---------------------------------------------------------------- host-side validation
+constexpr int32_t kCacheMagic = 0x51574d31;  // "QWM1"
+
+inline bool config_ok(const qwm_config* c) {
+  if (!c) return false;
+  if (c->heads < 1 || c->heads > 4096) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->group != 16 && c->group != 32) return false;
+  if (c->head_dim % c->group) return false;
+  if (c->n_centroids < 1 || c->n_centroids > 512) return false;
+  if (c->n_cand < 1 || c->n_cand > 8 || c->n_cand > c->n_centroids) return false;
+  if (c->rank < 0 || c->rank > 16) return false;
+  if (c->max_versions < 1 || c->max_versions > 65535) return false;
+  if (c->max_cent_versions < 1 || c->max_cent_versions > 65535) return false;
+  if ((c->flags & ~QWM_FLAG_QSAC_FULL) != 0) return false;
+  if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 40)) return false;
+  return true;
+}
+
+inline bool cache_ok(const qwm_cache* c) {
+  return c && c->magic == kCacheMagic && config_ok(&c->cfg);
+}
+
+inline Dims dims_of(const qwm_config* c) {
+  Dims D;
+  D.H = c->heads;
+  D.d = c->head_dim;
+  D.C = c->n_centroids;
+  D.G = c->group;
+  D.M = c->n_cand;
+  D.r = c->rank;
+  D.ng = c->head_dim / c->group;
+  D.tcap = (c->max_tokens + 127) / 128 * 128;
+  D.idx_bytes = c->n_centroids <= 256 ? 1 : 2;
+  D.qsac_full = (c->flags & QWM_FLAG_QSAC_FULL) ? 1 : 0;
+  return D;
+}
+
+// Common checks of a centroid build (either entry point) and the table slot it
+// writes: version 0 first; then, once tokens are cached, the next free slot
+// (they keep decoding with the tables they were encoded with); on an empty
+// cache the slot in force is rewritten, since no token references it.
+inline qwm_status centroid_build_slot(const qwm_cache* c, const void* K, const void* V, int64_t n,
+                                      int32_t iters, int* slot) {
+  if (!cache_ok(c) || !K || !V) return QWM_ERR_INVALID_ARG;
+  if (((uintptr_t)K % 16) || ((uintptr_t)V % 16)) return QWM_ERR_ALIGNMENT;
+  const Dims D = dims_of(&c->cfg);
+  if (n < D.C || n > D.tcap || iters < 1 || iters > 1000) return QWM_ERR_INVALID_ARG;
+  if (!c->has_centroids) {
+    *slot = 0;
+  } else if (c->len == 0) {
+    *slot = c->cur_cent_version;
+  } else {
+    if (c->n_cent_versions >= c->cfg.max_cent_versions) return QWM_ERR_CAPACITY;
+    *slot = c->n_cent_versions;
+  }
+  return QWM_OK;
+}
+
+// Host state after the tables of `slot` have been enqueued.
+inline void centroid_build_commit(qwm_cache* c, int slot) {
+  c->has_centroids = 1;
+  c->cur_cent_version = slot;
+  if (slot + 1 > c->n_cent_versions) c->n_cent_versions = slot + 1;
+}
+
 // fp32 snapshot A = M / n of head h kept with the refresh state (after the
 // first 32 Ritz-vector columns of the head's d x d fp64 block).
 __host__ __device__ inline float* qsnap_of(double* eigvec, int d, int h) {
@@ -42,6 +108,7 @@ struct CacheView {
   float* wgroup;
   float* basis;
   uint16_t* tokver;
+  uint16_t* centver;
   double* eigvec;
   void* workspace;
 };
@@ -63,10 +130,14 @@ inline CacheView view_of(const qwm_cache* c) {
   v.wgroup = (float*)c->buf.ptr[QWM_BUF_WGROUP];
   v.basis = (float*)c->buf.ptr[QWM_BUF_BASIS];
   v.tokver = (uint16_t*)c->buf.ptr[QWM_BUF_TOKVER];
+  v.centver = (uint16_t*)c->buf.ptr[QWM_BUF_CENTVER];
   v.eigvec = (double*)c->buf.ptr[QWM_BUF_EIGVEC];
   v.workspace = c->buf.ptr[QWM_BUF_WORKSPACE];
   return v;
 }
+
+// The centroid tables of one version: [H][C][d] bf16 starting at the slot.
+__host__ __device__ inline size_t cent_slot_elems(const Dims& D) { return (size_t)D.H * D.C * D.d; }
 
 // ---------------------------------------------------------------- device helpers
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -118,7 +189,7 @@ cudaError_t launch_stats_accumulate(const Dims& D, const uint16_t* Q, int64_t n,
 cudaError_t launch_refresh(const Dims& D, const CacheView& v, int64_t n_total, int version,
                            int warm, cudaStream_t s);
 cudaError_t launch_append(const Dims& D, const CacheView& v, const uint16_t* K, const uint16_t* V,
-                          int64_t n, int64_t t0, int version, cudaStream_t s);
+                          int64_t n, int64_t t0, int version, int cent_version, cudaStream_t s);
 cudaError_t launch_attention(const Dims& D, const CacheView& v, int64_t T, const uint16_t* Q,
                              int64_t nq, float scale, uint16_t* O, const Segment& sg,
                              cudaStream_t s);
@@ -141,6 +212,6 @@ int read_and_clear_append_timeout();
 bool append_tc_supported(const Dims& D);
 cudaError_t launch_append_tc(const Dims& D, const CacheView& v, const uint16_t* K,
                              const uint16_t* V, int64_t n, int64_t t0, int version,
-                             cudaStream_t s);
+                             int cent_version, cudaStream_t s);
 
 }  // namespace qwm

@@ -3,7 +3,8 @@
 //   V'_j = bf16(  c_bj + (mn_g + code_j sc_g) )
 // (QuantWM, "Flickering after quantization?" (SynthePulse), PSAC paragraph:
 // the Key is compensated when the cache is reconstructed; U is the basis
-// version in force when the token was appended.)
+// version in force when the token was appended, c the centroid of the table
+// version in force then.)
 #pragma once
 #include "common.cuh"
 
@@ -18,8 +19,10 @@ struct PackedHead {
   const uint8_t* v_codes;
   const uint16_t* v_params;
   const void* v_idx;
-  const uint16_t* cent_k;   // [C][d]
+  const uint16_t* cent_k;   // [C][d] of table version 0; version v at + v * cstride
   const uint16_t* cent_v;   // [C][d]
+  const uint16_t* centver;  // [tcap] table version of each token
+  size_t cstride;           // elements between table versions (H * C * d)
 };
 
 __device__ __forceinline__ PackedHead packed_head(const CacheView& v, const Dims& D, int h) {
@@ -35,6 +38,8 @@ __device__ __forceinline__ PackedHead packed_head(const CacheView& v, const Dims
   p.v_idx = (const uint8_t*)v.v_idx + base * D.idx_bytes;
   p.cent_k = v.cent_k + (size_t)h * D.C * D.d;
   p.cent_v = v.cent_v + (size_t)h * D.C * D.d;
+  p.centver = v.centver;
+  p.cstride = cent_slot_elems(D);
   return p;
 }
 
@@ -54,7 +59,8 @@ __device__ __forceinline__ float deq_int2(const uint8_t* codes, const uint16_t* 
 __device__ __forceinline__ float key_elem(const PackedHead& p, const Dims& D, const float* U_h,
                                           int64_t t, int j) {
   int a = load_idx(p.k_idx, t, D.idx_bytes);
-  float v = bf2f(p.cent_k[(size_t)a * D.d + j]) + deq_int2(p.k_codes, p.k_params, t, j, D.d, D.ng, D.G);
+  const uint16_t* ck = p.cent_k + (size_t)p.centver[t] * p.cstride;
+  float v = bf2f(ck[(size_t)a * D.d + j]) + deq_int2(p.k_codes, p.k_params, t, j, D.d, D.ng, D.G);
   if (D.r > 0) {
     float cs = h2f(p.k_cscale[t]);
     float corr = 0.0f;
@@ -67,7 +73,8 @@ __device__ __forceinline__ float key_elem(const PackedHead& p, const Dims& D, co
 
 __device__ __forceinline__ float value_elem(const PackedHead& p, const Dims& D, int64_t t, int j) {
   int b = load_idx(p.v_idx, t, D.idx_bytes);
-  return bf2f(p.cent_v[(size_t)b * D.d + j]) + deq_int2(p.v_codes, p.v_params, t, j, D.d, D.ng, D.G);
+  const uint16_t* cv = p.cent_v + (size_t)p.centver[t] * p.cstride;
+  return bf2f(cv[(size_t)b * D.d + j]) + deq_int2(p.v_codes, p.v_params, t, j, D.d, D.ng, D.G);
 }
 
 __device__ __forceinline__ const float* basis_of(const CacheView& v, const Dims& D, int ver, int h) {

@@ -45,30 +45,22 @@ using namespace qwm;
 
 extern "C" qwm_status qwm_build_centroids_noalloc(qwm_cache* c, const void* K, const void* V,
                                                   int64_t n, int32_t iters, void* stream) {
-  if (!c || c->magic != 0x51574d31 || !K || !V) return QWM_ERR_INVALID_ARG;
-  if (((uintptr_t)K % 16) || ((uintptr_t)V % 16)) return QWM_ERR_ALIGNMENT;
-  const qwm_config* cfg = &c->cfg;
-  if (n < cfg->n_centroids || n > c->tcap || iters < 1 || iters > 1000) return QWM_ERR_INVALID_ARG;
-  Dims D;
-  D.H = cfg->heads;
-  D.d = cfg->head_dim;
-  D.C = cfg->n_centroids;
-  D.G = cfg->group;
-  D.M = cfg->n_cand;
-  D.r = cfg->rank;
-  D.ng = cfg->head_dim / cfg->group;
-  D.idx_bytes = cfg->n_centroids <= 256 ? 1 : 2;
+  int slot = 0;
+  const qwm_status st = centroid_build_slot(c, K, V, n, iters, &slot);
+  if (st != QWM_OK) return st;
+  Dims D = dims_of(&c->cfg);
   D.tcap = n;  // the assignment scratch holds n tokens per head, not the capacity
   const size_t need = ((size_t)D.H * D.C * D.d * 4 + 255) / 256 * 256 + (size_t)D.H * n * 4;
   if (need > (size_t)QWM_NOALLOC_SCRATCH_BYTES) return QWM_ERR_CAPACITY;
   void* scratch = scratch_on_current_device();
   if (!scratch) return QWM_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  uint16_t* cent_k = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_K];
-  uint16_t* cent_v = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_V];
+  const size_t off = (size_t)slot * cent_slot_elems(D);
+  uint16_t* cent_k = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_K] + off;
+  uint16_t* cent_v = (uint16_t*)c->buf.ptr[QWM_BUF_CENT_V] + off;
   cudaError_t e = launch_kmeans(D, (const uint16_t*)K, n, iters, cent_k, scratch, s);
   if (e == cudaSuccess) e = launch_kmeans(D, (const uint16_t*)V, n, iters, cent_v, scratch, s);
   if (e != cudaSuccess) return QWM_ERR_CUDA;
-  c->has_centroids = 1;
+  centroid_build_commit(c, slot);
   return QWM_OK;
 }

@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define QWM_ABI_VERSION 1
+#define QWM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define QWM_API __attribute__((visibility("default")))
@@ -64,8 +64,8 @@ typedef enum qwm_status {
 
 /* Quantizer and capacity.  Supported: head_dim 64 or 128; group 16 or 32 and
  * dividing head_dim; 1 <= n_centroids <= 512; 1 <= n_cand <= min(8, C);
- * 0 <= rank <= 16; 1 <= max_versions <= 65535; max_tokens >= 1; flags a
- * combination of the QWM_FLAG_* bits. */
+ * 0 <= rank <= 16; 1 <= max_versions <= 65535; 1 <= max_cent_versions <= 65535;
+ * max_tokens >= 1; flags a combination of the QWM_FLAG_* bits. */
 
 /* QSAC stage 2 with the full quadratic form: each shortlisted centroid c is
  * scored by e^T A e, where e = k - (c + deq(INT2(k - c))) is the Key error
@@ -86,6 +86,7 @@ typedef struct qwm_config {
   int32_t rank;         /* r: PSAC rank                                  */
   int32_t max_versions; /* slots for successive bases U (one per refresh) */
   int32_t flags;        /* QWM_FLAG_* bits (0: the method as described)   */
+  int32_t max_cent_versions; /* slots for successive centroid tables      */
   int64_t max_tokens;   /* cache capacity per head                       */
 } qwm_config;
 
@@ -97,12 +98,14 @@ typedef struct qwm_config {
  *   K_COEF    [H][Tcap][r]     int8    PSAC coefficients
  *   K_CSCALE  [H][Tcap]        fp16    PSAC per-token scale
  *   V_CODES, V_PARAMS, V_IDX   as for K
- *   CENT_K, CENT_V [H][C][d]   bf16    centroid tables
+ *   CENT_K, CENT_V [max_cent_versions][H][C][d] bf16  centroid tables, slot =
+ *                                      centroid-table version
  *   QSTATS    [H][d][d]        fp64    running sum of q q^T
  *   SENS      [H][d]           fp32    s_j = E[q_j^2] in force
  *   WGROUP    [H][ng]          fp32    w_g = sum of s_j over group g
  *   BASIS     [max_versions][H][d][r] fp32  PSAC bases, slot = version
  *   TOKVER    [Tcap]           uint16  basis version of each cached token
+ *   CENTVER   [Tcap]           uint16  centroid-table version of each cached token
  *   EIGVEC    [H][d][d] + [H]  fp64    refresh state: per head the Ritz vectors
  *                                      of the last refresh (first 32 columns of d),
  *                                      then, with QWM_FLAG_QSAC_FULL, A = fp32(M/n)
@@ -114,7 +117,7 @@ typedef enum qwm_buffer_id {
   QWM_BUF_K_CODES = 0, QWM_BUF_K_PARAMS, QWM_BUF_K_IDX, QWM_BUF_K_COEF, QWM_BUF_K_CSCALE,
   QWM_BUF_V_CODES, QWM_BUF_V_PARAMS, QWM_BUF_V_IDX, QWM_BUF_CENT_K, QWM_BUF_CENT_V,
   QWM_BUF_QSTATS, QWM_BUF_SENS, QWM_BUF_WGROUP, QWM_BUF_BASIS, QWM_BUF_TOKVER,
-  QWM_BUF_EIGVEC, QWM_BUF_WORKSPACE, QWM_NBUF
+  QWM_BUF_CENTVER, QWM_BUF_EIGVEC, QWM_BUF_WORKSPACE, QWM_NBUF
 } qwm_buffer_id;
 
 typedef struct qwm_sizes {
@@ -140,6 +143,8 @@ typedef struct qwm_cache {
   int32_t has_centroids;
   int32_t has_eigvec;   /* EIGVEC holds a previous decomposition    */
   int32_t magic;
+  int32_t n_cent_versions;  /* centroid-table versions written      */
+  int32_t cur_cent_version; /* table version used by the next append */
 } qwm_cache;
 
 QWM_API int32_t qwm_abi_version(void);
@@ -156,14 +161,22 @@ QWM_API qwm_status qwm_cache_sizes(const qwm_config* cfg, qwm_sizes* out);
 QWM_API qwm_status qwm_cache_init(qwm_cache* c, const qwm_config* cfg, const qwm_buffers* bufs,
                           void* stream);
 
-/* Centroid tables from the first cached frame (k-means, per head, separately
- * for K and V).  The pages say only that each Key is assigned to a cluster
- * centre kept at higher precision (SynthePulse, QSAC paragraph).  Here:
- * centroid i starts at token floor(i n / C); `iters` Lloyd rounds with fp32
- * squared distances (ties to the lower index) and fp64 means taken in token
- * order; an empty cluster keeps its centroid; the result is rounded to bf16.
+/* Centroid tables (k-means, per head, separately for K and V) from n tokens,
+ * usually the newest frame.  The pages say only that each Key is assigned to a
+ * cluster centre kept at higher precision (SynthePulse, QSAC paragraph).
+ * Here: centroid i starts at token floor(i n / C); `iters` Lloyd rounds with
+ * fp32 squared distances (ties to the lower index) and fp64 means taken in
+ * token order; an empty cluster keeps its centroid; the result is rounded to
+ * bf16.
+ * Versions: the first call writes table version 0.  A later call on a cache
+ * that already holds tokens writes the next version (a centroid refresh under
+ * Key drift; the pages are silent on refreshing the centres): later appends
+ * encode against it, while every cached token keeps decoding with the version
+ * it was encoded with (CENTVER).  A later call on an empty cache rewrites the
+ * version in force, which no token references.
  * K, V: [n][H][d] bf16 device.  Requires n >= C, n <= tcap and
- * 1 <= iters <= 1000.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+ * 1 <= iters <= 1000.  Errors: INVALID_ARG, ALIGNMENT, CAPACITY (all
+ * max_cent_versions slots used), CUDA. */
 QWM_API qwm_status qwm_build_centroids(qwm_cache* c, const void* K, const void* V, int64_t n,
                                int32_t iters, void* stream);
 
@@ -182,7 +195,9 @@ QWM_API qwm_status qwm_update_query_stats(qwm_cache* c, const void* Q, int64_t n
                                   int32_t refresh_basis, void* stream);
 
 /* Quantize and append n tokens at position len (QSAC + INT2 + PSAC for Keys,
- * nearest centroid + INT2 for Values) with the statistics and basis in force.
+ * nearest centroid + INT2 for Values) with the statistics, basis and centroid
+ * tables in force; TOKVER and CENTVER of the new tokens record the basis and
+ * table versions.
  * Codes, indices and INT8 coefficients are bit-identical to the canonical
  * fp32 definition the CPU oracle implements.  K, V: [n][H][d] bf16 device.
  * Errors: INVALID_ARG, ALIGNMENT, CAPACITY (len + n > tcap), STATE (no
@@ -190,8 +205,12 @@ QWM_API qwm_status qwm_update_query_stats(qwm_cache* c, const void* Q, int64_t n
 QWM_API qwm_status qwm_append_kv(qwm_cache* c, const void* K, const void* V, int64_t n, void* stream);
 
 /* O = softmax(scale Q K'^T) V' over all `len` cached tokens, with K', V'
- * reconstructed on the fly from the packed cache (each key with the basis
- * version in force when it was appended).  No mask.  Q, O: [n_q][H][d] bf16
+ * reconstructed on the fly from the packed cache (each key with the basis and
+ * centroid-table versions in force when it was appended):
+ *   K'_j = bf16(C_K[a]_j + (mn + code_j sc) + sum_i U_ji (c8_i cs)),
+ *   V'_j = bf16(C_V[b]_j + (mn + code_j sc)),
+ * each element rounded once, so the attention reads exactly the bf16 cache
+ * that qwm_reconstruct returns (up to the order of the fp32 sum).  No mask.  Q, O: [n_q][H][d] bf16
  * device (O written, fp32 accumulation).  scale <= 0 selects 1/sqrt(d).
  * Errors: INVALID_ARG, ALIGNMENT, STATE (empty cache), CUDA. */
 QWM_API qwm_status qwm_attention(const qwm_cache* c, const void* Q, int64_t n_q, float scale, void* O,
@@ -239,10 +258,11 @@ QWM_API qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q
  * frameworks own the GPU memory budget and hand out fixed buffers; code running
  * inside them may not call cudaMalloc/cudaFree (these synchronize the device
  * and fragment the host's pool).  This variant writes the same centroid tables
- * as qwm_build_centroids but takes its scratch from one fixed device array
- * inside the library instead of the cache's WORKSPACE buffer, and allocates
- * nothing.  The array is QWM_NOALLOC_SCRATCH_BYTES long and stays allocated on
- * every GPU that loads the library until the process exits; the call needs
+ * as qwm_build_centroids (with the same version rules) but takes its scratch
+ * from one fixed device array inside the library instead of the cache's
+ * WORKSPACE buffer, and allocates nothing.  The array is
+ * QWM_NOALLOC_SCRATCH_BYTES long and stays allocated on every GPU that loads
+ * the library until the process exits; the call needs
  * 4*H*C*d bytes (rounded up to 256) + 4*H*n bytes of it and returns
  * QWM_ERR_CAPACITY when that exceeds the array.  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress, with that device
@@ -251,7 +271,8 @@ QWM_API qwm_status qwm_top1_shift(const qwm_cache* c, const void* Q, int64_t n_q
  * share the one array and it keeps the last call's contents: calls whose
  * kernels can overlap on the GPU (several streams of one device) race, and the
  * caller must order them.  Arguments and other errors as for
- * qwm_build_centroids: INVALID_ARG, ALIGNMENT, CAPACITY, CUDA. */
+ * qwm_build_centroids: INVALID_ARG, ALIGNMENT, CAPACITY (also when every
+ * table slot is used), CUDA. */
 QWM_API qwm_status qwm_build_centroids_noalloc(qwm_cache* c, const void* K, const void* V,
                                                int64_t n, int32_t iters, void* stream);
 

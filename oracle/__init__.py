@@ -251,6 +251,16 @@ def reconstruct_key_f64(c, codes, params, coef, cscale, U, G) -> np.ndarray:
     return out
 
 
+def reconstruct_value(c, codes, params, G) -> np.ndarray:
+    """V' = bf16(c + deq(codes, params)) of one Value row, as bf16 bits."""
+    c = np.ascontiguousarray(c, np.uint16)
+    d = c.shape[0]
+    out = np.zeros(d, np.uint16)
+    lib().qo_reconstruct_value(_p(c), _p(np.ascontiguousarray(codes, np.uint8)),
+                               _p(np.ascontiguousarray(params, np.uint16)), d, G, _p(out))
+    return out
+
+
 def attention_head(Q, Kp, Vp, scale):
     """Q [nq][d], K', V' [T][d] (bf16 bits) -> O [nq][d] fp64."""
     Q = np.ascontiguousarray(Q, np.uint16); Kp = np.ascontiguousarray(Kp, np.uint16)
@@ -446,8 +456,8 @@ class OracleCache:
         """O[rows][heads][d] in fp64 for the given query rows (default all)."""
         scale = 1.0 / math.sqrt(self.d) if scale is None else scale
         rows = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
-        heads = range(self.H) if heads is None else heads
-        out = np.zeros((len(rows), len(list(heads)), self.d), np.float64)
+        heads = list(range(self.H) if heads is None else heads)
+        out = np.zeros((len(rows), len(heads), self.d), np.float64)
         for i, h in enumerate(heads):
             Kp, Vp = self.reconstruct(h)
             out[:, i, :] = attention_head(Q[rows, h, :], Kp, Vp, scale)

@@ -72,9 +72,17 @@ def encode_frames(args):
     return {k: getattr(oc, k)[0, :n].copy() for k in fields}
 
 
+def attention_rows(args):
+    """Oracle fp64 attention of query rows Qs [n][d] over K', V' [T][d]."""
+    Qs, Kp, Vp, scale = args
+    return oracle.attention_head(Qs, Kp, Vp, scale)
+
+
 # ----------------------------------------------------------------- driver
-def run_full(name, heads, attn_frames, attn_rows, seed=None):
-    """Run configuration `name` at full size; returns measured discrepancies."""
+def run_full(name, heads, attn_frames, attn_rows, seed=None, full_rows_head=None):
+    """Run configuration `name` at full size; returns measured discrepancies.
+    With `full_rows_head` (one of `heads`), every query row of that head is also
+    compared at the last frame (which includes the last, partial, CTA of rows)."""
     import torch
 
     import bit_kv_cache_23_b200 as q
@@ -122,6 +130,13 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None):
                 Og = syn.bf16_bits_to_f32(u16(Od))
                 attn_out[f] = (rows, Q[rows][:, heads, :].copy(), Og[rows][:, heads, :].copy(),
                                g.len)
+            if full_rows_head is not None and f == F - 1:
+                if f not in attn_frames:
+                    Od = g.attention(Qd)
+                    torch.cuda.synchronize()
+                    assert q.qwm_device_status() == 0, "a bounded device wait timed out"
+                    Og = syn.bf16_bits_to_f32(u16(Od))
+                full_rows = (Q[:, full_rows_head, :].copy(), Og[:, full_rows_head, :].copy())
         torch.cuda.synchronize()
         out["refreshes"] = len(refreshes)
         CKg = g.view("cent_k").cpu().numpy().view(np.uint16)
@@ -181,4 +196,16 @@ def run_full(name, heads, attn_frames, attn_rows, seed=None):
             Oref = oc.attention(Qs[:, hi:hi + 1, :])
             mx, mean = attention_error(Og[:, hi:hi + 1, :], Oref)
             out["attn"].append((f, h, mx, mean))
+        if h == full_rows_head:
+            oc.len = F * N
+            Kp, Vp = oc.reconstruct(0)
+            Qh, Oh = full_rows
+            step = 64
+            tasks = [(np.ascontiguousarray(Qh[i:i + step]), Kp, Vp, 1.0 / math.sqrt(c.head_dim))
+                     for i in range(0, Qh.shape[0], step)]
+            with pool() as P:
+                Oref = np.concatenate(P.map(attention_rows, tasks, chunksize=1))
+            mx, mean = attention_error(Oh, Oref)
+            out["attn"].append(("all rows", h, mx, mean))
+            out["full_rows"] = Qh.shape[0]
     return out

@@ -4,6 +4,7 @@ and invalid calls return the documented status before touching the device."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -25,13 +26,13 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 10
     for n in names:
         assert hasattr(L, n), n
-    assert q.qwm_abi_version() == 1
+    assert q.qwm_abi_version() == 2
     assert q.qwm_status_string(3) == "capacity exceeded"
 
 
 def _cfg(**kw):
     base = dict(heads=40, head_dim=128, n_centroids=256, group=32, n_cand=4, rank=8,
-                max_versions=64, flags=0, max_tokens=37440)
+                max_versions=64, flags=0, max_cent_versions=1, max_tokens=37440)
     base.update(kw)
     return q.qwm_config(**base)
 
@@ -62,7 +63,8 @@ def test_sizes_follow_layout():
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(group=8), dict(n_centroids=0),
                                  dict(n_centroids=513), dict(n_cand=9), dict(n_cand=300),
                                  dict(rank=17), dict(max_versions=0), dict(flags=2), dict(flags=-1),
-                                 dict(max_tokens=0), dict(heads=0)])
+                                 dict(max_tokens=0), dict(heads=0), dict(max_cent_versions=0),
+                                 dict(max_cent_versions=65536)])
 def test_invalid_configs_rejected(bad):
     out = q.qwm_sizes()
     st = q.lib().qwm_cache_sizes(ctypes.byref(_cfg(**bad)), ctypes.byref(out))
@@ -138,11 +140,73 @@ def test_attention_ext_argument_checks():
     assert L.qwm_attention_ext(ctypes.byref(c), p, 0, p, p, 8, 0.0, p, None, None) == 0
 
 
+def _probe():
+    """Compile tests/c/abi_probe.c against include/qwm.h with gcc, link it to
+    libqwm.so and return its "key value" lines as a dict."""
+    import tempfile
+    lib = q.lib()  # noqa: F841 - the library is built
+    libdir = os.path.dirname(q.LIB_PATH)
+    with tempfile.TemporaryDirectory() as td:
+        exe = os.path.join(td, "abi_probe")
+        subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Werror", "-I",
+                               os.path.join(ROOT, "include"),
+                               os.path.join(ROOT, "tests", "c", "abi_probe.c"), "-L", libdir,
+                               "-l:libqwm.so", "-Wl,-rpath," + libdir, "-o", exe])
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    d = {}
+    for line in out.splitlines():
+        k, v = line.rsplit(" ", 1) if not line.startswith("status_") else line.split(" ", 1)
+        d[k] = v
+    return d
+
+
 def test_struct_layout_matches_header():
-    assert ctypes.sizeof(q.qwm_config) == 40
-    assert ctypes.sizeof(q.qwm_buffers) == 8 * q.NBUF
-    assert ctypes.sizeof(q.qwm_cache) == 40 + 8 * q.NBUF + 24 + 24
-    assert len(q.BUFFER_NAMES) == q.NBUF == 17
+    """The binding's ctypes structures, buffer order and status strings agree
+    with what a C compiler makes of include/qwm.h, and qwm_cache_sizes returns
+    the same sizes through the header as through the binding."""
+    d = _probe()
+    assert int(d["abi_macro"]) == int(d["abi_lib"]) == q.qwm_abi_version() == 2
+    assert int(d["nbuf"]) == q.NBUF == len(q.BUFFER_NAMES) == 18
+    assert int(d["noalloc_bytes"]) == q.QWM_NOALLOC_SCRATCH_BYTES
+    assert int(d["flag_qsac_full"]) == q.QWM_FLAG_QSAC_FULL
+    for name, st in (("qwm_config", q.qwm_config), ("qwm_sizes", q.qwm_sizes),
+                     ("qwm_buffers", q.qwm_buffers), ("qwm_cache", q.qwm_cache)):
+        assert int(d[f"size {name}"]) == ctypes.sizeof(st), name
+    for key, v in d.items():
+        if key.startswith("off "):
+            sname, field = key[4:].split(".")
+            st = getattr(q, sname)
+            assert getattr(st, field).offset == int(v), key
+    for e in ("K_CODES", "CENT_K", "TOKVER", "CENTVER", "WORKSPACE"):
+        assert q.BUFFER_NAMES[int(d[f"enum QWM_BUF_{e}"])] == e.lower(), e
+    s = q.qwm_cache_sizes(_cfg(max_cent_versions=2))
+    assert int(d["sizes_status"]) == 0 and int(d["sizes_bad_status"]) == 1
+    assert int(d["sizes_tcap"]) == s.tcap and int(d["sizes_bpth"]) == s.bytes_per_token_head
+    for i in range(q.NBUF):
+        assert int(d[f"sizes_bytes_{i}"]) == s.bytes[i], q.BUFFER_NAMES[i]
+    assert d["status_capacity"] == q.qwm_status_string(3) == "capacity exceeded"
+
+
+def test_centroid_versions_sizes_and_capacity():
+    """Centroid tables take one [H][C][d] bf16 slot per version and CENTVER one
+    uint16 per token; a rebuild on a cache that holds tokens needs a free slot
+    (QWM_ERR_CAPACITY otherwise, with the cache unchanged)."""
+    s1 = q.qwm_cache_sizes(_cfg())
+    s3 = q.qwm_cache_sizes(_cfg(max_cent_versions=3))
+    ck = q.BUFFER_NAMES.index("cent_k")
+    assert s1.bytes[ck] == 40 * 256 * 128 * 2 and s3.bytes[ck] == 3 * s1.bytes[ck]
+    assert s1.bytes[q.BUFFER_NAMES.index("centver")] == s1.tcap * 2
+    L = q.lib()
+    p = ctypes.c_void_p(0x200000)
+    c = _fake_cache(has_centroids=1, len=100, n_cent_versions=1)
+    assert L.qwm_build_centroids(ctypes.byref(c), p, p, 300, 10, None) == 3
+    assert L.qwm_build_centroids_noalloc(ctypes.byref(c), p, p, 300, 10, None) == 3
+    assert c.n_cent_versions == 1 and c.cur_cent_version == 0
+    # misaligned inputs and bad sizes are refused by both entry points alike
+    for fn in (L.qwm_build_centroids, L.qwm_build_centroids_noalloc):
+        assert fn(ctypes.byref(c), ctypes.c_void_p(0x200008), p, 300, 10, None) == 2
+        assert fn(ctypes.byref(c), p, p, 300, 0, None) == 1
+        assert fn(ctypes.byref(c), p, p, 2000, 10, None) == 1
 
 
 def test_binding_refuses_cpu_tensors():

@@ -31,8 +31,12 @@ def _check(out):
 
 
 def test_480p_full_size():
-    """40 heads x 128, 24 frames x 1560 tokens, C=256: heads 0, 23, 39."""
-    _check(run_full("480p", heads=[0, 23, 39], attn_frames={0, 11, 23}, attn_rows=16))
+    """40 heads x 128, 24 frames x 1560 tokens, C=256: heads 0, 23, 39; at the last
+    frame all 1560 query rows of head 23 (the last CTA holds rows 1536-1559)."""
+    out = run_full("480p", heads=[0, 23, 39], attn_frames={0, 11, 23}, attn_rows=16,
+                   full_rows_head=23)
+    _check(out)
+    assert out["full_rows"] == 1560
 
 
 def test_720p_full_size():

@@ -103,13 +103,18 @@ def test_qvg_mode_without_statistics():
         assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (d, err.max(), err.mean())
 
 
-@pytest.mark.parametrize("d,C,G,M,r", [(128, 64, 32, 4, 8), (64, 16, 16, 4, 4)])
-def test_full_quadratic_qsac(d, C, G, M, r):
+@pytest.mark.parametrize("d,C,G,M,r,n,nqa", [(128, 64, 32, 4, 8, 300, 300),
+                                              (128, 64, 32, 4, 8, 700, 200),
+                                              (64, 16, 16, 4, 4, 700, 200)])
+def test_full_quadratic_qsac(d, C, G, M, r, n, nqa):
     """QSAC stage 2 by e^T A e (the full-quadratic option, CUDA-core append): the
     GPU's snapshot A = fp32(M / n) equals the oracle's bit for bit, and every
-    packed field matches the oracle's encoding with the same option."""
+    packed field matches the oracle's encoding with the same option.  The first
+    case (900 cached keys, 300 queries of norm ~10, outlier channels, a peaky
+    softmax) is the one where attention is most sensitive to how each K' element
+    is rounded: the attention must read exactly the bf16 reconstruction."""
     q = pytest.importorskip("bit_kv_cache_23_b200")
-    H, n, F = 2, 700, 3
+    H, F = 2, 3
     g = q.QuantKVCache(H, d, C, G, M, r, F * n, max_versions=F + 2, qsac_full=True)
     oc = oracle.OracleCache(H, d, C, G, M, r, F * n, qsac_full=True)
     rng = np.random.default_rng(5000 + d)
@@ -144,7 +149,7 @@ def test_full_quadratic_qsac(d, C, G, M, r):
         oc.append_kv(K, V)
         assert compare_packed(g, oc, t0, g.len) == {}, f
     assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
-    Qa = Q[:200]
+    Qa = np.ascontiguousarray(Q[:nqa])
     O = g.attention(to_dev(Qa))
     torch.cuda.synchronize()
     assert q.qwm_device_status() == 0
@@ -257,3 +262,94 @@ def test_head128_shapes(G, C, M, r):
     Oref = oc.attention(Q, rows=rows)
     err = np.abs(syn.bf16_bits_to_f32(u16(O))[rows] - Oref)
     assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
+
+
+def _edge_tables(rng, C, d):
+    """Centroid tables built to hit the append's corner cases: rows 0..63 are
+    sign flips of one vector (a zero key is equally far from all 64, so far more
+    than 16 centroids survive the tensor-core prefilter and the full exact
+    rescoring runs), rows 64..66 are one row repeated (exact distance ties,
+    which go to the lower index), row 67 is all zero, the rest Gaussian with
+    outlier channels."""
+    base = 1.0 + np.arange(d) / d
+    signs = np.where(rng.integers(0, 2, (64, d)) == 1, 1.0, -1.0)
+    T = rng.standard_normal((C, d)) * np.where(np.arange(d) % 17 == 0, 6.0, 1.0)
+    T[:64] = signs * base
+    T[65] = T[64]
+    T[66] = T[64]
+    T[67] = 0.0
+    return _bf_rows(T)
+
+
+def _bf_rows(x):
+    return syn.f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def _edge_tokens(rng, tab, n, d):
+    """n rows mixing: zero rows, rows equal to a centroid (incl. the repeated
+    one), rows with constant and all-zero 32-channel groups, rows with channels
+    scaled by 100, rows next to the repeated centroid, and Gaussian rows."""
+    X = rng.standard_normal((n, d)) * np.where(np.arange(d) % 17 == 0, 6.0, 1.0)
+    tf = syn.bf16_bits_to_f32(tab).astype(np.float64)
+    kinds = np.arange(n) % 8
+    for i in range(n):
+        k = kinds[i]
+        if k == 0:
+            X[i] = 0.0
+        elif k == 1:
+            X[i] = tf[rng.integers(0, tab.shape[0])]
+        elif k == 2:
+            X[i] = tf[64]
+        elif k == 3:
+            X[i, :32] = 0.25
+            X[i, 64:96] = 0.0
+        elif k == 4:
+            X[i, rng.permutation(d)[:5]] *= 100.0
+        elif k == 5:
+            X[i] = tf[64] + 0.01 * rng.standard_normal(d)
+    return _bf_rows(X)
+
+
+@pytest.mark.parametrize("C", [256, 512])
+def test_append_tc_edge_cases(C):
+    """head_dim 128 (the tensor-core append): exact distance ties between
+    distinct centroid rows, keys equal to a centroid, zero and constant groups,
+    outlier channels scaled by 100 against the prefilter's error bound, and the
+    more-than-16-survivors fallback (zero keys against 64 equidistant rows):
+    every packed field bit for bit against the oracle."""
+    q = pytest.importorskip("bit_kv_cache_23_b200")
+    H, d, G, M, r, n = 2, 128, 32, 4, 8, 640
+    rng = np.random.default_rng(9000 + C)
+    g = q.QuantKVCache(H, d, C, G, M, r, 2 * n, max_versions=4)
+    oc = oracle.OracleCache(H, d, C, G, M, r, 2 * n)
+    K0 = _bf_rows(rng.standard_normal((C, H, d)))
+    g.build_centroids(to_dev(K0), to_dev(K0), iters=1)      # sets the state; tables replaced
+    CK = np.stack([_edge_tables(rng, C, d) for _ in range(H)])
+    CV = np.stack([_edge_tables(rng, C, d) for _ in range(H)])
+    g.view("cent_k").copy_(torch.from_numpy(CK.view(np.int16)))
+    g.view("cent_v").copy_(torch.from_numpy(CV.view(np.int16)))
+    oc.set_state(CK=CK, CV=CV)
+    basis = np.linalg.qr(rng.standard_normal((d, 8)))[0]
+    Mref = {h: np.zeros((d, d)) for h in range(H)}
+    rep = new_state_report()
+    for f in range(2):
+        Q = _bf_rows(3.0 * rng.standard_normal((300, H, 8)) @ basis.T
+                     + 0.5 * rng.standard_normal((300, H, d)))
+        g.update_query_stats(to_dev(Q), refresh_basis=True)
+        for h in range(H):
+            oracle.stats_accumulate(Q[:, h, :], Mref[h])
+        st = refresh_from_oracle(g, Mref, 300 * (f + 1), range(H), r, G, rep)
+        s, w, U = stack_state(st, H)
+        oc.set_state(s=s, w=w, U=U)
+        K = np.stack([_edge_tokens(rng, CK[h], n, d) for h in range(H)], axis=1)
+        V = np.stack([_edge_tokens(rng, CV[h], n, d) for h in range(H)], axis=1)
+        t0 = g.len
+        g.append_kv(to_dev(K), to_dev(V))
+        oc.append_kv(K, V)
+        assert compare_packed(g, oc, t0, g.len) == {}, f
+        assert q.qwm_device_status() == 0
+    assert rep["stats_mismatch"] == 0 and rep["sw_mismatch"] == 0, rep
+    # the zero keys really did meet 64 equidistant centroids
+    kz = np.zeros(d, np.uint16)
+    _, D = oracle.qsac_shortlist(kz, CK[0], s[0], M)
+    assert np.count_nonzero(D[:64] == D[:64].min()) == 64

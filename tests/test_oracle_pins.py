@@ -389,6 +389,98 @@ def test_kmeans_bruteforce_tiny():
         assert np.allclose(syn.bf16_bits_to_f32(cent), ce, rtol=1e-2, atol=1e-2)
 
 
+# ----------------------------------------------------------------- Values
+def _grid_rows(rng, shape, step=0.25, lim=2.0):
+    """bf16 rows on a coarse grid: differences, squares and sums of up to 128
+    of them are exact in fp32, so the oracle's fp32 fold equals the exact
+    distance and every tie it meets is a real tie."""
+    k = int(round(lim / step))
+    return _bf(rng.integers(-k, k + 1, shape).astype(np.float64) * step)
+
+
+def test_value_choice_is_bruteforce_nearest_centroid():
+    """qo_encode_value picks argmin_i sum_j (v_j - c_ij)^2 over all C centroids
+    (numpy fp64 brute force), ties to the lower index, and codes the fp32
+    residual v - c of that centroid with the INT2 rule.  3000 grid cases (exact
+    arithmetic; half of them with a duplicated nearest row, an exact tie that
+    must go to the lower index) plus 1000 Gaussian cases checked against the
+    fp32 fold's error bound."""
+    rng = np.random.default_rng(41)
+    ties = 0
+    for case in range(3000):
+        d = (16, 32, 64, 128)[case % 4]
+        G = 16 if d == 16 else (16, 32)[case % 2]
+        C = int(rng.integers(2, 40))
+        CV = _grid_rows(rng, (C, d))
+        v = _grid_rows(rng, d)
+        if case % 2:
+            i, j = sorted(rng.choice(C, 2, replace=False))
+            CV[j] = CV[i]
+            # v one grid step from the duplicated row: the pair is nearest
+            v = CV[i].copy()
+            v[int(rng.integers(d))] = _bf([syn.bf16_bits_to_f32(v[:1])[0] + 0.25])[0]
+        enc = oracle.encode_value(v, CV, G)
+        dist = ((syn.bf16_bits_to_f32(CV).astype(np.float64)
+                 - syn.bf16_bits_to_f32(v).astype(np.float64)) ** 2).sum(1)
+        want = int(np.argmin(dist))            # first index among equal minima
+        ties += int(np.count_nonzero(dist == dist.min()) > 1)
+        assert enc["idx"] == want, (case, enc["idx"], want)
+        rho = (syn.bf16_bits_to_f32(v) - syn.bf16_bits_to_f32(CV[want])).astype(np.float32)
+        codes, params = oracle.int2_encode(rho, G)
+        assert np.array_equal(enc["codes"], codes) and np.array_equal(enc["params"], params)
+    assert ties >= 1500            # the duplicated rows did produce exact ties
+    for case in range(1000):
+        d, G, C = 128, 32, 64
+        CV = _bf(rng.standard_normal((C, d)))
+        v = _bf(rng.standard_normal(d) * 1.3)
+        enc = oracle.encode_value(v, CV, G)
+        dist = ((syn.bf16_bits_to_f32(CV).astype(np.float64)
+                 - syn.bf16_bits_to_f32(v).astype(np.float64)) ** 2).sum(1)
+        # a left-to-right fp32 fold of d non-negative terms is within
+        # (d + 2) 2^-24 of the exact sum, relatively
+        tol = (d + 2) * 2.0 ** -24 * dist
+        assert dist[enc["idx"]] <= dist.min() + tol[enc["idx"]] + tol.min()
+        order = np.argsort(dist, kind="stable")
+        if dist[order[1]] - dist[order[0]] > 2 * tol[order[1]]:
+            assert enc["idx"] == order[0], case
+
+
+def test_value_reconstruction_hand_worked_cases():
+    """V' = bf16(c + mn_g + code_j sc_g) on fixtures worked out by hand: a
+    nonzero centroid with distinct group parameters (a dropped centroid or a
+    wrong group index changes every entry) and the single round-to-nearest-even
+    of the sum at exact bf16 midpoints."""
+    with open(os.path.join(GOLDEN, "value_reconstruct_hand_worked.json")) as f:
+        gold = json.load(f)
+    G = gold["group"]
+    for case in gold["cases"]:
+        c = _bf(case["centroid"])
+        assert np.array_equal(syn.bf16_bits_to_f32(c), np.array(case["centroid"], np.float32))
+        out = oracle.reconstruct_value(c, np.array(case["codes"], np.uint8),
+                                       np.array(case["params"], np.uint16), G)
+        got = syn.bf16_bits_to_f32(out)
+        assert np.array_equal(got, np.array(case["expected"], np.float32)), case["derivation"]
+
+
+@pytest.mark.parametrize("d,G,C", [(64, 16, 16), (128, 32, 256)])
+def test_value_round_trip_bound(d, G, C):
+    """Encoding then reconstructing a Value leaves |v - V'| <= sc_g / 2 plus half
+    a bf16 ulp of V' on every channel: the INT2 step bound of the residual and
+    the one rounding of the sum."""
+    rng = np.random.default_rng(43 + d)
+    CV = _bf(rng.standard_normal((C, d)))
+    for _ in range(300):
+        v = _bf(rng.standard_normal(d) * rng.uniform(0.2, 4.0))
+        enc = oracle.encode_value(v, CV, G)
+        out = oracle.reconstruct_value(CV[enc["idx"]], enc["codes"], enc["params"], G)
+        vf = syn.bf16_bits_to_f32(v).astype(np.float64)
+        of = syn.bf16_bits_to_f32(out).astype(np.float64)
+        sc = np.repeat(oracle.f16_bits_to_f32(enc["params"][1::2]).astype(np.float64), G)
+        half_ulp = np.where(of != 0, 2.0 ** (np.floor(np.log2(np.abs(of) + 1e-300)) - 8), 2.0 ** -134)
+        slack = 4 * 2.0 ** -24 * (np.abs(vf) + np.abs(of))      # fp32 residual and decode
+        assert np.all(np.abs(vf - of) <= sc / 2 + half_ulp + slack)
+
+
 # ----------------------------------------------------------------- attention, compression
 def test_attention_unquantized_matches_sdpa_fp64():
     rng = np.random.default_rng(31)

@@ -45,10 +45,24 @@ def test_noalloc_matches_workspace_build_on_two_calls():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # 64 heads x 512 centroids x 128 channels x 4 B = 16.8 MB > 16 MiB
-    g = q.QuantKVCache(64, 128, 512, 32, 4, 8, 1024, max_versions=2)
-    K = torch.zeros((600, 64, 128), dtype=torch.bfloat16, device="cuda")
+    # fp32 centroids 4 H C d + assignments 4 H n must fit the 16 MiB array.
+    # 32 heads x 512 x 128: 8 MiB of centroids, so n = 65536 tokens fill the
+    # array exactly and one more token does not fit.
+    H, C, d = 32, 512, 128
+    n_fit = (q.QWM_NOALLOC_SCRATCH_BYTES - 4 * H * C * d) // (4 * H)
+    assert n_fit == 65536
+    g = q.QuantKVCache(H, d, C, 32, 4, 8, n_fit + 1, max_versions=2)
+    K = torch.zeros((n_fit + 1, H, d), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(q.QwmError) as ei:
         q.qwm_build_centroids_noalloc(g.c, K, K, 1)
     assert ei.value.status == 3  # QWM_ERR_CAPACITY
     assert g.c.has_centroids == 0
+    q.qwm_build_centroids_noalloc(g.c, K[:n_fit], K[:n_fit], 1)   # exactly the array
+    torch.cuda.synchronize()
+    assert g.c.has_centroids == 1 and q.qwm_device_status() == 0
+    # the centroid part alone beyond the array: 64 heads x 512 x 128 x 4 B = 16 MiB
+    g2 = q.QuantKVCache(64, d, C, 32, 4, 8, 1024, max_versions=2)
+    K2 = torch.zeros((600, 64, d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(q.QwmError) as ei:
+        q.qwm_build_centroids_noalloc(g2.c, K2, K2, 1)
+    assert ei.value.status == 3
