@@ -178,7 +178,7 @@ class Workload:
         self.cache = q.QuantKVCache(len(self.heads), c.head_dim, c.n_centroids, c.group,
                                     c.n_cand, c.rank, c.total_tokens,
                                     max_versions=c.frames // c.refresh_every + extra_versions + 4,
-                                    device=device)
+                                    device=device, max_queries=c.q_rows)
         src = syn.FrameSource(c)
         self.src = src
         self.pool = []

@@ -22,7 +22,7 @@ __all__ = [
     "lib", "qwm_abi_version", "qwm_status_string", "qwm_cache_sizes", "qwm_cache_init",
     "qwm_build_centroids", "qwm_build_centroids_noalloc", "qwm_update_query_stats", "qwm_append_kv", "qwm_attention",
     "qwm_attention_ext", "qwm_reconstruct", "qwm_top1_shift", "qwm_device_status", "QuantKVCache",
-    "QWM_FLAG_QSAC_FULL", "QWM_NOALLOC_SCRATCH_BYTES",
+    "QWM_FLAG_QSAC_FULL", "QWM_NOALLOC_SCRATCH_BYTES", "QWM_ATTN_MAX_SPLIT",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +30,7 @@ LIB_PATH = os.path.join(_HERE, "libqwm.so")
 
 QWM_FLAG_QSAC_FULL = 1   # QSAC stage 2 by the full quadratic form e^T A e
 QWM_NOALLOC_SCRATCH_BYTES = 16 << 20   # fixed scratch of qwm_build_centroids_noalloc
+QWM_ATTN_MAX_SPLIT = 6                 # key ranges an attention call may be split into
 
 BUFFER_NAMES = ["k_codes", "k_params", "k_idx", "k_coef", "k_cscale", "v_codes", "v_params",
                 "v_idx", "cent_k", "cent_v", "qstats", "sens", "wgroup", "basis", "tokver",
@@ -45,7 +46,8 @@ class qwm_config(ctypes.Structure):
                 ("n_centroids", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("n_cand", ctypes.c_int32), ("rank", ctypes.c_int32),
                 ("max_versions", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("max_cent_versions", ctypes.c_int32), ("max_tokens", ctypes.c_int64)]
+                ("max_cent_versions", ctypes.c_int32), ("max_queries", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int64)]
 
 
 class qwm_sizes(ctypes.Structure):
@@ -251,13 +253,14 @@ class QuantKVCache:
 
     def __init__(self, heads: int, head_dim: int, n_centroids: int, group: int, n_cand: int,
                  rank: int, max_tokens: int, max_versions: int = 1024, device="cuda",
-                 stream=None, qsac_full: bool = False, max_cent_versions: int = 1):
+                 stream=None, qsac_full: bool = False, max_cent_versions: int = 1,
+                 max_queries: int = 0):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("QuantKVCache lives on a CUDA device")
         flags = QWM_FLAG_QSAC_FULL if qsac_full else 0
         self.cfg = qwm_config(heads, head_dim, n_centroids, group, n_cand, rank, max_versions,
-                              flags, max_cent_versions, max_tokens)
+                              flags, max_cent_versions, max_queries, max_tokens)
         self.sizes = qwm_cache_sizes(self.cfg)
         self.buffers = {}
         bufs = qwm_buffers()

@@ -58,7 +58,9 @@ qwm_status qwm_cache_sizes(const qwm_config* cfg, qwm_sizes* out) {
   out->bytes[QWM_BUF_TOKVER] = (uint64_t)D.tcap * 2;
   out->bytes[QWM_BUF_CENTVER] = (uint64_t)D.tcap * 2;
   out->bytes[QWM_BUF_EIGVEC] = (uint64_t)D.H * D.d * D.d * 8 + (uint64_t)D.H * 8;
-  out->bytes[QWM_BUF_WORKSPACE] = kmeans_workspace_bytes(D);
+  const size_t ws_attn = attn_partial_bytes(D, cfg->max_queries, QWM_ATTN_MAX_SPLIT);
+  const size_t ws_km = kmeans_workspace_bytes(D);
+  out->bytes[QWM_BUF_WORKSPACE] = ws_km > ws_attn ? ws_km : ws_attn;
   out->bytes_per_token_head = 2 * (D.d / 4 + 4 * D.ng + D.idx_bytes) + D.r + 2;
   return QWM_OK;
 }

@@ -9,27 +9,36 @@
 // fp32 and rounded once to bf16, so the tensor cores read the same bf16 cache
 // that the reconstruction returns.
 //
-// One CTA per (head, 256 query rows = two 128-row Q tiles); 608 threads:
-//   warps 0-7   softmax: warp w serves Q tile w/4, TMEM lanes 32(w%4)..+31 =
-//               query rows; online softmax in the log2 domain with a lazy
-//               rescale of O, P written back into TMEM over S (bf16 pairs).
-//   warps 8-15  dequant: warp 8+s owns channels [16s, 16s+16) of every key of
-//               a 64-key tile (lane l: keys l and l+32); it gathers those
-//               centroid chunks with 16-byte async copies two tiles ahead, then
-//               rewrites them in place as K' / V' (bf16, the 128B-swizzled
-//               layouts the UMMA descriptors read).  All lanes of a warp read the
-//               same basis rows, so the compensation's loads are broadcasts.
-//   warps 16-17 MMA: one issuing thread per Q tile, S = Q K'^T then, once the
-//               softmax has written P, O += P V'; the two threads interleave on
-//               the tensor pipe, which works on one Q tile while the softmax
-//               works on the other.
+// A pair of CTAs on two SMs (a cluster of 2) serves one (head, row block):
+// each CTA holds up to 256 query rows (two 128-row Q tiles, one per TMEM lane),
+// and the even CTA issues M = 256 tensor-core MMAs (tcgen05 cta_group::2) that
+// cover the rows of both.  The B operands of those MMAs are split between the
+// two CTAs' shared memory, so each CTA decodes only half of every key tile: K'
+// for its 32 of the tile's 64 keys (all 128 channels) and V' for its 64 of the
+// 128 channels (all 64 keys).  A pair thus decodes each key once for up to 512
+// query rows, and each SM decodes half a tile per tile.
+//
+// 608 threads per CTA:
+//   warps 0-7   softmax of this CTA's rows: warp w serves Q tile w/4, TMEM
+//               lanes 32(w%4)..+31; online softmax in the log2 domain with a
+//               lazy rescale of O, P written back into TMEM over S (bf16 pairs).
+//   warps 8-15  dequant: warp 8+s owns channels [16s, 16s+16) of this CTA's 32
+//               keys of K' (lane = key) and channel chunk s of this CTA's half of
+//               V' for keys lane and lane+32; it gathers the centroid chunks with
+//               16-byte async copies two tiles ahead, then rewrites them in place
+//               (bf16, the 128B-swizzled layouts the UMMA descriptors read).  All
+//               lanes of a warp read the same basis rows, so the compensation's
+//               loads are broadcasts.
+//   warps 16-17 MMA (even CTA only): one issuing thread per Q tile, S = Q K'^T
+//               then, once the softmax of both CTAs has written P, O += P V';
+//               completions are signalled to both CTAs (multicast commits).
 //   warp 18     producer: bulk-copies (TMA engine) the tile's packed codes,
 //               group parameters, coefficients, basis and table versions and
-//               centroid indices into the packed-field ring.
-// TMEM (512 columns): per Q tile p, Q at 256p (64 columns of bf16 pairs), S/P
-// at 256p+64, O at 256p+128.  Shared memory: a ring of 5 K' / V' stages
-// (released by the MMA) and a ring of 5 packed-field stages (released by the
-// dequant).
+//               centroid indices into this CTA's packed-field ring.
+// TMEM (512 columns, the same in both CTAs): per Q tile p, Q at 256p (64
+// columns of bf16 pairs), S/P at 256p+64, O at 256p+128.  Shared memory: a ring
+// of K' / V' half-tile stages (released by the MMA commits) and a ring of
+// packed-field stages (released by the dequant).
 //
 // The SEG instance also attends over a bf16 segment after the packed tokens
 // (the frame being generated): its tiles follow the packed ones, and the
@@ -38,7 +47,8 @@
 //
 // Every mbarrier wait is bounded (about 1 s); a timeout sets a device flag
 // that qwm_device_status() reports, every role then leaves its loop, and
-// in-flight copies and MMAs are drained (bounded) before the TMEM is freed.
+// in-flight copies and MMAs are drained (bounded) before both CTAs meet at the
+// final cluster barrier and free the TMEM.
 #include <math.h>
 
 #include "dequant.cuh"
@@ -53,40 +63,49 @@ using namespace tc;
 
 constexpr int DH = 128;        // head_dim handled here
 constexpr int KT = 64;         // keys per tile
+constexpr int KH = KT / 2;     // K' rows (keys) per CTA per tile
+constexpr int VH = DH / 2;     // V' columns (channels) per CTA
 constexpr int QT = 128;        // query rows per Q tile (TMEM lanes)
-constexpr int BQ = 2 * QT;     // query rows per CTA
-constexpr int NKV = 5;         // K' / V' stages (released by the MMA)
-constexpr int NPK = 5;         // packed-field stages (released by the dequant)
+constexpr int ROWS = 2 * QT;   // query rows per CTA at most
+constexpr int NKV = 6;         // K' / V' half-tile stages (released by the MMA)
+constexpr int NPK = 6;         // packed-field stages (released by the dequant)
 constexpr int NTHREADS = 608;  // 8 softmax + 8 dequant + 2 MMA + producer warps
 constexpr int W_MMA = 16;      // warps 16, 17 issue the MMAs of Q tiles 0, 1
 constexpr int W_PROD = 18;
 constexpr int NDQW = 8;        // dequant warps
+constexpr uint16_t BOTH = 3;   // multicast mask: both CTAs of the pair
+constexpr uint16_t LEAD = 1;   // the even CTA only
 
-// ---- shared memory (bytes); K' and V' tiles 1024-aligned for the swizzle
-constexpr uint32_t KV_TILE = KT * DH * 2;  // [2 column halves][64 rows][128 B]
-constexpr uint32_t ST_K = 0, ST_V = KV_TILE;
-constexpr uint32_t KVST = 2 * KV_TILE;     // 32 KB
+// ---- shared memory (bytes); K' and V' halves 1024-aligned for the swizzle
+constexpr uint32_t K_HALF = KH * DH * 2;   // [2 column blocks][32 rows][128 B]
+constexpr uint32_t V_HALF = KT * VH * 2;   // [64 rows][128 B]
+constexpr uint32_t ST_K = 0, ST_V = K_HALF;
+constexpr uint32_t KVST = K_HALF + V_HALF;  // 16 KB
+// Packed-field stage: the tile's fields, then the PSAC bases of the versions of
+// its first and last key, transposed to [r][d] fp32 (one slot when r > 8).
 constexpr uint32_t PK_KCODE = 0, PK_VCODE = 2048, PK_KPAR = 4096, PK_VPAR = 6144,
                    PK_KCOEF = 8192, PK_KCS = 9216, PK_TV = 9344, PK_KIDX = 9472,
-                   PK_VIDX = 9600, PK_CV = 9728, PK_BYTES = 9856;
+                   PK_VIDX = 9600, PK_CV = 9728, PK_U = 9856, PK_U_BYTES = 8192,
+                   PK_BYTES = PK_U + PK_U_BYTES;
 constexpr uint32_t OFF_KV = 0;
 constexpr uint32_t OFF_PK = OFF_KV + NKV * KVST;
 constexpr uint32_t OFF_BAR = (OFF_PK + NPK * PK_BYTES + 127) / 128 * 128;
-constexpr int NBAR = 32;
+constexpr int NBAR = 40;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the attention CTA");
 
 enum {
-  B_LOAD_FULL = 0,   // [NPK] producer bulk copies (tx bytes) -> dequant
-  B_PK_EMPTY = 5,    // [NPK] dequant (one arrival per warp) -> producer
-  B_KV_FULL = 10,    // [NKV] dequant (one arrival per warp) -> MMA
-  B_KV_EMPTY = 15,   // [NKV] MMA commit after each Q tile's P V' -> dequant
-  B_S_FULL = 20,     // [2] MMA commit after Q K'^T
-  B_P_FULL = 22,     // [2] softmax (per warp) -> MMA: P of that Q tile is in TMEM
-  B_Q_READY = 24,    // softmax (per warp) -> MMA: Q in TMEM
-  B_O_LAST = 25,     // [2] MMA commit after the last P V' of that Q tile
-  B_DONE = 27        // [2] MMA commit -> MMA (drain before exit)
+  B_LOAD_FULL = 0,         // [NPK] producer bulk copies (tx bytes) -> dequant (local)
+  B_PK_EMPTY = NPK,        // [NPK] dequant (one arrival per warp) -> producer (local)
+  B_KV_FULL = 2 * NPK,     // [NKV] dequant warps of both CTAs -> MMA (even CTA)
+  B_KV_EMPTY = B_KV_FULL + NKV,  // [NKV] MMA commit after each Q tile's P V' -> dequant (both)
+  B_S_FULL = B_KV_EMPTY + NKV,   // [2] MMA commit after Q K'^T -> softmax (both)
+  B_P_FULL = B_S_FULL + 2,       // [2] softmax warps of both CTAs -> MMA (even CTA)
+  B_Q_READY = B_P_FULL + 2,      // softmax warps of both CTAs -> MMA: Q in TMEM
+  B_O_LAST = B_Q_READY + 1,      // [2] MMA commit after the last P V' -> softmax (both)
+  B_DONE = B_O_LAST + 2          // [2] MMA commit -> MMA (drain before exit)
 };
+static_assert(B_DONE + 2 <= NBAR, "barrier slots");
 
 struct TcArgs {
   Dims Dm;
@@ -101,7 +120,28 @@ struct TcArgs {
   int64_t nseg;
   float* lse;    // [nq][H] natural-log softmax denominators, or null
   int ntp;       // key tiles of the packed part
+  int rc;        // query rows per CTA (<= 256); a pair serves 2 rc rows
+  int nqt;       // Q tiles per CTA with rows (1 or 2), the same in every pair
+  int npairs;    // row blocks (pairs) per key range
+  int nsplit;    // key ranges; > 1: fp32 partials to ws_o / ws_l, merged after
+  float* ws_o;   // [nsplit][nq][H][d] partial outputs (each over its own keys)
+  float* ws_l;   // [nsplit][nq][H] their natural-log softmax denominators
 };
+
+// The key tiles [j0, j0 + n) and the row block of this pair.
+struct Work {
+  int rb, chunk, j0, n;
+};
+
+__device__ __forceinline__ Work work_of(const TcArgs& A, int ntile) {
+  Work w;
+  const int unit = blockIdx.x >> 1;
+  w.rb = unit % A.npairs;
+  w.chunk = unit / A.npairs;
+  w.j0 = (int)((int64_t)w.chunk * ntile / A.nsplit);
+  w.n = (int)((int64_t)(w.chunk + 1) * ntile / A.nsplit) - w.j0;
+  return w;
+}
 
 // Valid keys of tile j: packed tiles first, then (SEG) the segment's tiles.
 template <bool SEG>
@@ -126,18 +166,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 __device__ __forceinline__ void timeout_flag() { atomicExch(&g_tc_timeout, 1); }
 
-// One arrival per warp: every lane has ordered its own writes (proxy fence or
-// tcgen05 fence) before calling; __syncwarp orders the lanes, then lane 0
-// arrives with release semantics.
+// One arrival per warp on this CTA's barrier: every lane has ordered its own
+// writes (proxy fence or tcgen05 fence) before calling; __syncwarp orders the
+// lanes, then lane 0 arrives with release semantics.
 __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// The same on the even CTA's barrier at `bar`'s offset.
+__device__ __forceinline__ void warp_arrive_lead(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cta(bar, 0);
 }
 
 // Bounded wait taken by a whole warp; false (on every lane) if any lane gave up.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   const bool w = mbar_wait(bar, parity);
   return __all_sync(0xffffffffu, w);
+}
+
+// First query row of this CTA.
+__device__ __forceinline__ int64_t cta_row0(const TcArgs& A, const Work& w, uint32_t rank) {
+  return (int64_t)w.rb * 2 * A.rc + (int64_t)rank * A.rc;
 }
 
 // ------------------------------------------------------------------ softmax role
@@ -167,25 +218,28 @@ __device__ __forceinline__ float row_max(const float (&s)[64], int n) {
 
 template <bool SEG>
 __device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, uint32_t tmem,
-                                             int ntile, int nqt) {
+                                             const Work& wk, uint32_t rank) {
   const int warp = threadIdx.x >> 5;
   const int p = warp >> 2;          // Q tile
   const int m = threadIdx.x & 127;  // row in the Q tile = TMEM lane
   const int h = blockIdx.y;
   const int H = A.Dm.H;
-  const int64_t q = (int64_t)blockIdx.x * BQ + p * QT + m;
+  const int64_t r0 = cta_row0(A, wk, rank);
+  const int64_t rend = (r0 + A.rc < A.nq) ? r0 + A.rc : A.nq;
+  const int64_t q = r0 + p * QT + m;
+  const bool valid = (p * QT + m < A.rc) && (q < rend);
   const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   const uint32_t tq = trow + 256 * p, ts = tq + 64, to = tq + 128;
   {
-    // Q row -> TMEM as bf16 pairs (dims 2i, 2i+1 in column i)
-    const uint4* src = reinterpret_cast<const uint4*>(A.Q + ((size_t)q * H + h) * DH);
+    // Q row -> TMEM as bf16 pairs (dims 2i, 2i+1 in column i); zero rows pad
+    const uint4* src = reinterpret_cast<const uint4*>(A.Q + ((size_t)(valid ? q : 0) * H + h) * DH);
 #pragma unroll
     for (int hlf = 0; hlf < 2; ++hlf) {
       uint32_t w[32];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 val = make_uint4(0, 0, 0, 0);
-        if (q < A.nq) val = __ldg(src + hlf * 8 + c);
+        if (valid) val = __ldg(src + hlf * 8 + c);
         w[4 * c] = val.x;
         w[4 * c + 1] = val.y;
         w[4 * c + 2] = val.z;
@@ -195,18 +249,18 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, ui
     }
   }
   tc_fence_before();
-  warp_arrive(&bars[B_Q_READY]);
-  if (p >= nqt) return;
+  warp_arrive_lead(&bars[B_Q_READY]);
+  if (p >= A.nqt) return;
 
   float m_used = -INFINITY;
   uint64_t l2 = 0;  // running row sum, as a pair of partial sums
   const float sl2 = A.scale_log2;
   const uint64_t sc2 = f2pack(sl2, sl2);
   bool ok = true;
-  for (int j = 0; j < ntile; ++j) {
+  for (int j = 0; j < wk.n; ++j) {
     if (!warp_wait(&bars[B_S_FULL + p], j & 1)) { ok = false; break; }
     tc_fence_after();
-    const int nvalid = tile_valid<SEG>(A, j);
+    const int nvalid = tile_valid<SEG>(A, wk.j0 + j);
     float m_row;
     {
       float s[64];
@@ -259,7 +313,7 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, ui
       tmem_st16u(ts + c * 16, pk);
     }
     tc_fence_before();
-    warp_arrive(&bars[B_P_FULL + p]);
+    warp_arrive_lead(&bars[B_P_FULL + p]);
   }
   if (ok) ok = warp_wait(&bars[B_O_LAST + p], 0);
   if (!ok) {
@@ -271,13 +325,32 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, ui
   f2unpack(l2, la, lb);
   const float inv = 1.0f / (la + lb);
   // sum_t 2^(s_t scale log2 e) = l 2^m_used
-  if (A.lse && q < A.nq) A.lse[(size_t)q * H + h] = (m_used + log2f(la + lb)) * 0.6931471805599453f;
-  uint4* dst = reinterpret_cast<uint4*>(A.O + ((size_t)q * H + h) * DH);
+  const float lse = (m_used + log2f(la + lb)) * 0.6931471805599453f;
+  if (A.nsplit > 1) {
+    // partial over this pair's key range: normalized output and its lse
+    const size_t row = ((size_t)wk.chunk * A.nq + (valid ? q : 0)) * H + h;
+    if (valid) A.ws_l[row] = lse;
+    float4* dstp = reinterpret_cast<float4*>(A.ws_o + row * DH);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float o[32];
+      tmem_ld32(to + c * 32, o);
+      if (valid) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dstp[c * 8 + k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
+                                        o[4 * k + 3] * inv);
+      }
+    }
+    return;
+  }
+  if (A.lse && valid) A.lse[(size_t)q * H + h] = lse;
+  uint4* dst = reinterpret_cast<uint4*>(A.O + ((size_t)(valid ? q : 0) * H + h) * DH);
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     float o[32];
     tmem_ld32(to + c * 32, o);
-    if (q < A.nq) {
+    if (valid) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         dst[c * 4 + k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
@@ -299,8 +372,23 @@ struct GroupConst {
   uint64_t s01, s23, m01, m23;  // {S_0, S_1}, {S_2, S_3}, {M_0, M_1}, {M_2, M_3}
 };
 
+// binary16 -> fp32 on the FMA and integer pipes (the conversion unit is left to
+// the softmax's exponentials): the 15 magnitude bits moved to the fp32
+// exponent/mantissa position give 2^-112 times the value, normals and
+// subnormals alike, so one exact multiply by 2^112 restores it.
+__device__ __forceinline__ float half_bits_to_f32(uint32_t h) {
+  const float m = __uint_as_float((h & 0x7fffu) << 13) * 0x1p112f;
+  return __uint_as_float(__float_as_uint(m) | ((h & 0x8000u) << 16));
+}
+
+// int8 -> fp32 without a conversion instruction: adding c to the bit pattern of
+// 1.5 * 2^23 gives 1.5 * 2^23 + c exactly (|c| < 2^22).
+__device__ __forceinline__ float i8_to_f32(int c) {
+  return __uint_as_float(0x4B400000u + (uint32_t)c) - 12582912.0f;
+}
+
 __device__ __forceinline__ GroupConst group_const(uint32_t par) {
-  const float mn = h2f((uint16_t)(par & 0xffff)), sc = h2f((uint16_t)(par >> 16));
+  const float mn = half_bits_to_f32(par & 0xffffu), sc = half_bits_to_f32(par >> 16);
   const float s0 = sc * 256.0f, s1 = sc * 64.0f, s2 = sc * 16.0f, s3 = sc * 4.0f;
   GroupConst g;
   g.s01 = f2pack(s0, s1);
@@ -346,66 +434,100 @@ __device__ __forceinline__ int staged_idx(const uint8_t* pk, uint32_t off, int k
   return ib == 1 ? (int)pk[off + k] : (int)reinterpret_cast<const uint16_t*>(pk + off)[k];
 }
 
-// Rank-8 compensation of one channel for two keys: sum_i U_ji cc_i with the
-// coefficients as pairs {cc_2m, cc_2m+1}; row j of each key's basis holds 8
-// fp32 values (two 16-byte loads; all lanes of the warp read the same row when
-// the keys share a basis version).
-__device__ __forceinline__ void corr8_pair(const float* U0, const float* U1, bool same,
-                                           const uint64_t (&c0)[4], const uint64_t (&c1)[4],
-                                           float& o0, float& o1) {
-  const float4 a0 = __ldg(reinterpret_cast<const float4*>(U0));
-  const float4 b0 = __ldg(reinterpret_cast<const float4*>(U0) + 1);
-  float4 a1 = a0, b1 = b0;
-  if (!same) {
-    a1 = __ldg(reinterpret_cast<const float4*>(U1));
-    b1 = __ldg(reinterpret_cast<const float4*>(U1) + 1);
+// Compensation U (c8 cs) of this thread's 16 channels as 8 channel pairs,
+// from the basis staged transposed ([r][d], row i = column i of U): for each
+// rank i one broadcast of cc_i and four 16-byte loads that every lane of the
+// warp shares when the keys have the same version; 8 independent f32x2 chains.
+__device__ __forceinline__ void corr_staged(const float* Ut, const int8_t* cf, float cs, int r,
+                                            uint64_t (&acc)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0ull;
+#pragma unroll 4
+  for (int i = 0; i < r; ++i) {
+    const float ci = i8_to_f32(cf[i]) * cs;  // exact: 8-bit times 11-bit significands
+    const uint64_t cc = f2pack(ci, ci);
+    const float4* u = reinterpret_cast<const float4*>(Ut + i * DH);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 x = u[q];
+      acc[2 * q] = ffma2(f2pack(x.x, x.y), cc, acc[2 * q]);
+      acc[2 * q + 1] = ffma2(f2pack(x.z, x.w), cc, acc[2 * q + 1]);
+    }
   }
-  uint64_t s0 = ffma2(f2pack(a0.x, a0.y), c0[0], 0ull);
-  uint64_t s1 = ffma2(f2pack(a1.x, a1.y), c1[0], 0ull);
-  s0 = ffma2(f2pack(a0.z, a0.w), c0[1], s0);
-  s1 = ffma2(f2pack(a1.z, a1.w), c1[1], s1);
-  s0 = ffma2(f2pack(b0.x, b0.y), c0[2], s0);
-  s1 = ffma2(f2pack(b1.x, b1.y), c1[2], s1);
-  s0 = ffma2(f2pack(b0.z, b0.w), c0[3], s0);
-  s1 = ffma2(f2pack(b1.z, b1.w), c1[3], s1);
-  float x, y;
-  f2unpack(s0, x, y);
-  o0 = x + y;
-  f2unpack(s1, x, y);
-  o1 = x + y;
 }
 
-// Compensation of one channel for any rank: sequential fold of U_ji c8_i cs
-// (the coefficients read from the staged packed fields).
-__device__ __forceinline__ float corr_any(const float* Uj, const int8_t* cf, float cs, int r) {
-  float acc = 0.0f;
-  for (int i = 0; i < r; ++i) acc = fmaf(__ldg(Uj + i), (float)cf[i] * cs, acc);
-  return acc;
+// The same from the basis in global memory ([d][r], channel j at row j) for a
+// key whose version is not staged with its tile.
+__device__ __forceinline__ void corr_global(const float* Uj0, const int8_t* cf, float cs, int r,
+                                            uint64_t (&acc)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float a = 0.0f, b = 0.0f;
+    for (int i = 0; i < r; ++i) {
+      const float ci = (float)cf[i] * cs;
+      a = fmaf(__ldg(Uj0 + (size_t)(2 * q) * r + i), ci, a);
+      b = fmaf(__ldg(Uj0 + (size_t)(2 * q + 1) * r + i), ci, b);
+    }
+    acc[q] = f2pack(a, b);
+  }
 }
 
-// Issue this thread's 16-byte centroid-chunk copies for tile jj: keys l and
-// l + 32, channel chunks 2s and 2s + 1 of K and V (s = dequant warp), each from
-// the table version the key was encoded with; one commit group per tile.
+// Rewrite chunk c (8 channels) of row `row` of an R-row swizzled tile in place:
+// centroid chunk from the stage, residual (and compensation) added in fp32, one
+// bf16 rounding.
+template <int R>
+__device__ __forceinline__ void deq_chunk(uint8_t* base, int row, int c, uint32_t bits16,
+                                          uint32_t par, const uint64_t* corr) {
+  const GroupConst g = group_const(par);
+  const uint32_t off = sw128_off(row, c, R);
+  const uint4 cw = *reinterpret_cast<const uint4*>(base + off);
+  uint64_t v2[4];
+  deq_chunk_f32(cw, bits16, g, v2);
+  if (corr) {
+#pragma unroll
+    for (int pi = 0; pi < 4; ++pi) v2[pi] = fadd2(v2[pi], corr[pi]);
+  }
+  *reinterpret_cast<uint4*>(base + off) = pack_chunk(v2);
+}
+
+template <int R>
+__device__ __forceinline__ void zero_chunk(uint8_t* base, int row, int c) {
+  *reinterpret_cast<uint4*>(base + sw128_off(row, c, R)) = make_uint4(0, 0, 0, 0);
+}
+
+// This thread's share of a tile (rank = CTA in the pair, sw = dequant warp):
+//   K': key kk = 32 rank + lane of the tile, channel chunks 2sw, 2sw+1;
+//   V': keys lane and lane + 32, channel chunk cvc = 8 rank + sw (chunk sw of
+//       this CTA's 64-channel half).
+struct DqShare {
+  int kk, sw, lane, cvc;
+};
+
+// Issue the 16-byte centroid-chunk copies of tile jj, each from the table
+// version its key was encoded with; one commit group per tile.
 __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, const PackedHead& ph,
-                                             int jj, int lane, int sw) {
-  const uint8_t* pk = smem + OFF_PK + (jj % NPK) * PK_BYTES;
-  const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
+                                             int jj, int jl, const DqShare& d) {
+  const uint8_t* pk = smem + OFF_PK + (jl % NPK) * PK_BYTES;
+  const uint32_t st = smem_u32(smem + OFF_KV + (jl % NKV) * KVST);
   const int ib = A.Dm.idx_bytes;
   const uint16_t* cvs = reinterpret_cast<const uint16_t*>(pk + PK_CV);
+  const int64_t t0 = (int64_t)jj * KT;
+  if (t0 + d.kk < A.T) {
+    const uint16_t* ck = ph.cent_k + (size_t)cvs[d.kk] * ph.cstride +
+                         (size_t)staged_idx(pk, PK_KIDX, d.kk, ib) * DH;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * d.sw + cc;
+      cp_async16_cg(st + ST_K + sw128_off(d.lane, c, KH), ck + c * 8);
+    }
+  }
 #pragma unroll
   for (int kk = 0; kk < 2; ++kk) {
-    const int k = lane + 32 * kk;
-    const int64_t t = (int64_t)jj * KT + k;
-    if (t < A.T) {
-      const size_t vo = (size_t)cvs[k] * ph.cstride;
-      const uint16_t* ck = ph.cent_k + vo + (size_t)staged_idx(pk, PK_KIDX, k, ib) * DH;
-      const uint16_t* cv = ph.cent_v + vo + (size_t)staged_idx(pk, PK_VIDX, k, ib) * DH;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * sw + cc;
-        cp_async16(st + ST_K + sw128_off(k, c, KT), ck + c * 8);
-        cp_async16(st + ST_V + sw128_off(k, c, KT), cv + c * 8);
-      }
+    const int k = d.lane + 32 * kk;
+    if (t0 + k < A.T) {
+      const uint16_t* cv = ph.cent_v + (size_t)cvs[k] * ph.cstride +
+                           (size_t)staged_idx(pk, PK_VIDX, k, ib) * DH;
+      cp_async16_cg(st + ST_V + sw128_off(k, d.sw, KT), cv + d.cvc * 8);
     }
   }
   cp_async_commit();
@@ -413,178 +535,134 @@ __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, con
 
 // Segment tile jj (jj >= ntp): this thread's 16-byte chunks of the bf16 K and V
 // rows copied as they are into the same swizzled stage positions.
-__device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem, int jj, int lane,
-                                                 int sw) {
-  const uint32_t st = smem_u32(smem + OFF_KV + (jj % NKV) * KVST);
+__device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem, int jj, int jl,
+                                                 const DqShare& d) {
+  const uint32_t st = smem_u32(smem + OFF_KV + (jl % NKV) * KVST);
+  const int64_t t0 = (int64_t)(jj - A.ntp) * KT;
+  if (t0 + d.kk < A.nseg) {
+    const uint16_t* kr = A.Ks + ((size_t)(t0 + d.kk) * A.Dm.H + blockIdx.y) * DH;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * d.sw + cc;
+      cp_async16_cg(st + ST_K + sw128_off(d.lane, c, KH), kr + c * 8);
+    }
+  }
 #pragma unroll
   for (int kk = 0; kk < 2; ++kk) {
-    const int k = lane + 32 * kk;
-    const int64_t t = (int64_t)(jj - A.ntp) * KT + k;
-    if (t < A.nseg) {
-      const size_t row = ((size_t)t * A.Dm.H + blockIdx.y) * DH;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * sw + cc;
-        cp_async16(st + ST_K + sw128_off(k, c, KT), A.Ks + row + c * 8);
-        cp_async16(st + ST_V + sw128_off(k, c, KT), A.Vs + row + c * 8);
-      }
+    const int k = d.lane + 32 * kk;
+    if (t0 + k < A.nseg) {
+      const uint16_t* vr = A.Vs + ((size_t)(t0 + k) * A.Dm.H + blockIdx.y) * DH;
+      cp_async16_cg(st + ST_V + sw128_off(k, d.sw, KT), vr + d.cvc * 8);
     }
   }
   cp_async_commit();
 }
 
-// Rewrite chunk c (8 channels) of key row k in place: centroid chunk from the
-// stage, residual (and compensation) added in fp32, one bf16 rounding.
-__device__ __forceinline__ void deq_chunk(uint8_t* base, int k, int c, uint32_t bits16,
-                                          uint32_t par, const float* corr) {
-  const GroupConst g = group_const(par);
-  const uint32_t off = sw128_off(k, c, KT);
-  const uint4 cw = *reinterpret_cast<const uint4*>(base + off);
-  uint64_t v2[4];
-  deq_chunk_f32(cw, bits16, g, v2);
-  if (corr) {
-#pragma unroll
-    for (int pi = 0; pi < 4; ++pi) v2[pi] = fadd2(v2[pi], f2pack(corr[2 * pi], corr[2 * pi + 1]));
-  }
-  *reinterpret_cast<uint4*>(base + off) = pack_chunk(v2);
-}
-
-__device__ __forceinline__ void zero_chunks(uint8_t* kb, uint8_t* vb, int k, int sw) {
-#pragma unroll
-  for (int cc = 0; cc < 2; ++cc) {
-    const uint32_t off = sw128_off(k, 2 * sw + cc, KT);
-    *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
-  }
-}
-
 template <bool SEG>
 __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
-                                             int ntile) {
+                                             const Work& wk, uint32_t rank) {
   const int dq = threadIdx.x - 256;  // 0..255
-  const int sw = dq >> 5;            // channel slice [16 sw, 16 sw + 16)
-  const int lane = dq & 31;          // keys lane, lane + 32
+  DqShare d;
+  d.sw = dq >> 5;
+  d.lane = dq & 31;
+  d.kk = KH * (int)rank + d.lane;
+  d.cvc = 8 * (int)rank + d.sw;
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
   const int G = Dm.G, ng = Dm.ng, r = Dm.r;
-  const int gi = (16 * sw) / G;      // the slice's INT2 group (one group: G = 16 or 32)
+  const int gik = (16 * d.sw) / G;   // INT2 group of the K' channels (one group)
+  const int giv = (8 * d.cvc) / G;   // INT2 group of the V' chunk
   const size_t ustride = (size_t)Dm.H * DH * (r > 0 ? r : 1);  // floats per basis version
-  const float* ubase = A.v.basis + (size_t)h * DH * (r > 0 ? r : 1) + (size_t)16 * sw * r;
+  const float* ubase = A.v.basis + (size_t)h * DH * (r > 0 ? r : 1) + (size_t)16 * d.sw * r;
   bool ok = true;
-  const int ntp = SEG ? A.ntp : ntile;
-  // prologue: gathers of tiles 0 and 1 (their K' / V' stages start free)
-  for (int jj = 0; jj < 2 && jj < ntile; ++jj) {
-    if (!SEG || jj < ntp) {
-      if (!warp_wait(&bars[B_LOAD_FULL + jj], 0)) { ok = false; break; }
-      issue_gather(A, smem, ph, jj, lane, sw);
+  const int ntp = A.ntp;  // tiles below ntp are packed, the rest (SEG) the segment's
+  const int n = wk.n, j0 = wk.j0;
+  // prologue: gathers of the range's first two tiles (their stages start free);
+  // ring slots and barrier phases count tiles from the start of the range
+  for (int jl = 0; jl < 2 && jl < n; ++jl) {
+    if (!SEG || j0 + jl < ntp) {
+      if (!warp_wait(&bars[B_LOAD_FULL + jl], 0)) { ok = false; break; }
+      issue_gather(A, smem, ph, j0 + jl, jl, d);
     } else {
-      issue_seg_gather(A, smem, jj, lane, sw);
+      issue_seg_gather(A, smem, j0 + jl, jl, d);
     }
   }
-  for (int j = 0; ok && j < ntile; ++j) {
-    if (j + 2 < ntile) {
-      const int j2 = j + 2;
-      if ((!SEG || j2 < ntp) &&
-          !warp_wait(&bars[B_LOAD_FULL + j2 % NPK], (j2 / NPK) & 1)) { ok = false; break; }
-      if (j2 >= NKV &&
-          !warp_wait(&bars[B_KV_EMPTY + j2 % NKV], ((j2 / NKV) - 1) & 1)) { ok = false; break; }
-      if (!SEG || j2 < ntp) issue_gather(A, smem, ph, j2, lane, sw);
-      else issue_seg_gather(A, smem, j2, lane, sw);
+  for (int jl = 0; ok && jl < n; ++jl) {
+    const int j = j0 + jl;
+    if (jl + 2 < n) {
+      const int l2 = jl + 2;
+      if ((!SEG || j0 + l2 < ntp) &&
+          !warp_wait(&bars[B_LOAD_FULL + l2 % NPK], (l2 / NPK) & 1)) { ok = false; break; }
+      if (l2 >= NKV &&
+          !warp_wait(&bars[B_KV_EMPTY + l2 % NKV], ((l2 / NKV) - 1) & 1)) { ok = false; break; }
+      if (!SEG || j0 + l2 < ntp) issue_gather(A, smem, ph, j0 + l2, l2, d);
+      else issue_seg_gather(A, smem, j0 + l2, l2, d);
       cp_async_wait<2>();
-    } else if (j + 1 < ntile) {
+    } else if (jl + 1 < n) {
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
-    const int s = j % NKV, sp = j % NPK;
+    const int s = jl % NKV, sp = jl % NPK;
     uint8_t* st = smem + OFF_KV + s * KVST;
     uint8_t* kb = st + ST_K;
     uint8_t* vb = st + ST_V;
     if (SEG && j >= ntp) {
       // segment tile: rows already in place; zero rows past the segment's end
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const int k = lane + 32 * kk;
-        if ((int64_t)(j - ntp) * KT + k >= A.nseg) {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t off = sw128_off(k, 2 * sw + cc, KT);
-            *reinterpret_cast<uint4*>(kb + off) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(vb + off) = make_uint4(0, 0, 0, 0);
-          }
-        }
+      const int64_t t0 = (int64_t)(j - ntp) * KT;
+      if (t0 + d.kk >= A.nseg) {
+        zero_chunk<KH>(kb, d.lane, 2 * d.sw);
+        zero_chunk<KH>(kb, d.lane, 2 * d.sw + 1);
       }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+        if (t0 + d.lane + 32 * kk >= A.nseg) zero_chunk<KT>(vb, d.lane + 32 * kk, d.sw);
       fence_proxy_async_smem();
-      warp_arrive(&bars[B_KV_FULL + s]);
+      warp_arrive_lead(&bars[B_KV_FULL + s]);
       continue;
     }
     const uint8_t* pk = smem + OFF_PK + sp * PK_BYTES;
     const int64_t t0 = (int64_t)j * KT;
-    const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
-    const uint16_t* kcs = reinterpret_cast<const uint16_t*>(pk + PK_KCS);
-    const int8_t* kcf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF);
-    const int k0 = lane, k1 = lane + 32;
-    const bool in0 = t0 + k0 < A.T, in1 = t0 + k1 < A.T;
-    const uint32_t* kpar = reinterpret_cast<const uint32_t*>(pk + PK_KPAR);
-    const uint32_t* vpar = reinterpret_cast<const uint32_t*>(pk + PK_VPAR);
-    // ---- K' rows: residual plus the compensation of this slice's channels
-    {
-      const uint32_t kw0 = *reinterpret_cast<const uint32_t*>(pk + PK_KCODE + k0 * 32 + 4 * sw);
-      const uint32_t kw1 = *reinterpret_cast<const uint32_t*>(pk + PK_KCODE + k1 * 32 + 4 * sw);
-      const uint32_t p0 = kpar[k0 * ng + gi], p1 = kpar[k1 * ng + gi];
-      const int v0 = in0 ? tv[k0] : 0, v1 = in1 ? tv[k1] : v0;
-      const float* U0 = ubase + (size_t)v0 * ustride;
-      const float* U1 = ubase + (size_t)v1 * ustride;
-      const float cs0 = in0 ? h2f(kcs[k0]) : 0.0f, cs1 = in1 ? h2f(kcs[k1]) : 0.0f;
-      uint64_t c0[4], c1[4];
-      if (r == 8) {
-        const int2 w0 = *reinterpret_cast<const int2*>(kcf + 8 * k0);
-        const int2 w1 = *reinterpret_cast<const int2*>(kcf + 8 * k1);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t x0 = m < 2 ? (uint32_t)w0.x : (uint32_t)w0.y;
-          const uint32_t x1 = m < 2 ? (uint32_t)w1.x : (uint32_t)w1.y;
-          const int sh = 16 * (m & 1);
-          // c8 * cs is exact in fp32 (8-bit times 11-bit significands)
-          c0[m] = f2pack((float)(int8_t)(x0 >> sh) * cs0, (float)(int8_t)(x0 >> (sh + 8)) * cs0);
-          c1[m] = f2pack((float)(int8_t)(x1 >> sh) * cs1, (float)(int8_t)(x1 >> (sh + 8)) * cs1);
-        }
+    // ---- K': residual plus the compensation of this slice's 16 channels
+    if (t0 + d.kk < A.T) {
+      const int kk = d.kk;
+      const uint32_t kw = *reinterpret_cast<const uint32_t*>(pk + PK_KCODE + kk * 32 + 4 * d.sw);
+      const uint32_t kp = reinterpret_cast<const uint32_t*>(pk + PK_KPAR)[kk * ng + gik];
+      uint64_t corr[8];
+      if (r > 0) {
+        // the basis of the key's version: a staged slot (the versions of the
+        // tile's first and last key), else global memory
+        const uint16_t* tv = reinterpret_cast<const uint16_t*>(pk + PK_TV);
+        const int ver = tv[kk];
+        const int nval = (int)((A.T - t0) < KT ? (A.T - t0) : KT);
+        const float cs = half_bits_to_f32(reinterpret_cast<const uint16_t*>(pk + PK_KCS)[kk]);
+        const int8_t* kcf = reinterpret_cast<const int8_t*>(pk + PK_KCOEF) + kk * r;
+        const float* us = reinterpret_cast<const float*>(pk + PK_U) + 16 * d.sw;
+        if (ver == tv[0]) corr_staged(us, kcf, cs, r, corr);
+        else if (r <= 8 && ver == tv[nval - 1]) corr_staged(us + r * DH, kcf, cs, r, corr);
+        else corr_global(ubase + (size_t)ver * ustride, kcf, cs, r, corr);
       }
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        float q0[8], q1[8];
-        if (r == 8) {
-          const bool same = (v0 == v1);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            corr8_pair(U0 + 8 * (8 * cc + e), U1 + 8 * (8 * cc + e), same, c0, c1, q0[e], q1[e]);
-        } else if (r > 0) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            q0[e] = corr_any(U0 + (size_t)(8 * cc + e) * r, kcf + k0 * r, cs0, r);
-            q1[e] = corr_any(U1 + (size_t)(8 * cc + e) * r, kcf + k1 * r, cs1, r);
-          }
-        }
-        if (in0) deq_chunk(kb, k0, 2 * sw + cc, (kw0 >> (16 * cc)) & 0xffffu, p0, r > 0 ? q0 : nullptr);
-        if (in1) deq_chunk(kb, k1, 2 * sw + cc, (kw1 >> (16 * cc)) & 0xffffu, p1, r > 0 ? q1 : nullptr);
-      }
+      deq_chunk<KH>(kb, d.lane, 2 * d.sw, kw & 0xffffu, kp, r > 0 ? corr : nullptr);
+      deq_chunk<KH>(kb, d.lane, 2 * d.sw + 1, kw >> 16, kp, r > 0 ? corr + 4 : nullptr);
+    } else {
+      zero_chunk<KH>(kb, d.lane, 2 * d.sw);
+      zero_chunk<KH>(kb, d.lane, 2 * d.sw + 1);
     }
-    // ---- V' rows
+    // ---- V': this CTA's channel chunk of keys lane and lane + 32
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk) {
-      const int k = lane + 32 * kk;
-      if (kk == 0 ? in0 : in1) {
-        const uint32_t vw = *reinterpret_cast<const uint32_t*>(pk + PK_VCODE + k * 32 + 4 * sw);
-        const uint32_t vp = vpar[k * ng + gi];
-        deq_chunk(vb, k, 2 * sw, vw & 0xffffu, vp, nullptr);
-        deq_chunk(vb, k, 2 * sw + 1, vw >> 16, vp, nullptr);
+      const int k = d.lane + 32 * kk;
+      if (t0 + k < A.T) {
+        const uint32_t vw = *reinterpret_cast<const uint16_t*>(pk + PK_VCODE + k * 32 + 2 * d.cvc);
+        const uint32_t vp = reinterpret_cast<const uint32_t*>(pk + PK_VPAR)[k * ng + giv];
+        deq_chunk<KT>(vb, k, d.sw, vw, vp, nullptr);
       } else {
-        zero_chunks(kb, vb, k, sw);
+        zero_chunk<KT>(vb, k, d.sw);
       }
     }
     fence_proxy_async_smem();
-    warp_arrive(&bars[B_KV_FULL + s]);
+    warp_arrive_lead(&bars[B_KV_FULL + s]);
     warp_arrive(&bars[B_PK_EMPTY + sp]);
   }
   cp_async_wait<0>();
@@ -593,27 +671,60 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
 
 // ------------------------------------------------------------------ producer role
 __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
-                                              int ntile) {
+                                              const Work& wk) {
   const int lane = threadIdx.x & 31;
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
   const int ng = Dm.ng, r = Dm.r, ib = Dm.idx_bytes;
   const uint32_t par_bytes = KT * ng * 4, coef_bytes = KT * r, idx_bytes = KT * ib;
-  const uint32_t tx = 2 * (KT * DH / 4) + 2 * par_bytes + (r > 0 ? coef_bytes + KT * 2 : 0) +
-                      2 * KT * 2 + 2 * idx_bytes;
+  const uint32_t tx0 = 2 * (KT * DH / 4) + 2 * par_bytes + (r > 0 ? coef_bytes + KT * 2 : 0) +
+                       2 * KT * 2 + 2 * idx_bytes;
+  const int un = r * DH;  // floats of one basis version of this head
+  const float* ub = A.v.basis + (size_t)h * DH * r;
+  const size_t vs = (size_t)Dm.H * DH * r;
+  int pva = -1, pvb = -1;            // versions staged with the previous tile
+  const float* prevU = nullptr;
   bool ok = true;
   int issued = 0;
-  for (int j = 0; j < ntile; ++j) {
-    const int s = j % NPK;
-    if (j >= NPK) {
-      if (!warp_wait(&bars[B_PK_EMPTY + s], ((j / NPK) - 1) & 1)) { ok = false; break; }
+  // the packed tiles of the range (segment tiles need no fields)
+  const int npk = (wk.j0 + wk.n < A.ntp ? wk.j0 + wk.n : A.ntp) - wk.j0;
+  for (int jl = 0; jl < npk; ++jl) {
+    const int s = jl % NPK;
+    if (jl >= NPK) {
+      if (!warp_wait(&bars[B_PK_EMPTY + s], ((jl / NPK) - 1) & 1)) { ok = false; break; }
     }
     uint8_t* pk = smem + OFF_PK + s * PK_BYTES;
-    const int64_t t0 = (int64_t)j * KT;
+    const int64_t t0 = (int64_t)(wk.j0 + jl) * KT;
+    if (r > 0) {
+      // the bases of the versions of the tile's first and last key, transposed
+      // to [r][d]: copied from the previous tile's stage when the version was
+      // staged there, else gathered from global memory (once per version)
+      const int64_t t1 = (t0 + KT < A.T ? t0 + KT : A.T) - 1;
+      const int va = A.v.tokver[t0], vb = A.v.tokver[t1];
+      const int nsl = (r <= 8 && vb != va) ? 2 : 1;
+      float* Ut = reinterpret_cast<float*>(pk + PK_U);
+      for (int sl = 0; sl < nsl; ++sl) {
+        const int v = sl ? vb : va;
+        float* dst = Ut + sl * un;
+        const float* src = (v == pva) ? prevU : (v == pvb ? prevU + un : nullptr);
+        if (src) {
+          for (int e = 4 * lane; e < un; e += 128)
+            *reinterpret_cast<float4*>(dst + e) = *reinterpret_cast<const float4*>(src + e);
+        } else {
+          const float* Ug = ub + (size_t)v * vs;
+#pragma unroll 8
+          for (int e = lane; e < un; e += 32) dst[e] = __ldg(Ug + (size_t)(e & (DH - 1)) * r + (e >> 7));
+        }
+      }
+      pva = va;
+      pvb = nsl == 2 ? vb : -1;
+      prevU = Ut;
+    }
+    __syncwarp();  // the lanes' staged basis is written before lane 0 arrives
     if (lane == 0) {
       uint64_t* bar = &bars[B_LOAD_FULL + s];
-      mbar_arrive_expect_tx(bar, tx);
+      mbar_arrive_expect_tx(bar, tx0);
       bulk_g2s(smem_u32(pk + PK_KCODE), ph.k_codes + t0 * (DH / 4), KT * DH / 4, bar);
       bulk_g2s(smem_u32(pk + PK_VCODE), ph.v_codes + t0 * (DH / 4), KT * DH / 4, bar);
       bulk_g2s(smem_u32(pk + PK_KPAR), ph.k_params + t0 * ng * 2, par_bytes, bar);
@@ -638,48 +749,53 @@ __device__ __forceinline__ void producer_role(const TcArgs& A, uint8_t* smem, ui
 
 // ------------------------------------------------------------------ MMA role
 // Descriptors are built once; a stage or K-step offset is added to the start
-// address field (bytes / 16; no carry out of the 14-bit field in 227 KB).
+// address field (bytes / 16; no carry out of the 14-bit field in 227 KB).  Both
+// CTAs lay out their halves at the same offsets, so one descriptor addresses
+// both.
 struct MmaDesc {
   uint64_t k, v;
 };
 
-// S_p = Q_p K'^T (8 K16 steps, A from TMEM) for the tile in stage s.
+// S_p = Q_p K'^T for the tile in stage s: M = 256 rows of the pair, N = 64 keys
+// (32 in each CTA's K' half), 8 K16 steps with A = Q from TMEM.
 __device__ __forceinline__ void issue_qk(const MmaDesc& D, uint32_t tmem, int p, int s) {
-  constexpr uint32_t IDQ = idesc_bf16(128, KT, false, false);
+  constexpr uint32_t IDQ = idesc_bf16(256, KT, false, false);
   const uint32_t tq = tmem + 256 * p, ts = tq + 64;
   const uint64_t kd = D.k + (uint64_t)((s * KVST) >> 4);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint32_t koff = ((k >> 2) * (KT * 128) + (k & 3) * 32) >> 4;
-    mma_bf16_ts(ts, tq + 8 * k, kd + koff, IDQ, k > 0);
+    const uint32_t koff = ((k >> 2) * (KH * 128) + (k & 3) * 32) >> 4;
+    mma2_bf16_ts(ts, tq + 8 * k, kd + koff, IDQ, k > 0);
   }
 }
 
-// O_p += P_p V' (stage s) with P read from TMEM (the S columns of Q tile p).
+// O_p += P_p V' (stage s): M = 256, N = 128 channels (64 in each CTA's V' half),
+// 4 K16 steps over the tile's keys with A = P from TMEM.
 __device__ __forceinline__ void issue_pv(const MmaDesc& D, uint32_t tmem, int p, int s,
                                          bool first) {
-  constexpr uint32_t IDP = idesc_bf16(128, DH, false, true);
+  constexpr uint32_t IDP = idesc_bf16(256, DH, false, true);
   const uint32_t ts = tmem + 256 * p + 64, to = tmem + 256 * p + 128;
   const uint64_t vd = D.v + (uint64_t)((s * KVST) >> 4);
 #pragma unroll
   for (int k = 0; k < KT / 16; ++k)
-    mma_bf16_ts(to, ts + 8 * k, vd + (uint64_t)((k * 2048) >> 4), IDP,
-                (!first || k > 0) ? 1u : 0u);
+    mma2_bf16_ts(to, ts + 8 * k, vd + (uint64_t)((k * 16 * 128) >> 4), IDP,
+                 (!first || k > 0) ? 1u : 0u);
 }
 
-// One issuing thread per Q tile p (warps 16 and 17), each running
-//   Q K'^T(p, t) -> wait for the softmax -> P V'(p, t) -> Q K'^T(p, t + 1) -> ...
-// with blocking waits; the two threads interleave on the tensor pipe, which
-// works on one Q tile while the softmax works on the other.  Q K'^T(p, t + 1)
+// One issuing thread per Q tile p in the even CTA (warps 16 and 17), each
+// running  Q K'^T(p, t) -> wait for P -> P V'(p, t) -> Q K'^T(p, t + 1) -> ...
+// with blocking waits; the two threads interleave on the tensor pipes, which
+// work on one Q tile while the softmax works on the other.  Q K'^T(p, t + 1)
 // comes after P V'(p, t) in the thread's issue order, so an MMA that
 // overwrites the S/P columns never overtakes the P V' that reads them.  A stage
-// is released after both threads' P V' (one commit each).
+// is released in both CTAs after both threads' P V' (one commit each).
 __device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_t* bars,
                                          uint32_t tmem, int ntile, int p) {
+  // ntile: tiles of this pair's key range
   const uint32_t sbase = smem_u32(smem);
   MmaDesc D;
   D.k = desc_sw128(sbase + OFF_KV + ST_K, 16, 1024);
-  D.v = desc_sw128(sbase + OFF_KV + ST_V, KT * 128, 1024);
+  D.v = desc_sw128(sbase + OFF_KV + ST_V, 16, 1024);
   bool ok = mbar_wait(&bars[B_Q_READY], 0);
   tc_fence_after();
   for (int t = 0; ok && t < ntile; ++t) {
@@ -687,71 +803,139 @@ __device__ __forceinline__ void mma_role(const TcArgs& A, uint8_t* smem, uint64_
     if (!mbar_wait(&bars[B_KV_FULL + s], (t / NKV) & 1)) { ok = false; break; }
     tc_fence_after();
     issue_qk(D, tmem, p, s);
-    mma_commit(&bars[B_S_FULL + p]);
+    mma2_commit_mc(&bars[B_S_FULL + p], BOTH);
     if (!mbar_wait(&bars[B_P_FULL + p], t & 1)) { ok = false; break; }
     tc_fence_after();
     issue_pv(D, tmem, p, s, t == 0);
-    mma_commit(&bars[B_KV_EMPTY + s]);
-    if (t == ntile - 1) mma_commit(&bars[B_O_LAST + p]);
+    mma2_commit_mc(&bars[B_KV_EMPTY + s], BOTH);
+    if (t == ntile - 1) mma2_commit_mc(&bars[B_O_LAST + p], BOTH);
   }
-  mma_commit(&bars[B_DONE + p]);
+  mma2_commit_mc(&bars[B_DONE + p], LEAD);
   if (!mbar_wait(&bars[B_DONE + p], 0)) ok = false;
   if (!ok) timeout_flag();
 }
 
 template <bool SEG>
-__global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const TcArgs A) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    attn_tc_kernel(const TcArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_BAR + NBAR * 8);
   const int warp = threadIdx.x / 32;
+  const uint32_t rank = cluster_rank();
   const int ntile = SEG ? A.ntp + (int)((A.nseg + KT - 1) / KT) : A.ntp;
-  const int nqt = ((int64_t)blockIdx.x * BQ + QT < A.nq) ? 2 : 1;
+  const Work wk = work_of(A, ntile);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NPK; ++i) {
       mbar_init(&bars[B_LOAD_FULL + i], 1);
       mbar_init(&bars[B_PK_EMPTY + i], NDQW);
     }
     for (int i = 0; i < NKV; ++i) {
-      mbar_init(&bars[B_KV_FULL + i], NDQW);
-      mbar_init(&bars[B_KV_EMPTY + i], nqt);  // one commit per Q tile
+      mbar_init(&bars[B_KV_FULL + i], 2 * NDQW);  // dequant warps of both CTAs
+      mbar_init(&bars[B_KV_EMPTY + i], A.nqt);    // one commit per Q tile
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[B_S_FULL + i], 1);
-      mbar_init(&bars[B_P_FULL + i], 4);
+      mbar_init(&bars[B_P_FULL + i], 8);           // 4 softmax warps in each CTA
       mbar_init(&bars[B_O_LAST + i], 1);
       mbar_init(&bars[B_DONE + i], 1);
     }
-    mbar_init(&bars[B_Q_READY], 8);
+    mbar_init(&bars[B_Q_READY], 16);
     fence_mbar_init();
   }
   if (warp == W_MMA) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
+    tmem_alloc2(tmem_holder, 512);
+    tmem_relinquish2();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any arrival crosses the pair
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   if (warp < 8) {
-    softmax_role<SEG>(A, bars, tmem, ntile, nqt);
+    softmax_role<SEG>(A, bars, tmem, wk, rank);
   } else if (warp < 8 + NDQW) {
-    dequant_role<SEG>(A, smem, bars, ntile);
+    dequant_role<SEG>(A, smem, bars, wk, rank);
   } else if (warp < W_PROD) {
     const int p = warp - W_MMA;
-    if ((threadIdx.x & 31) == 0 && p < nqt) mma_role(A, smem, bars, tmem, ntile, p);
+    if (rank == 0 && (threadIdx.x & 31) == 0 && p < A.nqt) mma_role(A, smem, bars, tmem, wk.n, p);
     __syncwarp();
   } else {
-    producer_role(A, smem, bars, A.ntp);  // packed tiles only
+    producer_role(A, smem, bars, wk);
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // no MMA of the pair reads this CTA's memory any more
   if (warp == W_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc2(tmem, 512);
   }
+}
+
+// Merge of the key ranges' partials: for each (query row, head) one warp, lane
+// l holding channels 4l .. 4l+3.  With L_c the ranges' log-sum-exps and O_c
+// their normalized outputs, O = sum_c e^(L_c - L) O_c / sum_c e^(L_c - L) and
+// the row's log-sum-exp is L + ln sum_c e^(L_c - L), L = max_c L_c.
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ ws_o,
+                                                         const float* __restrict__ ws_l,
+                                                         int nsplit, int64_t rows,
+                                                         uint16_t* __restrict__ O,
+                                                         float* __restrict__ lse) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // q * H + h
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float L = -INFINITY;
+  for (int c = 0; c < nsplit; ++c) L = fmaxf(L, __ldg(ws_l + (size_t)c * rows + row));
+  float den = 0.0f;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int c = 0; c < nsplit; ++c) {
+    const float w = expf(__ldg(ws_l + (size_t)c * rows + row) - L);
+    const float4 o = __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)c * rows + row) * DH) + lane);
+    den += w;
+    acc.x = fmaf(w, o.x, acc.x);
+    acc.y = fmaf(w, o.y, acc.y);
+    acc.z = fmaf(w, o.z, acc.z);
+    acc.w = fmaf(w, o.w, acc.w);
+  }
+  const float inv = 1.0f / den;
+  uint2 out = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+  *reinterpret_cast<uint2*>(O + row * DH + 4 * lane) = out;
+  if (lse && lane == 0) lse[row] = L + logf(den);
+}
+
+// Number of SMs of the current device (cached per device).
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Key ranges for `units` (row block, head) pairs of CTAs over `ntile` tiles:
+// the count that minimizes (rounds of pairs on the GPU) x (tiles per range
+// plus a fixed per-range cost of about 4 tiles), within the workspace.
+int choose_split(int64_t units, int ntile, int64_t nq, const Dims& D) {
+  if (nq > D.max_queries || ntile < 16) return 1;
+  const int64_t slots = device_sms() / 2;
+  int best = 1;
+  double bestc = 1e300;
+  for (int s = 1; s <= QWM_ATTN_MAX_SPLIT && s <= ntile / 8; ++s) {
+    const double rounds = (double)((units * s + slots - 1) / slots);
+    const double c = rounds * ((double)ntile / s + 4.0);
+    if (c < bestc * 0.98) {
+      bestc = c;
+      best = s;
+    }
+  }
+  return best;
 }
 
 }  // namespace
@@ -774,13 +958,32 @@ cudaError_t launch_attention_tc(const Dims& D, const CacheView& v, int64_t T, co
   a.nseg = sg.n;
   a.lse = sg.lse;
   a.ntp = (int)((T + KT - 1) / KT);
+  // row blocks of at most 2 x 256 rows per pair, spread evenly over the pairs
+  const int64_t npairs = (nq + 2 * ROWS - 1) / (2 * ROWS);
+  a.rc = (int)((nq + 2 * npairs - 1) / (2 * npairs));
+  a.nqt = a.rc > QT ? 2 : 1;
+  a.npairs = (int)npairs;
+  const int ntile = a.ntp + (int)((sg.n + KT - 1) / KT);
+  // key ranges across pairs, so that the last round of pairs on the GPU fills
+  a.nsplit = choose_split(npairs * D.H, ntile, nq, D);
+  a.ws_o = nullptr;
+  a.ws_l = nullptr;
+  if (a.nsplit > 1) {
+    a.ws_o = reinterpret_cast<float*>(v.workspace);
+    a.ws_l = a.ws_o + (size_t)a.nsplit * nq * D.H * DH;
+  }
   // the segment variant only when there is one (no extra branches otherwise)
   auto kern = sg.n > 0 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((nq + BQ - 1) / BQ), D.H);
+  dim3 grid((unsigned)(2 * npairs * a.nsplit), D.H);
   kern<<<grid, NTHREADS, SMEM_BYTES, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.nsplit == 1) return e;
+  const int64_t rows = nq * D.H;
+  attn_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.ws_o, a.ws_l, a.nsplit, rows, O,
+                                                               sg.lse);
   return cudaGetLastError();
 }
 

@@ -17,6 +17,7 @@ struct Dims {
   int64_t tcap;
   int idx_bytes;  // 1 if C <= 256 else 2
   int qsac_full;  // QSAC stage 2 by the full quadratic form e^T A e
+  int max_queries;  // query rows the WORKSPACE holds attention partials for
 };
 
 // ---------------------------------------------------------------- host-side validation
@@ -33,6 +34,7 @@ inline bool config_ok(const qwm_config* c) {
   if (c->rank < 0 || c->rank > 16) return false;
   if (c->max_versions < 1 || c->max_versions > 65535) return false;
   if (c->max_cent_versions < 1 || c->max_cent_versions > 65535) return false;
+  if (c->max_queries < 0 || c->max_queries > (1 << 24)) return false;
   if ((c->flags & ~QWM_FLAG_QSAC_FULL) != 0) return false;
   if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 40)) return false;
   return true;
@@ -54,6 +56,7 @@ inline Dims dims_of(const qwm_config* c) {
   D.tcap = (c->max_tokens + 127) / 128 * 128;
   D.idx_bytes = c->n_centroids <= 256 ? 1 : 2;
   D.qsac_full = (c->flags & QWM_FLAG_QSAC_FULL) ? 1 : 0;
+  D.max_queries = c->max_queries;
   return D;
 }
 
@@ -134,6 +137,12 @@ inline CacheView view_of(const qwm_cache* c) {
   v.eigvec = (double*)c->buf.ptr[QWM_BUF_EIGVEC];
   v.workspace = c->buf.ptr[QWM_BUF_WORKSPACE];
   return v;
+}
+
+// Attention partials of a split key range: per range, [nq][H][d] fp32 outputs
+// (each normalized by its own softmax sum) then [nq][H] fp32 log-sum-exps.
+inline size_t attn_partial_bytes(const Dims& D, int64_t nq, int nsplit) {
+  return (size_t)nsplit * (size_t)nq * D.H * (D.d + 1) * 4;
 }
 
 // The centroid tables of one version: [H][C][d] bf16 starting at the slot.

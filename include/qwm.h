@@ -65,7 +65,15 @@ typedef enum qwm_status {
 /* Quantizer and capacity.  Supported: head_dim 64 or 128; group 16 or 32 and
  * dividing head_dim; 1 <= n_centroids <= 512; 1 <= n_cand <= min(8, C);
  * 0 <= rank <= 16; 1 <= max_versions <= 65535; 1 <= max_cent_versions <= 65535;
- * max_tokens >= 1; flags a combination of the QWM_FLAG_* bits. */
+ * 0 <= max_queries <= 2^24; max_tokens >= 1; flags a combination of the
+ * QWM_FLAG_* bits. */
+
+/* Split of the key range across CTA pairs in qwm_attention: at most this many
+ * key ranges, each giving an fp32 partial result per query row and head that a
+ * final pass merges through the log-sum-exp.  The WORKSPACE buffer holds the
+ * partials for up to max_queries query rows; calls with more rows (or
+ * max_queries == 0) attend over the whole key range in one pass. */
+#define QWM_ATTN_MAX_SPLIT 6
 
 /* QSAC stage 2 with the full quadratic form: each shortlisted centroid c is
  * scored by e^T A e, where e = k - (c + deq(INT2(k - c))) is the Key error
@@ -87,6 +95,8 @@ typedef struct qwm_config {
   int32_t max_versions; /* slots for successive bases U (one per refresh) */
   int32_t flags;        /* QWM_FLAG_* bits (0: the method as described)   */
   int32_t max_cent_versions; /* slots for successive centroid tables      */
+  int32_t max_queries;  /* query rows per attention call the WORKSPACE
+                           holds split-key partials for (0: none)         */
   int64_t max_tokens;   /* cache capacity per head                       */
 } qwm_config;
 
@@ -112,7 +122,10 @@ typedef struct qwm_config {
  *                                      in force ([d][d] fp32 from double offset
  *                                      32 d); after all heads one warm-start flag
  *                                      per head
- *   WORKSPACE                  bytes   scratch for centroid building and basis refresh */
+ *   WORKSPACE                  bytes   scratch for centroid building, basis refresh
+ *                                      and attention partials: at least
+ *                                      QWM_ATTN_MAX_SPLIT x max_queries x H x
+ *                                      (d + 1) fp32 */
 typedef enum qwm_buffer_id {
   QWM_BUF_K_CODES = 0, QWM_BUF_K_PARAMS, QWM_BUF_K_IDX, QWM_BUF_K_COEF, QWM_BUF_K_CSCALE,
   QWM_BUF_V_CODES, QWM_BUF_V_PARAMS, QWM_BUF_V_IDX, QWM_BUF_CENT_K, QWM_BUF_CENT_V,

@@ -16,6 +16,7 @@ int main(void) {
   printf("nbuf %d\n", (int)QWM_NBUF);
   printf("noalloc_bytes %u\n", (unsigned)QWM_NOALLOC_SCRATCH_BYTES);
   printf("flag_qsac_full %d\n", (int)QWM_FLAG_QSAC_FULL);
+  printf("attn_max_split %d\n", (int)QWM_ATTN_MAX_SPLIT);
   printf("size qwm_config %zu\n", sizeof(qwm_config));
   printf("size qwm_sizes %zu\n", sizeof(qwm_sizes));
   printf("size qwm_buffers %zu\n", sizeof(qwm_buffers));
@@ -23,7 +24,8 @@ int main(void) {
   FIELD(qwm_config, heads); FIELD(qwm_config, head_dim); FIELD(qwm_config, n_centroids);
   FIELD(qwm_config, group); FIELD(qwm_config, n_cand); FIELD(qwm_config, rank);
   FIELD(qwm_config, max_versions); FIELD(qwm_config, flags);
-  FIELD(qwm_config, max_cent_versions); FIELD(qwm_config, max_tokens);
+  FIELD(qwm_config, max_cent_versions); FIELD(qwm_config, max_queries);
+  FIELD(qwm_config, max_tokens);
   FIELD(qwm_sizes, bytes); FIELD(qwm_sizes, tcap); FIELD(qwm_sizes, bytes_per_token_head);
   FIELD(qwm_cache, cfg); FIELD(qwm_cache, buf); FIELD(qwm_cache, tcap); FIELD(qwm_cache, len);
   FIELD(qwm_cache, n_queries); FIELD(qwm_cache, frames); FIELD(qwm_cache, n_versions);
@@ -37,7 +39,7 @@ int main(void) {
   /* the 480p layer's configuration, two centroid-table slots */
   qwm_config cfg = {.heads = 40, .head_dim = 128, .n_centroids = 256, .group = 32,
                     .n_cand = 4, .rank = 8, .max_versions = 64, .flags = 0,
-                    .max_cent_versions = 2, .max_tokens = 37440};
+                    .max_cent_versions = 2, .max_queries = 1560, .max_tokens = 37440};
   qwm_sizes s;
   qwm_status st = qwm_cache_sizes(&cfg, &s);
   printf("sizes_status %d\n", (int)st);

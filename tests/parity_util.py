@@ -35,10 +35,12 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 
 def make_gpu_cache(c: syn.LayerConfig, max_tokens=None, max_versions=None) -> q.QuantKVCache:
+    """The layer's cache as the benchmark makes it: workspace for split-key
+    attention partials of one frame's query chunk."""
     T = c.total_tokens if max_tokens is None else max_tokens
     nv = (c.frames // c.refresh_every + 2) if max_versions is None else max_versions
     return q.QuantKVCache(c.heads, c.head_dim, c.n_centroids, c.group, c.n_cand, c.rank, T,
-                          max_versions=nv)
+                          max_versions=nv, max_queries=c.q_rows)
 
 
 def make_oracle_cache(c: syn.LayerConfig) -> oracle.OracleCache:

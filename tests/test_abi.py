@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 def _cfg(**kw):
     base = dict(heads=40, head_dim=128, n_centroids=256, group=32, n_cand=4, rank=8,
-                max_versions=64, flags=0, max_cent_versions=1, max_tokens=37440)
+                max_versions=64, flags=0, max_cent_versions=1, max_queries=0, max_tokens=37440)
     base.update(kw)
     return q.qwm_config(**base)
 
@@ -64,7 +64,8 @@ def test_sizes_follow_layout():
                                  dict(n_centroids=513), dict(n_cand=9), dict(n_cand=300),
                                  dict(rank=17), dict(max_versions=0), dict(flags=2), dict(flags=-1),
                                  dict(max_tokens=0), dict(heads=0), dict(max_cent_versions=0),
-                                 dict(max_cent_versions=65536)])
+                                 dict(max_cent_versions=65536), dict(max_queries=-1),
+                                 dict(max_queries=(1 << 24) + 1)])
 def test_invalid_configs_rejected(bad):
     out = q.qwm_sizes()
     st = q.lib().qwm_cache_sizes(ctypes.byref(_cfg(**bad)), ctypes.byref(out))
@@ -169,6 +170,7 @@ def test_struct_layout_matches_header():
     assert int(d["nbuf"]) == q.NBUF == len(q.BUFFER_NAMES) == 18
     assert int(d["noalloc_bytes"]) == q.QWM_NOALLOC_SCRATCH_BYTES
     assert int(d["flag_qsac_full"]) == q.QWM_FLAG_QSAC_FULL
+    assert int(d["attn_max_split"]) == q.QWM_ATTN_MAX_SPLIT
     for name, st in (("qwm_config", q.qwm_config), ("qwm_sizes", q.qwm_sizes),
                      ("qwm_buffers", q.qwm_buffers), ("qwm_cache", q.qwm_cache)):
         assert int(d[f"size {name}"]) == ctypes.sizeof(st), name
@@ -179,12 +181,24 @@ def test_struct_layout_matches_header():
             assert getattr(st, field).offset == int(v), key
     for e in ("K_CODES", "CENT_K", "TOKVER", "CENTVER", "WORKSPACE"):
         assert q.BUFFER_NAMES[int(d[f"enum QWM_BUF_{e}"])] == e.lower(), e
-    s = q.qwm_cache_sizes(_cfg(max_cent_versions=2))
+    s = q.qwm_cache_sizes(_cfg(max_cent_versions=2, max_queries=1560))
     assert int(d["sizes_status"]) == 0 and int(d["sizes_bad_status"]) == 1
     assert int(d["sizes_tcap"]) == s.tcap and int(d["sizes_bpth"]) == s.bytes_per_token_head
     for i in range(q.NBUF):
         assert int(d[f"sizes_bytes_{i}"]) == s.bytes[i], q.BUFFER_NAMES[i]
     assert d["status_capacity"] == q.qwm_status_string(3) == "capacity exceeded"
+
+
+def test_workspace_holds_split_attention_partials():
+    """The WORKSPACE buffer covers QWM_ATTN_MAX_SPLIT fp32 partial outputs and
+    log-sum-exps of max_queries rows and every head (and is never smaller than
+    the centroid build's scratch)."""
+    ws = q.BUFFER_NAMES.index("workspace")
+    base = q.qwm_cache_sizes(_cfg()).bytes[ws]
+    s = q.qwm_cache_sizes(_cfg(max_queries=1560))
+    need = q.QWM_ATTN_MAX_SPLIT * 1560 * 40 * (128 + 1) * 4
+    assert s.bytes[ws] == max(need, base)
+    assert q.qwm_cache_sizes(_cfg(max_queries=1)).bytes[ws] == base
 
 
 def test_centroid_versions_sizes_and_capacity():

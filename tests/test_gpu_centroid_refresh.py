@@ -33,7 +33,7 @@ def _layer(heads, n, frames, rebuild_every, refresh_every):
     H, d, C = len(heads), c.head_dim, c.n_centroids
     nver = frames // rebuild_every + 1
     g = q.QuantKVCache(H, d, C, c.group, c.n_cand, c.rank, frames * n,
-                       max_versions=frames + 2, max_cent_versions=nver)
+                       max_versions=frames + 2, max_cent_versions=nver, max_queries=n)
     oc = oracle.OracleCache(H, d, C, c.group, c.n_cand, c.rank, frames * n)
     Mref = {h: np.zeros((d, d)) for h in range(H)}
     rep = new_state_report()

@@ -219,7 +219,8 @@ def test_head128_shapes(G, C, M, r):
     (M = 1), and ranks 2 and 4."""
     H, d, n = 3, 128, 700
     q = pytest.importorskip("bit_kv_cache_23_b200")
-    g = q.QuantKVCache(H, d, C, G, M, r, 3 * n, max_versions=8)
+    # workspace for split-key attention (the key range is split across pairs)
+    g = q.QuantKVCache(H, d, C, G, M, r, 3 * n, max_versions=8, max_queries=200)
     oc = oracle.OracleCache(H, d, C, G, M, r, 3 * n)
     rng = np.random.default_rng(1000 + G + C + r)
     w = np.ones(d)

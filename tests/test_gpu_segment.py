@@ -30,13 +30,13 @@ def _bf(x):
     return syn.f32_to_bf16_bits(np.asarray(x, np.float32))
 
 
-def _filled_cache(H, d, C, G, M, r, frames, n, seed):
+def _filled_cache(H, d, C, G, M, r, frames, n, seed, max_queries=0):
     """GPU cache and oracle cache, filled with the same frames, both encoding with
     the oracle's own state; returns (g, oc, frames of (Q, K, V))."""
     q = pytest.importorskip("bit_kv_cache_23_b200")
     rng = np.random.default_rng(seed)
     T = frames * n
-    g = q.QuantKVCache(H, d, C, G, M, r, T, max_versions=frames + 2)
+    g = q.QuantKVCache(H, d, C, G, M, r, T, max_versions=frames + 2, max_queries=max_queries)
     oc = oracle.OracleCache(H, d, C, G, M, r, T)
     w = np.ones(d)
     w[rng.permutation(d)[:4]] = 6.0
@@ -108,14 +108,16 @@ def _run_ext(g, Q, Kseg, Vseg):
     return u16(O), lse.cpu().numpy()
 
 
-@pytest.mark.parametrize("d,C,G,M,r,n,nseg,nq", [
-    (128, 64, 32, 4, 8, 700, 300, 300),    # tensor-core kernel, ragged tiles, two CTAs
-    (128, 64, 16, 1, 0, 650, 64, 130),     # no compensation (rank 0), one full segment tile
-    (64, 16, 16, 4, 4, 300, 77, 70),       # CUDA-core kernel
+@pytest.mark.parametrize("d,C,G,M,r,n,nseg,nq,split", [
+    (128, 64, 32, 4, 8, 700, 300, 300, False),   # tensor-core kernel, ragged tiles, one pair
+    (128, 64, 32, 4, 8, 700, 300, 300, True),    # the same with the key range split across pairs
+    (128, 64, 16, 1, 0, 650, 64, 130, True),     # no compensation (rank 0), one full segment tile
+    (64, 16, 16, 4, 4, 300, 77, 70, False),      # CUDA-core kernel
 ])
-def test_history_plus_segment(d, C, G, M, r, n, nseg, nq):
+def test_history_plus_segment(d, C, G, M, r, n, nseg, nq, split):
     H = 3 if d == 128 else 2
-    g, oc, data = _filled_cache(H, d, C, G, M, r, 2, n, seed=500 + d + r)
+    g, oc, data = _filled_cache(H, d, C, G, M, r, 2, n, seed=500 + d + r,
+                                max_queries=nq if split else 0)
     rng = np.random.default_rng(600 + d)
     Kseg = _bf(rng.standard_normal((nseg, H, d)) * 1.5)
     Vseg = _bf(rng.standard_normal((nseg, H, d)))
