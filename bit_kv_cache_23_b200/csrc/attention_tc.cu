@@ -276,42 +276,47 @@ __device__ __forceinline__ void softmax_role(const TcArgs& A, uint64_t* bars, ui
         // tracks every MMA issued before Q K'^T of tile j.
         const float f = need ? ex2(m_used - m_row) : 1.0f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(to + c * 32, o);
-          uint32_t ou[32];
+        for (int c = 0; c < 16; ++c) {
+          float o[8];
+          tmem_ld8(to + c * 8, o);
+          uint32_t ou[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(o[e] * f);
-          tmem_st32u(to + c * 32, ou);
+          for (int e = 0; e < 8; ++e) ou[e] = __float_as_uint(o[e] * f);
+          tmem_st8u_nw(to + c * 8, ou);
+          tmem_wait_st();
         }
         l2 = ffma2(l2, f2pack(f, f), 0ull);
         if (need) m_used = m_row;
       }
     }
     // P (bf16 pairs) over the S columns already read: keys 2i, 2i+1 of the tile
-    // in column i (the A-operand layout of the P V' MMA).
+    // in column i (the A-operand layout of the P V' MMA); the scores are read
+    // again 32 columns at a time.
     const uint64_t nm2 = f2pack(-m_used, -m_used);
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int h2 = 0; h2 < 2; ++h2) {
       float s[32];
-      tmem_ld32(ts + c * 32, s);
-      uint32_t pk[16];
+      tmem_ld32(ts + 32 * h2, s);
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
+    for (int c = 2 * h2; c < 2 * h2 + 2; ++c) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
         float x0, x1;
-        f2unpack(ffma2(f2pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+        f2unpack(ffma2(f2pack(s[16 * (c & 1) + e], s[16 * (c & 1) + e + 1]), sc2, nm2), x0, x1);
         float p0 = ex2(x0), p1 = ex2(x1);
         if (nvalid < KT) {
-          const int col = c * 32 + e;
+          const int col = c * 16 + e;
           if (col >= nvalid) p0 = 0.0f;
           if (col + 1 >= nvalid) p1 = 0.0f;
         }
-        const uint64_t pp = f2pack(p0, p1);
-        l2 = fadd2(l2, pp);
+        l2 = fadd2(l2, f2pack(p0, p1));
         pk[e / 2] = pack_bf16(p0, p1);
       }
-      tmem_st16u(ts + c * 16, pk);
+      tmem_st8u_nw(ts + c * 8, pk);
     }
+    }
+    tmem_wait_st();
     tc_fence_before();
     warp_arrive_lead(&bars[B_P_FULL + p]);
   }
@@ -472,14 +477,11 @@ __device__ __forceinline__ void corr_global(const float* Uj0, const int8_t* cf, 
   }
 }
 
-// Rewrite chunk c (8 channels) of row `row` of an R-row swizzled tile in place:
+// Rewrite the 8-channel chunk at byte `off` of a swizzled stage tile in place:
 // centroid chunk from the stage, residual (and compensation) added in fp32, one
 // bf16 rounding.
-template <int R>
-__device__ __forceinline__ void deq_chunk(uint8_t* base, int row, int c, uint32_t bits16,
-                                          uint32_t par, const uint64_t* corr) {
-  const GroupConst g = group_const(par);
-  const uint32_t off = sw128_off(row, c, R);
+__device__ __forceinline__ void deq_chunk(uint8_t* base, uint32_t off, uint32_t bits16,
+                                          const GroupConst& g, const uint64_t* corr) {
   const uint4 cw = *reinterpret_cast<const uint4*>(base + off);
   uint64_t v2[4];
   deq_chunk_f32(cw, bits16, g, v2);
@@ -490,9 +492,8 @@ __device__ __forceinline__ void deq_chunk(uint8_t* base, int row, int c, uint32_
   *reinterpret_cast<uint4*>(base + off) = pack_chunk(v2);
 }
 
-template <int R>
-__device__ __forceinline__ void zero_chunk(uint8_t* base, int row, int c) {
-  *reinterpret_cast<uint4*>(base + sw128_off(row, c, R)) = make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void zero_chunk(uint8_t* base, uint32_t off) {
+  *reinterpret_cast<uint4*>(base + off) = make_uint4(0, 0, 0, 0);
 }
 
 // This thread's share of a tile (rank = CTA in the pair, sw = dequant warp):
@@ -501,6 +502,8 @@ __device__ __forceinline__ void zero_chunk(uint8_t* base, int row, int c) {
 //       this CTA's 64-channel half).
 struct DqShare {
   int kk, sw, lane, cvc;
+  uint32_t koff[2];   // stage offsets of the K' chunks (row lane, chunks 2sw, 2sw+1)
+  uint32_t voff[2];   // stage offsets of the V' chunk (rows lane, lane+32, chunk sw)
 };
 
 // Issue the 16-byte centroid-chunk copies of tile jj, each from the table
@@ -515,11 +518,8 @@ __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, con
   if (t0 + d.kk < A.T) {
     const uint16_t* ck = ph.cent_k + (size_t)cvs[d.kk] * ph.cstride +
                          (size_t)staged_idx(pk, PK_KIDX, d.kk, ib) * DH;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 2 * d.sw + cc;
-      cp_async16_cg(st + ST_K + sw128_off(d.lane, c, KH), ck + c * 8);
-    }
+    cp_async16_cg(st + d.koff[0], ck + 16 * d.sw);
+    cp_async16_cg(st + d.koff[1], ck + 16 * d.sw + 8);
   }
 #pragma unroll
   for (int kk = 0; kk < 2; ++kk) {
@@ -527,7 +527,7 @@ __device__ __forceinline__ void issue_gather(const TcArgs& A, uint8_t* smem, con
     if (t0 + k < A.T) {
       const uint16_t* cv = ph.cent_v + (size_t)cvs[k] * ph.cstride +
                            (size_t)staged_idx(pk, PK_VIDX, k, ib) * DH;
-      cp_async16_cg(st + ST_V + sw128_off(k, d.sw, KT), cv + d.cvc * 8);
+      cp_async16_cg(st + d.voff[kk], cv + d.cvc * 8);
     }
   }
   cp_async_commit();
@@ -541,18 +541,15 @@ __device__ __forceinline__ void issue_seg_gather(const TcArgs& A, uint8_t* smem,
   const int64_t t0 = (int64_t)(jj - A.ntp) * KT;
   if (t0 + d.kk < A.nseg) {
     const uint16_t* kr = A.Ks + ((size_t)(t0 + d.kk) * A.Dm.H + blockIdx.y) * DH;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 2 * d.sw + cc;
-      cp_async16_cg(st + ST_K + sw128_off(d.lane, c, KH), kr + c * 8);
-    }
+    cp_async16_cg(st + d.koff[0], kr + 16 * d.sw);
+    cp_async16_cg(st + d.koff[1], kr + 16 * d.sw + 8);
   }
 #pragma unroll
   for (int kk = 0; kk < 2; ++kk) {
     const int k = d.lane + 32 * kk;
     if (t0 + k < A.nseg) {
       const uint16_t* vr = A.Vs + ((size_t)(t0 + k) * A.Dm.H + blockIdx.y) * DH;
-      cp_async16_cg(st + ST_V + sw128_off(k, d.sw, KT), vr + d.cvc * 8);
+      cp_async16_cg(st + d.voff[kk], vr + d.cvc * 8);
     }
   }
   cp_async_commit();
@@ -567,6 +564,10 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
   d.lane = dq & 31;
   d.kk = KH * (int)rank + d.lane;
   d.cvc = 8 * (int)rank + d.sw;
+  d.koff[0] = ST_K + sw128_off(d.lane, 2 * d.sw, KH);
+  d.koff[1] = ST_K + sw128_off(d.lane, 2 * d.sw + 1, KH);
+  d.voff[0] = ST_V + sw128_off(d.lane, d.sw, KT);
+  d.voff[1] = ST_V + sw128_off(d.lane + 32, d.sw, KT);
   const Dims& Dm = A.Dm;
   const int h = blockIdx.y;
   const PackedHead ph = packed_head(A.v, Dm, h);
@@ -606,18 +607,16 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
     }
     const int s = jl % NKV, sp = jl % NPK;
     uint8_t* st = smem + OFF_KV + s * KVST;
-    uint8_t* kb = st + ST_K;
-    uint8_t* vb = st + ST_V;
     if (SEG && j >= ntp) {
       // segment tile: rows already in place; zero rows past the segment's end
       const int64_t t0 = (int64_t)(j - ntp) * KT;
       if (t0 + d.kk >= A.nseg) {
-        zero_chunk<KH>(kb, d.lane, 2 * d.sw);
-        zero_chunk<KH>(kb, d.lane, 2 * d.sw + 1);
+        zero_chunk(st, d.koff[0]);
+        zero_chunk(st, d.koff[1]);
       }
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk)
-        if (t0 + d.lane + 32 * kk >= A.nseg) zero_chunk<KT>(vb, d.lane + 32 * kk, d.sw);
+        if (t0 + d.lane + 32 * kk >= A.nseg) zero_chunk(st, d.voff[kk]);
       fence_proxy_async_smem();
       warp_arrive_lead(&bars[B_KV_FULL + s]);
       continue;
@@ -643,11 +642,12 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
         else if (r <= 8 && ver == tv[nval - 1]) corr_staged(us + r * DH, kcf, cs, r, corr);
         else corr_global(ubase + (size_t)ver * ustride, kcf, cs, r, corr);
       }
-      deq_chunk<KH>(kb, d.lane, 2 * d.sw, kw & 0xffffu, kp, r > 0 ? corr : nullptr);
-      deq_chunk<KH>(kb, d.lane, 2 * d.sw + 1, kw >> 16, kp, r > 0 ? corr + 4 : nullptr);
+      const GroupConst g = group_const(kp);  // both chunks lie in one INT2 group
+      deq_chunk(st, d.koff[0], kw & 0xffffu, g, r > 0 ? corr : nullptr);
+      deq_chunk(st, d.koff[1], kw >> 16, g, r > 0 ? corr + 4 : nullptr);
     } else {
-      zero_chunk<KH>(kb, d.lane, 2 * d.sw);
-      zero_chunk<KH>(kb, d.lane, 2 * d.sw + 1);
+      zero_chunk(st, d.koff[0]);
+      zero_chunk(st, d.koff[1]);
     }
     // ---- V': this CTA's channel chunk of keys lane and lane + 32
 #pragma unroll
@@ -656,9 +656,9 @@ __device__ __forceinline__ void dequant_role(const TcArgs& A, uint8_t* smem, uin
       if (t0 + k < A.T) {
         const uint32_t vw = *reinterpret_cast<const uint16_t*>(pk + PK_VCODE + k * 32 + 2 * d.cvc);
         const uint32_t vp = reinterpret_cast<const uint32_t*>(pk + PK_VPAR)[k * ng + giv];
-        deq_chunk<KT>(vb, k, d.sw, vw, vp, nullptr);
+        deq_chunk(st, d.voff[kk], vw, group_const(vp), nullptr);
       } else {
-        zero_chunk<KT>(vb, k, d.sw);
+        zero_chunk(st, d.voff[kk]);
       }
     }
     fence_proxy_async_smem();
