@@ -167,7 +167,7 @@ __device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t*
 }
 
 template <bool KEY, int G, int NT>
-__global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
+__device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   using L = Lay<NT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -359,6 +359,9 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
   float topv[8];
 #pragma unroll
   for (int m = 0; m < 8; ++m) topv[m] = INFINITY;
+  // list length: the shortlist size rounded up to 1, 4 or 8 (shorter lists
+  // need fewer compare-exchanges per group)
+  const int tl = Mc <= 1 ? 1 : (Mc <= 4 ? 4 : 8);
 #pragma unroll 1
   for (int c0 = 0; c0 < nchunk * NCH; c0 += 32) {
     float v[32];
@@ -370,11 +373,23 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x = fminf(x, v[8 * gq + e]);
       }
+      // insertion into the sorted list
+      if (tl == 1) {
+        topv[0] = fminf(topv[0], x);
+      } else if (tl == 4) {
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {  // insertion into the sorted list
-        const float lo = fminf(topv[m], x);
-        x = fmaxf(topv[m], x);
-        topv[m] = lo;
+        for (int m = 0; m < 4; ++m) {
+          const float lo = fminf(topv[m], x);
+          x = fmaxf(topv[m], x);
+          topv[m] = lo;
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float lo = fminf(topv[m], x);
+          x = fmaxf(topv[m], x);
+          topv[m] = lo;
+        }
       }
     }
   }
@@ -410,7 +425,16 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
   float candD[8];
 #pragma unroll
   for (int m = 0; m < 8; ++m) { cand[m] = -1; candD[m] = INFINITY; }
-  if (valid) {
+  // With exactly Mc survivors they are the shortlist (every member of the exact
+  // top Mc survives); their order by (D, i) is needed only to break a tie of
+  // the stage-2 score (or never, for a shortlist of one), so the exact
+  // distances are computed later for tied candidates only.
+  const bool exact_set = (cnt == Mc);
+  if (valid && exact_set) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (m < Mc) cand[m] = (int)surv[tid * SURV_MAX + m];
+  } else if (valid) {
     const bool all = cnt > SURV_MAX || cnt < Mc;  // overflow, or no usable approximation
     const int nloop = all ? C : cnt;
 #pragma unroll 1
@@ -454,6 +478,8 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
   if (KEY && Mc > 1) {
     float best = 0.0f;
     int bm = -1;
+    uint32_t tied = 0;  // candidates whose score equals the lowest so far
+    float scores[8];
 #pragma unroll 1
     for (int m = 0; m < Mc; ++m) {
       int cm = cand[0];
@@ -480,12 +506,39 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
         const float R = __fsub_rn(hi, lo);
         score = __fmaf_rn(w_s[g], __fmul_rn(R, R), score);
       }
+#pragma unroll
+      for (int mm = 0; mm < 8; ++mm)
+        if (mm == m) scores[mm] = score;
       if (bm < 0 || score < best) {
         best = score;
         bm = m;
         a = cm;
+        tied = 1u << m;
+      } else if (score == best) {
+        tied |= 1u << m;
       }
     }
+    if (exact_set && __popc(tied) > 1) {
+      // a tie among unordered candidates: the earliest in (D, i) order wins
+      float bd = INFINITY;
+      int bi = -1;
+#pragma unroll 1
+      for (int m = 0; m < Mc; ++m) {
+        if (!((tied >> m) & 1u)) continue;
+        int cm = cand[0];
+#pragma unroll
+        for (int mm = 0; mm < 8; ++mm)
+          if (mm == m) cm = cand[mm];
+        float D, Dx;
+        canon_dist2<KEY>(krow, bt, cent, C, cm, cm, s_s, D, Dx);
+        if (bi < 0 || lex_less(D, cm, bd, bi)) {
+          bd = D;
+          bi = cm;
+        }
+      }
+      a = bi;
+    }
+    (void)scores;
   }
 
   // ---- P7: INT2 residual and PSAC coefficients, group by group in channel order
@@ -582,23 +635,30 @@ __global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs A) {
   }
 }
 
-template <bool KEY, int G, int NT>
-cudaError_t run_tc(const ApArgs& a, cudaStream_t s) {
+// Keys (blockIdx.z == 0) and Values (z == 1) in one launch: the Value CTAs,
+// which finish sooner, fill the last wave of the Key CTAs.
+template <int G, int NT>
+__global__ void __launch_bounds__(NT, 1) append_tc_kernel(const ApArgs AK, const ApArgs AV) {
+  if (blockIdx.z == 0) append_tc_body<true, G, NT>(AK);
+  else append_tc_body<false, G, NT>(AV);
+}
+
+template <int G, int NT>
+cudaError_t run_tc(const ApArgs& ak, const ApArgs& av, cudaStream_t s) {
   const int smem = (int)Lay<NT>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<KEY, G, NT>,
+  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel<G, NT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.n + NT - 1) / NT), a.H);
-  append_tc_kernel<KEY, G, NT><<<grid, NT, smem, s>>>(a);
+  dim3 grid((unsigned)((ak.n + NT - 1) / NT), ak.H, 2);
+  append_tc_kernel<G, NT><<<grid, NT, smem, s>>>(ak, av);
   return cudaGetLastError();
 }
 
 // 256 tokens per CTA (two MMA halves sharing one B tile) when the centroid
 // table fits one 256-row tile, else 128.
-template <bool KEY>
-cudaError_t run_tc_g(const ApArgs& a, cudaStream_t s) {
-  if (a.C <= NCH) return a.G == 32 ? run_tc<KEY, 32, 256>(a, s) : run_tc<KEY, 16, 256>(a, s);
-  return a.G == 32 ? run_tc<KEY, 32, 128>(a, s) : run_tc<KEY, 16, 128>(a, s);
+cudaError_t run_tc_g(const ApArgs& ak, const ApArgs& av, cudaStream_t s) {
+  if (ak.C <= NCH) return ak.G == 32 ? run_tc<32, 256>(ak, av, s) : run_tc<16, 256>(ak, av, s);
+  return ak.G == 32 ? run_tc<32, 128>(ak, av, s) : run_tc<16, 128>(ak, av, s);
 }
 
 }  // namespace
@@ -643,16 +703,15 @@ cudaError_t launch_append_tc(const Dims& Dm, const CacheView& v, const uint16_t*
   a.cscale = v.k_cscale;
   a.tokver = v.tokver;
   a.centver = v.centver;
-  cudaError_t e = run_tc_g<true>(a, s);
-  if (e != cudaSuccess) return e;
-  a.X = V;
-  a.cent = v.cent_v + coff;
-  a.codes = v.v_codes;
-  a.params = v.v_params;
-  a.idx = v.v_idx;
-  a.coef = nullptr;
-  a.cscale = nullptr;
-  return run_tc_g<false>(a, s);
+  ApArgs b = a;
+  b.X = V;
+  b.cent = v.cent_v + coff;
+  b.codes = v.v_codes;
+  b.params = v.v_params;
+  b.idx = v.v_idx;
+  b.coef = nullptr;
+  b.cscale = nullptr;
+  return run_tc_g(a, b, s);
 }
 
 }  // namespace qwm
