@@ -362,43 +362,66 @@ __global__ void __launch_bounds__(P == 32 ? 256 : 512) refresh_kernel(const doub
     }
   }
   __syncthreads();
-  // ---- orthogonal iteration: a fixed number of steps (the top-r subspace
-  // converges at rate lambda_{p+1}/lambda_r per step; the trailing part of the
-  // block may be nearly degenerate, so the block as a whole is not a stopping
-  // test).  Warm starts track a basis that moves little between refreshes.
-  const int iters = warm ? 3 : 30;
+  // ---- orthogonal iteration (the top-r subspace converges at rate
+  // lambda_{p+1}/lambda_r per step), then a Rayleigh-Ritz step whose residuals
+  // decide whether to go on: every one of the top r Ritz pairs must satisfy
+  // |A v - theta v| <= 1e-7 theta_1, else 8 more steps follow, up to a bound.
+  // Warm starts track a basis that moves little between refreshes.
+  const int cap = warm ? 64 : 160;
+  int target = warm ? 3 : 30;
+  int it = 0;
   double* Xc = S.X;  // the current block; the product goes to the other buffer
   double* Yc = S.Y;
-  for (int it = 0; it < iters; ++it) {
+  double* Hc = S.G;  // Rayleigh quotient, rotated in place by the Jacobi
+  double* W = S.L;   // its eigenvectors
+  while (true) {
+    for (; it < target; ++it) {
+      cholqr<D, P>(Xc, S.G, S.L);
+      gemm_AX<D, P>(S.A, Xc, Yc);
+      double* t = Xc;
+      Xc = Yc;
+      Yc = t;
+    }
     cholqr<D, P>(Xc, S.G, S.L);
-    gemm_AX<D, P>(S.A, Xc, Yc);
-    double* t = Xc;
-    Xc = Yc;
-    Yc = t;
+    cholqr<D, P>(Xc, S.G, S.L);
+    gemm_AX<D, P>(S.A, Xc, Yc);              // Y = A Q
+    gram(Xc, Yc, Hc, d, p);                  // H = Q^T A Q (column-major, symmetric)
+    small_jacobi<P>(Hc, W);
+    if (tid < p) {
+      double acc = 0.0;
+      for (int i = 0; i < p; ++i) acc += Hc[tid * p + i] * Hc[tid * p + i];
+      S.th[tid] = sqrt(acc);
+    }
+    __syncthreads();
+    if (tid < p) {
+      const double v = S.th[tid];
+      int rank = 0;
+      for (int j = 0; j < p; ++j) rank += (S.th[j] > v) || (S.th[j] == v && j < tid);
+      S.ord[rank] = tid;
+    }
+    if (tid < 32) S.red[tid] = 0.0;
+    __syncthreads();
+    // squared residuals of the top r Ritz pairs: (Y W_k - theta_k Q W_k)_i
+    const int rr = r < p ? r : p;
+    for (int e = tid; e < rr * d; e += nt) {
+      const int c = e / d, i = e % d;
+      const int k = S.ord[c];
+      double av = 0.0, v = 0.0;
+      for (int m = 0; m < p; ++m) {
+        av = fma(Yc[m * (d + 1) + i], W[k * p + m], av);
+        v = fma(Xc[m * (d + 1) + i], W[k * p + m], v);
+      }
+      const double res = av - S.th[k] * v;
+      atomicAdd(&S.red[c], res * res);
+    }
+    __syncthreads();
+    bool done = true;
+    const double tol = 1e-7 * S.th[S.ord[0]];
+    for (int c = 0; c < rr; ++c) done = done && (sqrt(S.red[c]) <= tol);
+    if (done || it >= cap) break;
+    target = it + 8;
+    __syncthreads();
   }
-  // ---- Rayleigh-Ritz on the final block
-  cholqr<D, P>(Xc, S.G, S.L);
-  cholqr<D, P>(Xc, S.G, S.L);
-  gemm_AX<D, P>(S.A, Xc, Yc);
-  gram(Xc, Yc, S.G, d, p);                 // H = Q^T A Q (column-major, symmetric)
-  double* W = Yc;                          // Y is free again: W [p][p] in its space
-  double* Hc = Yc + p * p;                 // copy of H to rotate
-  for (int e = tid; e < p * p; e += nt) Hc[e] = S.G[e];
-  __syncthreads();
-  small_jacobi<P>(Hc, W);
-  if (tid < p) {
-    double acc = 0.0;
-    for (int i = 0; i < p; ++i) acc += Hc[tid * p + i] * Hc[tid * p + i];
-    S.th[tid] = sqrt(acc);
-  }
-  __syncthreads();
-  if (tid < p) {
-    const double v = S.th[tid];
-    int rank = 0;
-    for (int j = 0; j < p; ++j) rank += (S.th[j] > v) || (S.th[j] == v && j < tid);
-    S.ord[rank] = tid;
-  }
-  __syncthreads();
   // Ritz vectors V = Q W (sorted), written to eigvec (column-major) for the
   // next warm start; the first r columns, sign-normalized, are U.
   double* Vout = eigvec + (size_t)h * d * d;
