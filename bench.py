@@ -189,17 +189,20 @@ class Workload:
     """The layer (or this rank's block of its heads) filled with all its frames."""
 
     def __init__(self, cfg: syn.LayerConfig, device, extra_versions: int, pool: int = 4,
-                 heads=None):
+                 heads=None, rebuild_every: int = 0):
         import bit_kv_cache_23_b200 as q
 
         self.cfg = cfg
         self.device = device
         c = cfg
         self.heads = list(range(c.heads)) if heads is None else list(heads)
+        nrb = (c.frames - 1) // rebuild_every if rebuild_every > 0 else 0
         self.cache = q.QuantKVCache(len(self.heads), c.head_dim, c.n_centroids, c.group,
                                     c.n_cand, c.rank, c.total_tokens,
                                     max_versions=c.frames // c.refresh_every + extra_versions + 4,
-                                    device=device, max_queries=c.q_rows)
+                                    device=device, max_queries=c.q_rows,
+                                    max_cent_versions=nrb + 1)
+        self.rebuilds = 0
         src = syn.FrameSource(c)
         self.src = src
         self.pool = []
@@ -208,8 +211,11 @@ class Workload:
         for f in range(c.frames):
             Q, K, V = src.frame(f, hs)
             Qd, Kd, Vd = dev_bf16(Q, device), dev_bf16(K, device), dev_bf16(V, device)
-            if f == 0:
+            if f == 0 or (rebuild_every > 0 and f % rebuild_every == 0):
+                # the first tables, then (with rebuild_every) a new table version
+                # from the newest frame under Key drift
                 self.cache.build_centroids(Kd, Vd, iters=c.kmeans_iters)
+                self.rebuilds += f > 0
             self.cache.update_query_stats(Qd, refresh_basis=(f % c.refresh_every) == 0)
             self.cache.append_kv(Kd, Vd)
             if f >= c.frames - pool:
@@ -540,6 +546,10 @@ def main():
     ap.add_argument("--ablation", action="store_true",
                     help="instead of timing, print one JSON line per quantization setting "
                          "(QVG, QSAC only, rank sweep, K-only, V-only) with its quality")
+    ap.add_argument("--rebuild-every", type=int, default=0,
+                    help="while filling the cache, rebuild the centroid tables from the newest "
+                         "frame every N frames (a new table version each time; the 1-minute "
+                         "layer's Key distribution drifts)")
     ap.add_argument("--segment", action="store_true",
                     help="instead of the step, time attention over the packed history, over "
                          "history + the frame's bf16 segment, and over all keys in bf16")
@@ -554,6 +564,9 @@ def main():
                      f"{cfg.frames} latent frames x {cfg.tokens_per_frame} tokens, "
                      f"{cfg.q_rows}-query chunk, C={cfg.n_centroids}, G={cfg.group}, "
                      f"M={cfg.n_cand}, r={cfg.rank}")
+    if args.rebuild_every > 0:
+        workload_name += (f", centroid tables rebuilt every {args.rebuild_every} frames "
+                          "(one table version per rebuild)")
 
     if args.segment:
         if rank == 0:
@@ -614,7 +627,8 @@ def main():
         heads = list(range(h0, h1))
     else:
         heads = None
-    wl = Workload(cfg, device, extra_versions=2 * (W + K) + 8, heads=heads)
+    wl = Workload(cfg, device, extra_versions=2 * (W + K) + 8, heads=heads,
+                  rebuild_every=args.rebuild_every)
     nh = len(wl.heads)
     # query tokens of the whole layer this rank serves per step (a fraction of a
     # layer when the heads are split)
@@ -688,7 +702,9 @@ def main():
     per_tok = 2 * (c.head_dim // 4 + 4 * (c.head_dim // c.group) + (1 if c.n_centroids <= 256 else 2)) + c.rank + 2
     app_bytes = c.tokens_per_frame * nh * (4 * c.head_dim + per_tok)
     app_gbs = app_bytes / (app_ms * 1e-3) / 1e9
-    fixed = 2 * c.heads * c.n_centroids * c.head_dim * 2 + (c.frames // c.refresh_every) * c.heads * c.head_dim * c.rank * 4
+    # fixed bytes: every centroid-table version in use and every basis version
+    fixed = ((1 + wl.rebuilds) * 2 * c.heads * c.n_centroids * c.head_dim * 2
+             + (c.frames // c.refresh_every) * c.heads * c.head_dim * c.rank * 4)
     compression = (4.0 * c.head_dim * T * c.heads) / (T * c.heads * per_tok + fixed)
 
     top1 = None
