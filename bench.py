@@ -137,23 +137,26 @@ class ClockSampler:
 
 
 # DRAM bytes (read + write) per attention launch on the 480p workload (24 cached
-# frames): ncu dram__bytes_read.sum + dram__bytes_write.sum captured at 6 cached
-# frames and scaled to 24 by the packed-cache bytes (see the attention profile
-# summary).  Valid only for the kernel source it was taken on (hash below).
-ATTN_TRAFFIC = {"sha256_16": "152b87895d45369e", "config": "480p", "frames": 24,
-                "bytes_per_launch": 63.00e6 + 1.66e6 + (161.7e6 - 40.4e6)}
+# frames), from one ncu capture of dram__bytes_read.sum + dram__bytes_write.sum
+# at that size: 187.3 MB read (the 161.7 MB packed cache, Q, the centroid
+# tables) and 147.5 MB written (the split key ranges' fp32 partials, which the
+# merge kernel reads back, and O).  Valid only for the kernel sources it was
+# taken on (hash of attention_tc.cu, dequant.cuh and tc.cuh below).
+ATTN_TRAFFIC = {"sha256_16": "ced8e64a298ce612", "config": "480p", "frames": 24,
+                "bytes_per_launch": 187332864 + 147464448}
 
 
 def attention_traffic(cfg) -> float | None:
     import hashlib
 
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_kv_cache_23_b200", "csrc",
-                       "attention_tc.cu")
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_kv_cache_23_b200", "csrc")
+    h = hashlib.sha256()
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for f in ("attention_tc.cu", "dequant.cuh", "tc.cuh"):
+            h.update(open(os.path.join(src, f), "rb").read())
     except OSError:
         return None
-    if (h != ATTN_TRAFFIC["sha256_16"] or cfg.name != ATTN_TRAFFIC["config"]
+    if (h.hexdigest()[:16] != ATTN_TRAFFIC["sha256_16"] or cfg.name != ATTN_TRAFFIC["config"]
             or cfg.frames != ATTN_TRAFFIC["frames"]):
         return None
     return ATTN_TRAFFIC["bytes_per_launch"]
