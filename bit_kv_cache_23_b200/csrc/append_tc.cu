@@ -62,7 +62,7 @@ struct Lay {
   static constexpr uint32_t B = ALO + TILE_A;
   static constexpr uint32_t AEXT = B + TILE_B;                     // [128][16] bf16 no swizzle
   static constexpr uint32_t BEXT = AEXT + 128 * 16 * 2;            // [256][16]
-  static constexpr uint32_t SURV = BEXT + NCH * 16 * 2;            // [NT][SURV_MAX] u16
+  static constexpr uint32_t SURV = BEXT + NCH * 16 * 2;            // [SURV_MAX][NT] u16
   static constexpr uint32_t S = SURV + NT * SURV_MAX * 2;          // [128] s
   static constexpr uint32_t W = S + 128 * 4;                       // [8] w
   static constexpr uint32_t U = W + 8 * 4;                         // [128][16] U
@@ -136,23 +136,26 @@ __device__ __forceinline__ void tok_chunk(const uint16_t* krow, int q, float (&k
   }
 }
 
-// Canonical distances of the token to centroids i0 and i1 (two independent
-// channel-order folds interleaved for instruction-level parallelism).
+// Canonical distances of token row r0 to centroid i0 and of row r1 to i1 (two
+// independent channel-order folds interleaved for instruction-level
+// parallelism).
 template <bool KEY>
-__device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t* bt,
-                                            const uint16_t* cent, int C, int i0, int i1,
-                                            const float* s, float& d0, float& d1) {
+__device__ __forceinline__ void canon_dist2x(const uint16_t* r0, const uint16_t* r1,
+                                             const uint8_t* bt, const uint16_t* cent, int C,
+                                             int i0, int i1, const float* s, float& d0,
+                                             float& d1) {
   float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll 2
   for (int q = 0; q < DH / 8; ++q) {
-    float k[8], c0[8], c1[8];
-    tok_chunk(krow, q, k);
+    float k0[8], k1[8], c0[8], c1[8];
+    tok_chunk(r0, q, k0);
+    tok_chunk(r1, q, k1);
     cent_chunk(bt, cent, C, i0, q, c0);
     cent_chunk(bt, cent, C, i1, q, c1);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int j = q * 8 + e;
-      const float l0 = __fsub_rn(k[e], c0[e]), l1 = __fsub_rn(k[e], c1[e]);
+      const float l0 = __fsub_rn(k0[e], c0[e]), l1 = __fsub_rn(k1[e], c1[e]);
       if (KEY) {
         a0 = __fmaf_rn(s[j], __fmul_rn(l0, l0), a0);
         a1 = __fmaf_rn(s[j], __fmul_rn(l1, l1), a1);
@@ -166,6 +169,14 @@ __device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t*
   d1 = a1;
 }
 
+// The same token row against two centroids.
+template <bool KEY>
+__device__ __forceinline__ void canon_dist2(const uint16_t* krow, const uint8_t* bt,
+                                            const uint16_t* cent, int C, int i0, int i1,
+                                            const float* s, float& d0, float& d1) {
+  canon_dist2x<KEY>(krow, krow, bt, cent, C, i0, i1, s, d0, d1);
+}
+
 template <bool KEY, int G, int NT>
 __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   using L = Lay<NT>;
@@ -175,6 +186,10 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR + 8);
   uint16_t* surv = reinterpret_cast<uint16_t*>(smem + L::SURV);
+  // the survivors' approximations [SURV_MAX][NT], in the A tiles, which are
+  // free once the MMAs have completed
+  float* sval = reinterpret_cast<float*>(smem + L::AHI);
+  static_assert(SURV_MAX * NT * 4 <= 2 * L::TILE_A, "survivor values fit the A tiles");
   float* s_s = reinterpret_cast<float*>(smem + L::S);
   float* w_s = reinterpret_cast<float*>(smem + L::W);
   float* U_s = reinterpret_cast<float*>(smem + L::U);
@@ -190,9 +205,11 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   const bool valid = tok < A.n;
   const uint16_t* cent = A.cent + (size_t)h * C * DH;
 
+  int* qcount = reinterpret_cast<int*>(smem + L::BAR + 16);
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
+    *qcount = 0;
   }
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
@@ -408,7 +425,10 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       if (c0 + e < C && v[e] <= theta) {
-        if (cnt < SURV_MAX) surv[tid * SURV_MAX + cnt] = (uint16_t)(c0 + e);
+        if (cnt < SURV_MAX) {
+          surv[cnt * NT + tid] = (uint16_t)(c0 + e);
+          sval[cnt * NT + tid] = v[e];
+        }
         ++cnt;
       }
     }
@@ -429,21 +449,103 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   // top Mc survives); their order by (D, i) is needed only to break a tie of
   // the stage-2 score (or never, for a shortlist of one), so the exact
   // distances are computed later for tied candidates only.
-  const bool exact_set = (cnt == Mc);
+  bool exact_set = (cnt == Mc);
   if (valid && exact_set) {
 #pragma unroll
     for (int m = 0; m < 8; ++m)
-      if (m < Mc) cand[m] = (int)surv[tid * SURV_MAX + m];
-  } else if (valid) {
-    const bool all = cnt > SURV_MAX || cnt < Mc;  // overflow, or no usable approximation
+      if (m < Mc) cand[m] = (int)surv[m * NT + tid];
+  } else if (valid && cnt > Mc && cnt <= SURV_MAX) {
+    // More survivors: the Mc smallest approximations are still the shortlist
+    // when the gap to the next one exceeds what the errors can close.  With
+    // S those Mc, any j outside S has d~_j >= d~(Mc+1) (non-survivors lie
+    // above theta >= d~(Mc+1)), so for i in S the exact values satisfy
+    // D*_j - D*_i >= delta = d~(Mc+1) - d~(Mc) - 2E, and the canonical folds
+    // (relative error gamma) keep D_j > D_i when
+    // delta (1 - gamma) > 2 gamma D*_i, D*_i <= A_t / (1 - gamma) + d~(Mc) + E.
+    float sd[9];
+    int si[9];
+#pragma unroll
+    for (int m = 0; m < 9; ++m) { sd[m] = INFINITY; si[m] = 0x7fffffff; }
+#pragma unroll 1
+    for (int q = 0; q < cnt; ++q) {
+      float xv = sval[q * NT + tid];
+      int xi = (int)surv[q * NT + tid];
+#pragma unroll
+      for (int m = 0; m < 9; ++m) {
+        if (m <= Mc && lex_less(xv, xi, sd[m], si[m])) {
+          const float tv = sd[m];
+          const int ti = si[m];
+          sd[m] = xv;
+          si[m] = xi;
+          xv = tv;
+          xi = ti;
+        }
+      }
+    }
+    float dm = sd[0], dn = sd[1];
+#pragma unroll
+    for (int m = 1; m < 9; ++m) {
+      if (m == Mc - 1) dm = sd[m];
+      if (m == Mc) dn = sd[m];
+    }
+    // 1 + 2 gamma >= 1 / (1 - gamma); the last term covers this test's own rounding
+    const float g2 = 1.0f + 2.0f * gam;
+    const float dhi = fmaxf(At * g2 + dm + E, 0.0f);
+    const float delta = dn - dm - 2.0f * E;
+    const float need = 2.0f * gam * g2 * dhi + 1e-6f * (fabsf(dn) + fabsf(dm) + At + E) + 1e-30f;
+    if (delta > need) {
+      exact_set = true;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (m < Mc) cand[m] = si[m];
+    }
+  }
+  // The remaining tokens' survivors are rescored as one queue of (token,
+  // centroid) pairs that every thread of the CTA shares (two pairs per thread
+  // at a time), so that a few such tokens do not hold up their whole warps;
+  // the owner then ranks its own results.  A token whose survivors overflowed
+  // the list, or with fewer than Mc, rescores all C centroids itself.
+  const bool all = valid && !exact_set && (cnt > SURV_MAX || cnt < Mc);
+  const bool queued = valid && !exact_set && !all;
+  int qbase = 0;
+  uint32_t* qent = reinterpret_cast<uint32_t*>(smem + L::ALO);     // [NT * SURV_MAX]
+  float* qd = reinterpret_cast<float*>(smem + L::ALO) + NT * SURV_MAX;
+  static_assert(NT * SURV_MAX * 8 <= L::TILE_A, "the rescoring queue fits one A tile");
+  if (queued) {
+    qbase = atomicAdd(qcount, cnt);
+    for (int q = 0; q < cnt; ++q) qent[qbase + q] = ((uint32_t)tid << 16) | surv[q * NT + tid];
+  }
+  __syncthreads();
+  const int qn = *qcount;
+#pragma unroll 1
+  for (int e0 = tid; e0 < qn; e0 += 2 * NT) {
+    const int e1 = e0 + NT < qn ? e0 + NT : e0;
+    const uint32_t x0 = qent[e0], x1 = qent[e1];
+    const uint16_t* r0 = reinterpret_cast<const uint16_t*>(smem + L::KR) + (x0 >> 16) * KROW;
+    const uint16_t* r1 = reinterpret_cast<const uint16_t*>(smem + L::KR) + (x1 >> 16) * KROW;
+    float D0, D1;
+    canon_dist2x<KEY>(r0, r1, bt, cent, C, (int)(x0 & 0xffffu), (int)(x1 & 0xffffu), s_s, D0, D1);
+    qd[e0] = D0;
+    qd[e1] = D1;
+  }
+  __syncthreads();
+  if (queued || all) {
     const int nloop = all ? C : cnt;
 #pragma unroll 1
     for (int q = 0; q < nloop; q += 2) {
-      const int i0 = all ? q : (int)surv[tid * SURV_MAX + q];
       const bool two = q + 1 < nloop;
-      const int i1 = two ? (all ? q + 1 : (int)surv[tid * SURV_MAX + q + 1]) : i0;
+      int i0, i1;
       float D0, D1;
-      canon_dist2<KEY>(krow, bt, cent, C, i0, i1, s_s, D0, D1);
+      if (all) {
+        i0 = q;
+        i1 = two ? q + 1 : q;
+        canon_dist2<KEY>(krow, bt, cent, C, i0, i1, s_s, D0, D1);
+      } else {
+        i0 = (int)surv[q * NT + tid];
+        i1 = two ? (int)surv[(q + 1) * NT + tid] : i0;
+        D0 = qd[qbase + q];
+        D1 = two ? qd[qbase + q + 1] : D0;
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         if (u == 1 && !two) break;
@@ -468,10 +570,15 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
       }
     }
   }
-  if (!valid) return;
-
   constexpr int NG = DH / G;     // groups per row
   constexpr int QG = G / 8;      // 8-channel chunks per group
+  // Code words, group parameters and INT8 coefficients are staged per token in
+  // the A tiles (free again) and written to the cache with coalesced 16-byte
+  // stores once the whole CTA has encoded its tokens.
+  constexpr uint32_t SO_PAR = NT * (DH / 4), SO_COEF = SO_PAR + NT * NG * 4;
+  static_assert(SO_COEF + NT * 16 <= 2 * L::TILE_A, "staged outputs fit the A tiles");
+  uint8_t* so = smem + L::AHI;
+  if (valid) {
 
   // ---- P6: QSAC stage 2 (keys): expected squared logit perturbation
   int a = cand[0];
@@ -543,8 +650,8 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
 
   // ---- P7: INT2 residual and PSAC coefficients, group by group in channel order
   const size_t slot = (size_t)h * A.tcap + (size_t)(A.t0 + tok);
-  uint16_t* codew = reinterpret_cast<uint16_t*>(A.codes + slot * (DH / 4));
-  uint32_t* pdst = reinterpret_cast<uint32_t*>(A.params) + slot * NG;
+  uint16_t* codew = reinterpret_cast<uint16_t*>(so + tid * (DH / 4));
+  uint32_t* pdst = reinterpret_cast<uint32_t*>(so + SO_PAR) + tid * NG;
   float cq[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) cq[i] = 0.0f;
@@ -628,10 +735,35 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
           q8 = __float2int_rn(__fdiv_rn(cq[i], cs));
           q8 = max(-127, min(127, q8));
         }
-        A.coef[slot * r + i] = (int8_t)q8;
+        so[SO_COEF + tid * r + i] = (uint8_t)(int8_t)q8;
       }
     }
     A.cscale[slot] = csh;
+  }
+  }  // valid
+  __syncthreads();
+  // the CTA's tokens are contiguous in every field: copy the staged rows out
+  const int64_t tok0 = (int64_t)blockIdx.x * NT;
+  const int nv = (int)(A.n - tok0 < NT ? A.n - tok0 : NT);
+  const size_t slot0 = (size_t)h * A.tcap + (size_t)(A.t0 + tok0);
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(so);
+    uint4* dst = reinterpret_cast<uint4*>(A.codes + slot0 * (DH / 4));
+    for (int u = tid; u < nv * (DH / 64); u += NT) dst[u] = src[u];
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(so + SO_PAR);
+    uint4* dst = reinterpret_cast<uint4*>(A.params + slot0 * NG * 2);
+    for (int u = tid; u < nv * (NG / 4); u += NT) dst[u] = src[u];
+  }
+  if (KEY && r > 0) {
+    if ((r & 7) == 0) {
+      const uint2* src = reinterpret_cast<const uint2*>(so + SO_COEF);
+      uint2* dst = reinterpret_cast<uint2*>(A.coef + slot0 * r);
+      for (int u = tid; u < nv * (r / 8); u += NT) dst[u] = src[u];
+    } else {
+      for (int u = tid; u < nv * r; u += NT) A.coef[slot0 * r + u] = (int8_t)so[SO_COEF + u];
+    }
   }
 }
 
