@@ -144,7 +144,9 @@ __device__ __forceinline__ void canon_dist2x(const uint16_t* r0, const uint16_t*
                                              const uint8_t* bt, const uint16_t* cent, int C,
                                              int i0, int i1, const float* s, float& d0,
                                              float& d1) {
-  float a0 = 0.0f, a1 = 0.0f;
+  // the two folds as the lanes of f32x2 operations (each lane rounds exactly as
+  // the scalar operation would)
+  uint64_t acc = 0ull;
 #pragma unroll 2
   for (int q = 0; q < DH / 8; ++q) {
     float k0[8], k1[8], c0[8], c1[8];
@@ -155,18 +157,12 @@ __device__ __forceinline__ void canon_dist2x(const uint16_t* r0, const uint16_t*
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int j = q * 8 + e;
-      const float l0 = __fsub_rn(k0[e], c0[e]), l1 = __fsub_rn(k1[e], c1[e]);
-      if (KEY) {
-        a0 = __fmaf_rn(s[j], __fmul_rn(l0, l0), a0);
-        a1 = __fmaf_rn(s[j], __fmul_rn(l1, l1), a1);
-      } else {
-        a0 = __fmaf_rn(l0, l0, a0);
-        a1 = __fmaf_rn(l1, l1, a1);
-      }
+      const uint64_t l = fsub2(f2pack(k0[e], k1[e]), f2pack(c0[e], c1[e]));
+      if (KEY) acc = ffma2(f2pack(s[j], s[j]), fmul2(l, l), acc);
+      else acc = ffma2(l, l, acc);
     }
   }
-  d0 = a0;
-  d1 = a1;
+  f2unpack(acc, d0, d1);
 }
 
 // The same token row against two centroids.
@@ -655,6 +651,7 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
   float cq[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) cq[i] = 0.0f;
+  uint64_t cq2[4] = {0ull, 0ull, 0ull, 0ull};  // r == 8: coefficient pairs (2i, 2i + 1)
 #pragma unroll 1
   for (int g = 0; g < NG; ++g) {
     float lo = 0.0f, hi = 0.0f;
@@ -696,14 +693,11 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
           if (r == 8) {
             const float4 u0 = *reinterpret_cast<const float4*>(Uj);
             const float4 u1 = *reinterpret_cast<const float4*>(Uj + 4);
-            cq[0] = __fmaf_rn(u0.x, ej, cq[0]);
-            cq[1] = __fmaf_rn(u0.y, ej, cq[1]);
-            cq[2] = __fmaf_rn(u0.z, ej, cq[2]);
-            cq[3] = __fmaf_rn(u0.w, ej, cq[3]);
-            cq[4] = __fmaf_rn(u1.x, ej, cq[4]);
-            cq[5] = __fmaf_rn(u1.y, ej, cq[5]);
-            cq[6] = __fmaf_rn(u1.z, ej, cq[6]);
-            cq[7] = __fmaf_rn(u1.w, ej, cq[7]);
+            const uint64_t e2 = f2pack(ej, ej);
+            cq2[0] = ffma2(f2pack(u0.x, u0.y), e2, cq2[0]);
+            cq2[1] = ffma2(f2pack(u0.z, u0.w), e2, cq2[1]);
+            cq2[2] = ffma2(f2pack(u1.x, u1.y), e2, cq2[2]);
+            cq2[3] = ffma2(f2pack(u1.z, u1.w), e2, cq2[3]);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -720,6 +714,10 @@ __device__ __forceinline__ void append_tc_body(const ApArgs& A) {
     if (h == 0) {
       A.tokver[A.t0 + tok] = (uint16_t)A.version;
       A.centver[A.t0 + tok] = (uint16_t)A.cver;
+    }
+    if (r == 8) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f2unpack(cq2[q], cq[2 * q], cq[2 * q + 1]);
     }
     float amax = 0.0f;
 #pragma unroll
