@@ -184,6 +184,25 @@ def attention_splits(cfg, heads: int, device) -> bool:
 
 
 # ----------------------------------------------------------------------------- workload
+def packed_bytes_per_token_head(c: syn.LayerConfig) -> int:
+    """Stored bytes of one token of one head: K and V codes, group parameters and
+    centroid index, plus the Key's INT8 coefficients and their fp16 scale."""
+    idx = 1 if c.n_centroids <= 256 else 2
+    return 2 * (c.head_dim // 4 + 4 * (c.head_dim // c.group) + idx) + c.rank + 2
+
+
+def config_dict(c: syn.LayerConfig, workload_name: str, world: int, shard_mode: str,
+                nh: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    cache = c.total_tokens * nh * packed_bytes_per_token_head(c)
+    return {"workload": workload_name,
+            "l2": (f"packed cache of {cache / 1e6:.0f} MB read per step "
+                   f"({'larger' if cache > 126e6 else 'smaller'} than "
+                   "the 126 MB L2), step inputs rotate over 4 HBM-resident frames"),
+            "parallelism": (f"heads split over {world} ranks ({nh} on rank 0)"
+                            if shard_mode == "heads" else f"replicas x{world}")}
+
+
 def dev_bf16(a: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
 
@@ -603,7 +622,12 @@ def main():
             "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": len(runs), "warmup": 0, "ms_per_step": 1e3 * cfg.q_rows / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": {"workload": workload_name},
+            "data": "synthetic",
+            # rank 0's heads under --shard heads: the first heads % world ranks
+            # hold one more (the partition the ours arm uses)
+            "config": config_dict(cfg, workload_name, world, args.shard,
+                                  cfg.heads if args.shard != "heads"
+                                  else -(-cfg.heads // world)),
             "cpu_baseline": {"kind": "oracle", "cores": r0["cores"], "host_cores": r0["host_cores"],
                              "cpu_model": r0["cpu_model"], "sample": r0["note"], "value": v,
                              "unit": UNIT, "single_thread": statistics.median(
@@ -702,7 +726,7 @@ def main():
     # per launch on this rank (its heads)
     att_flop = 4.0 * c.q_rows * T * c.head_dim * nh
     att_tflops = att_flop / (att_ms * 1e-3) / 1e12
-    per_tok = 2 * (c.head_dim // 4 + 4 * (c.head_dim // c.group) + (1 if c.n_centroids <= 256 else 2)) + c.rank + 2
+    per_tok = packed_bytes_per_token_head(c)
     app_bytes = c.tokens_per_frame * nh * (4 * c.head_dim + per_tok)
     app_gbs = app_bytes / (app_ms * 1e-3) / 1e9
     # fixed bytes: every centroid-table version in use and every basis version
@@ -724,12 +748,7 @@ def main():
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_name,
-                   "l2": (f"packed cache of {T * nh * per_tok / 1e6:.0f} MB read per step "
-                          f"({'larger' if T * nh * per_tok > 126e6 else 'smaller'} than "
-                          "the 126 MB L2), step inputs rotate over 4 HBM-resident frames"),
-                   "parallelism": (f"heads split over {world} ranks ({nh} on rank 0)"
-                                   if args.shard == "heads" else f"replicas x{world}")},
+        "config": config_dict(c, workload_name, world, args.shard, nh),
         "gpu_launches": n_launches,
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16"],
                      "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
