@@ -142,7 +142,7 @@ class ClockSampler:
 # tables) and 147.5 MB written (the split key ranges' fp32 partials, which the
 # merge kernel reads back, and O).  Valid only for the kernel sources it was
 # taken on (hash of attention_tc.cu, dequant.cuh and tc.cuh below).
-ATTN_TRAFFIC = {"sha256_16": "ced8e64a298ce612", "config": "480p", "frames": 24,
+ATTN_TRAFFIC = {"sha256_16": "b194f56ffdbd9d07", "config": "480p", "frames": 24,
                 "bytes_per_launch": 187332864 + 147464448}
 
 
