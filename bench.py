@@ -621,7 +621,7 @@ def main():
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": len(runs), "warmup": 0, "ms_per_step": 1e3 * cfg.q_rows / v,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             # rank 0's heads under --shard heads: the first heads % world ranks
             # hold one more (the partition the ours arm uses)
